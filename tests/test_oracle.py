@@ -1,0 +1,293 @@
+"""Pins for the CPU oracle against things other than itself.
+
+Each test ties one part of the oracle to a fact fixed outside it: the IEEE binary16 definition
+(exhaustively, against numpy's decoder), hand-derived fixtures under tests/golden/ for the Q4_K
+scale table, nibble order and dequantization (GGML Q4_K / Q8_0 layouts, as the T4 dossier's
+"QUANTIZATION MIX" names them), closed forms (all-zero q gives -dmin*m*sum(x)), exact integer
+special cases, linearity, and brute force against a numpy fp64 matmul on tiny shapes.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from conftest import read_golden
+from quant_dequant_gemv_q4_b200 import synth
+
+Q4_K, Q8_0 = 12, 8
+
+
+def _hexbytes(tokens):
+    return np.array([int(t, 16) for t in tokens], dtype=np.uint8)
+
+
+def _q4k_block(d_bits, dmin_bits, scales, qs):
+    blk = np.zeros(144, np.uint8)
+    blk[0:2] = np.array([d_bits & 0xFF, d_bits >> 8], np.uint8)
+    blk[2:4] = np.array([dmin_bits & 0xFF, dmin_bits >> 8], np.uint8)
+    blk[4:16] = scales
+    blk[16:144] = qs
+    return blk
+
+
+# --- fp16 decoding -----------------------------------------------------------------------------
+
+def test_fp16_exhaustive_matches_numpy(orc):
+    """All 65536 binary16 patterns decode to numpy's float16 -> float64 value (NaN to NaN)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([orc.half_to_double(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zeros keep their sign
+    assert math.copysign(1.0, orc.half_to_double(0x8000)) == -1.0
+
+
+def test_fp16_textbook_values(orc):
+    for bits_s, val_s in read_golden("fp16_values.txt")["_rows"]:
+        got = orc.half_to_double(int(bits_s, 16))
+        want = float(val_s)
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), (bits_s, got, want)
+
+
+# --- Q4_K scale table ---------------------------------------------------------------------------
+
+def test_scale_table_golden(orc):
+    g = read_golden("q4k_scale_table.txt")
+    scales = _hexbytes(g["scales"][0])
+    sc = [int(v) for v in g["sc"][0]]
+    m = [int(v) for v in g["m"][0]]
+    for j in range(8):
+        assert orc.q4k_scale_min(scales, j) == (sc[j], m[j]), j
+
+
+def test_scale_table_is_a_bit_permutation(orc):
+    """Each of the 96 table bits drives exactly one bit of one 6-bit value, and every value bit is
+    driven by exactly one table bit: the packing is one-to-one, so uniform random table bytes are
+    uniform independent (sc_j, m_j) pairs."""
+    seen = set()
+    zero = np.zeros(12, np.uint8)
+    for j in range(8):
+        assert orc.q4k_scale_min(zero, j) == (0, 0)
+    for byte in range(12):
+        for bit in range(8):
+            s = zero.copy()
+            s[byte] = 1 << bit
+            hits = []
+            for j in range(8):
+                sc, m = orc.q4k_scale_min(s, j)
+                if sc:
+                    hits.append(("sc", j, sc))
+                if m:
+                    hits.append(("m", j, m))
+            assert len(hits) == 1, (byte, bit, hits)
+            kind, j, val = hits[0]
+            assert val & (val - 1) == 0  # a single bit
+            key = (kind, j, val.bit_length() - 1)
+            assert key not in seen
+            seen.add(key)
+    assert len(seen) == 96
+
+
+def test_scale_table_linear_in_bytes(orc):
+    """Values of a table equal the sum of the values of its individual bits (random tables)."""
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        s = rng.integers(0, 256, 12, dtype=np.uint8)
+        tot = np.zeros((8, 2), int)
+        for byte in range(12):
+            for bit in range(8):
+                if s[byte] >> bit & 1:
+                    one = np.zeros(12, np.uint8)
+                    one[byte] = 1 << bit
+                    tot += np.array([orc.q4k_scale_min(one, j) for j in range(8)])
+        assert np.array_equal(tot, np.array([orc.q4k_scale_min(s, j) for j in range(8)]))
+
+
+# --- Q4_K dequantization ------------------------------------------------------------------------
+
+def _golden_superblock():
+    g = read_golden("q4k_superblock.txt")
+    qs = np.zeros(128, np.uint8)
+    for c in range(4):
+        for l in range(32):
+            qs[32 * c + l] = (l & 15) | (((l + c) & 15) << 4)
+    blk = _q4k_block(int(g["d"][0][0], 16), int(g["dmin"][0][0], 16), _hexbytes(g["scales"][0]), qs)
+    return blk, g
+
+
+def test_q4k_superblock_golden(orc):
+    blk, g = _golden_superblock()
+    w = orc.dequant(blk, Q4_K, 1, 256)[0]
+    for idx, val in g["w"]:
+        assert w[int(idx)] == np.float32(float(val)), (idx, w[int(idx)], val)
+    x = np.ones((256, 1), np.float16)
+    y, A = orc.gemv(blk, Q4_K, 1, 256, x, 1)
+    assert y[0, 0] == float(g["y_ones"][0][0])
+    assert A[0, 0] == np.abs(w.astype(np.float64)).sum()
+
+
+def test_q4k_nibble_order_identity(orc):
+    """d=1, dmin=0, every sc=1, q_i = i mod 16  =>  w_i = i mod 16."""
+    scales = np.array([1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1], np.uint8)  # sc_j = 1, m_j = 0
+    qs = np.array([(l % 16) * 0x11 for c in range(4) for l in range(32)], np.uint8)
+    blk = _q4k_block(0x3C00, 0x0000, scales, qs)
+    w = orc.dequant(blk, Q4_K, 1, 256)[0]
+    assert np.array_equal(w, (np.arange(256) % 16).astype(np.float32))
+
+
+def test_q4k_distinct_scales_per_subblock(orc):
+    """sc_j = j+1, m=0, d=1, q_i = i mod 16  =>  w_i = (i//32 + 1) * (i mod 16)."""
+    scales = np.array([1, 2, 3, 4, 0, 0, 0, 0, 5, 6, 7, 8], np.uint8)
+    qs = np.array([(l % 16) * 0x11 for c in range(4) for l in range(32)], np.uint8)
+    blk = _q4k_block(0x3C00, 0x0000, scales, qs)
+    w = orc.dequant(blk, Q4_K, 1, 256)[0]
+    i = np.arange(256)
+    assert np.array_equal(w, ((i // 32 + 1) * (i % 16)).astype(np.float32))
+
+
+def test_q4k_high_nibbles_are_second_half_of_chunk(orc):
+    """qs = 0xF0 everywhere (low nibble 0, high 15), d=1, dmin=0, sc=1: weights 64c..64c+31 are 0
+    and 64c+32..64c+63 are 15."""
+    scales = np.array([1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1], np.uint8)
+    blk = _q4k_block(0x3C00, 0, scales, np.full(128, 0xF0, np.uint8))
+    w = orc.dequant(blk, Q4_K, 1, 256)[0]
+    want = np.where((np.arange(256) % 64) < 32, 0, 15).astype(np.float32)
+    assert np.array_equal(w, want)
+
+
+def test_q4k_min_term_closed_form(orc):
+    """All-zero q: w = -dmin*m_j, so y = -dmin * sum_j m_j * X_j with X_j = sum of x over
+    sub-block j (for each superblock), here with random d, dmin, table and x."""
+    rng = np.random.default_rng(11)
+    N, K, B = 3, 512, 2
+    W = synth.q4k_weights(N, K, seed=7).reshape(-1, 144).copy()
+    W[:, 16:] = 0
+    W = W.reshape(-1)
+    x = rng.standard_normal((K, B)).astype(np.float16)
+    y, _ = orc.gemv(W, Q4_K, N, K, x, B)
+    blocks = W.reshape(N, K // 256, 144)
+    xd = x.astype(np.float64)
+    for n in range(N):
+        for b in range(B):
+            want = 0.0
+            for s in range(K // 256):
+                dmin = blocks[n, s, 2:4].view(np.float16)[0].astype(np.float64)
+                for j in range(8):
+                    _, m = orc.q4k_scale_min(blocks[n, s, 4:16], j)
+                    Xj = xd[256 * s + 32 * j: 256 * s + 32 * j + 32, b].sum()
+                    want -= float(np.float32(dmin * m)) * Xj
+            assert y[n, b] == pytest.approx(want, rel=1e-12, abs=1e-15)
+
+
+def test_q4k_exact_integer_case(orc):
+    """d = 2^-10, dmin = 2^-12 and integer x in [-2, 2]: every w is a multiple of 2^-12, so
+    y * 2^12 = sum_k (4*sc*q - m) * x exactly, an integer computed here from raw bytes."""
+    rng = np.random.default_rng(3)
+    N, K, B = 4, 512, 3
+    W = synth.q4k_weights(N, K, seed=9).reshape(-1, 144).copy()
+    W[:, 0:2] = np.array([0x00, 0x14], np.uint8)  # 2^-10 = fp16 0x1400
+    W[:, 2:4] = np.array([0x00, 0x0C], np.uint8)  # 2^-12 = fp16 0x0C00
+    W = W.reshape(-1)
+    x = rng.integers(-2, 3, size=(K, B)).astype(np.float16)
+    y, _ = orc.gemv(W, Q4_K, N, K, x, B)
+    f = orc.unpack_q4k(W, N * K // 256)
+    q = f["q"].reshape(N, K).astype(np.int64)
+    sc = np.repeat(f["sc"].reshape(N, K // 32), 32, axis=1).astype(np.int64)
+    m = np.repeat(f["m"].reshape(N, K // 32), 32, axis=1).astype(np.int64)
+    wint = 4 * sc * q - m
+    want = wint @ x.astype(np.int64)
+    assert np.array_equal(y * 4096.0, want.astype(np.float64))
+
+
+# --- Q8_0 ----------------------------------------------------------------------------------------
+
+def test_q8_0_golden(orc):
+    g = read_golden("q8_0_block.txt")
+    q = np.arange(32, dtype=np.int64) - 16
+    for i, v in g["q"]:
+        q[int(i)] = int(v)
+    blk = np.zeros(34, np.uint8)
+    d = int(g["d"][0][0], 16)
+    blk[0:2] = [d & 0xFF, d >> 8]
+    blk[2:] = q.astype(np.int8).view(np.uint8)
+    w = orc.dequant(blk, Q8_0, 1, 32)[0]
+    for i, v in g["w"]:
+        assert w[int(i)] == np.float32(float(v))
+
+
+def test_q8_0_exact_integer_case(orc):
+    """d = 1 and integer x with |x| <= 16: y = sum q*x exactly, computed from the raw bytes."""
+    rng = np.random.default_rng(4)
+    N, K, B = 5, 320, 2
+    W = synth.q8_0_weights(N, K, seed=1).reshape(-1, 34).copy()
+    W[:, 0:2] = np.array([0x00, 0x3C], np.uint8)
+    q = W[:, 2:].view(np.int8).astype(np.int64).reshape(N, K)
+    x = rng.integers(-16, 17, size=(K, B)).astype(np.float16)
+    y, A = orc.gemv(W.reshape(-1), Q8_0, N, K, x, B)
+    assert np.array_equal(y, (q @ x.astype(np.int64)).astype(np.float64))
+    assert np.array_equal(A, (np.abs(q) @ np.abs(x.astype(np.int64))).astype(np.float64))
+
+
+# --- the GEMV as a whole ------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0])
+@pytest.mark.parametrize("N,K", [(1, 256), (2, 512), (3, 256), (3, 512)])
+def test_brute_force_tiny(orc, fmt, N, K):
+    """Oracle y and A equal a numpy fp64 matmul of the dequantized matrix, for B = 1..8."""
+    W = synth.weights(fmt, N, K, seed=N * 1000 + K)
+    Wf = orc.dequant(W, fmt, N, K).astype(np.float64)
+    for B in range(1, 9):
+        x = synth.activations(K, B, seed=B)
+        y, A = orc.gemv(W, fmt, N, K, x, B)
+        xd = x.astype(np.float64)
+        np.testing.assert_allclose(y, Wf @ xd, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(A, np.abs(Wf) @ np.abs(xd), rtol=1e-13, atol=0)
+
+
+def test_rows_subset_matches_full(orc):
+    N, K, B = 7, 512, 3
+    W = synth.q4k_weights(N, K, seed=2)
+    x = synth.activations(K, B, seed=2)
+    y, A = orc.gemv(W, Q4_K, N, K, x, B)
+    rows = np.array([6, 0, 3])
+    ys, As = orc.gemv(W, Q4_K, N, K, x, B, rows=rows)
+    assert np.array_equal(ys, y[rows]) and np.array_equal(As, A[rows])
+
+
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0])
+def test_linearity(orc, fmt):
+    """y(2x) = 2 y(x) and y(x/8) = y(x)/8 exactly (power-of-two scalings are exact in fp16 for
+    these magnitudes); y(x1) + y(x2) = y(x1 + x2) for x1, x2 with disjoint supports."""
+    N, K = 4, 1024
+    W = synth.weights(fmt, N, K, seed=21)
+    x = synth.activations(K, 2, seed=21)
+    # keep |x| >= 2^-10 so that x/8 stays a normal fp16 number (exactly representable)
+    x = np.where(np.abs(x.astype(np.float32)) < 2.0 ** -10, np.float16(0.5), x)
+    y, _ = orc.gemv(W, fmt, N, K, x, 2)
+    y2, _ = orc.gemv(W, fmt, N, K, (x.astype(np.float32) * 2).astype(np.float16), 2)
+    y8, _ = orc.gemv(W, fmt, N, K, (x.astype(np.float32) / 8).astype(np.float16), 2)
+    assert np.array_equal(y2, 2 * y) and np.array_equal(y8, y / 8)
+    mask = (np.arange(K) % 3 == 0)[:, None]
+    x1 = np.where(mask, x, np.float16(0))
+    x2 = np.where(mask, np.float16(0), x)
+    ya, _ = orc.gemv(W, fmt, N, K, x1, 2)
+    yb, _ = orc.gemv(W, fmt, N, K, x2, 2)
+    np.testing.assert_allclose(ya + yb, y, rtol=1e-12, atol=1e-12)
+
+
+def test_weight_bytes(orc):
+    assert orc.weight_bytes(Q4_K, 17408, 5120) == 50_135_040
+    assert orc.weight_bytes(Q4_K, 5120, 17408) == 50_135_040
+    assert orc.weight_bytes(Q8_0, 12288, 5120) == 66_846_720
+    assert orc.weight_bytes(Q4_K, 1024, 5120) == 2_949_120
+    assert orc.weight_bytes(Q4_K, 10, 300) == 0
+    assert orc.weight_bytes(99, 10, 256) == 0
+
+
+def test_invalid_arguments_raise(orc):
+    W = synth.q4k_weights(1, 256, seed=0)
+    x = synth.activations(256, 1, seed=0)
+    with pytest.raises(ValueError):
+        orc.gemv(W, Q4_K, 1, 256, x, 1, rows=np.array([1]))
