@@ -1,0 +1,566 @@
+"""Benchmark of the Q4_K / Q8_0 dequant GEMV on B200 (one JSON line on stdout, rank 0).
+
+Headline (value): effective HBM GB/s of one Q4_K GEMV y = dequant(W) . x at B = 1 on the FFN gate
+shape N=17408, K=5120 of a 27B-class hybrid decoder (weight + x + y bytes / time).  A step is one
+such call; the weights rotate over enough distinct device copies that every step reads them from
+HBM (the copies together exceed 4x the L2).  Steps are replayed from CUDA graphs and timed with
+CUDA events on the launching stream.  The same line carries B = 8 on the same tensor, every other
+workload of the suite (per call: us, GB/s, fraction of the measured HBM copy bandwidth), the
+end-to-end number through the Python API with host buffers, the roofline of the kernel, clocks
+sampled during the timed region, and the CPU oracle's throughput on a bounded sample.
+
+--impl reference times the CPU oracle (the plain C dequant + fp64 dot) instead, on the same
+metric and workload, each step a bounded sample of rows.
+
+Multi-GPU: the GEMV does not shard across GPUs here (replicas only): each rank runs its own copy
+of the workload, the timed region is bracketed by barriers, its time is the max over ranks and
+value = all ranks' bytes / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from quant_dequant_gemv_q4_b200 import synth  # noqa: E402
+
+METRIC = "Q4_K GEMV effective HBM GB/s and % of B200 HBM roofline (us/call), B=1 and B=8"
+UNIT = "GB/s"
+HEADLINE = synth.Gemv("ffn_gate", synth.Q4_K, 17408, 5120, 1, 0)
+HEADLINE_B8 = synth.Gemv("ffn_gate_b8", synth.Q4_K, 17408, 5120, 8, 0)
+HEADLINE_SEED = 4  # the batched-verify workload's seed
+FALLBACK_HBM_GBS = 6650.0
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("qg_device.cuh", "qg_api.cu"):
+        with open(os.path.join(ROOT, "quant_dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured", "raw": d}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback", "raw": None}
+
+
+# ------------------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ------------------------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_max(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def aggregate(local_seconds: float, local_bytes: float, device) -> tuple[float, float]:
+    """(max seconds over ranks, total bytes over ranks): a replica job's time and work."""
+    return dist_max(local_seconds, device), dist_sum(local_bytes, device)
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="qg_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        maxp = max(r[2] for r in rows)
+        loaded = [r for r in rows if r[2] >= 0.5 * maxp] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in loaded:
+            for name, flag in zip(names, r[3][1:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": maxp,
+                "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU measurement
+# ------------------------------------------------------------------------------------------------
+class CallSet:
+    """Device inputs of a list of GEMV calls, replicated over R copies of the weights."""
+
+    def __init__(self, calls, seed, device, l2_bytes, min_copies=2, max_copies=4096):
+        import torch
+        import quant_dequant_gemv_q4_b200 as qg
+        self.qg = qg
+        self.calls = list(calls)
+        self.device = device
+        wl = synth.Workload("bench", seed, tuple(self.calls))
+        per_step = sum(c.weight_bytes for c in self.calls)
+        self.copies = int(min(max_copies, max(min_copies, -(-4 * l2_bytes // per_step))))
+        self.W, self.x, self.y, self.x_host = [], [], [], []
+        for c in self.calls:
+            W, x = wl.inputs(c)
+            base = torch.from_numpy(W).to(device)
+            self.W.append([base] + [base.clone() for _ in range(self.copies - 1)])
+            self.x_host.append(x)
+            self.x.append(torch.from_numpy(x.view(np.uint16)).to(device))
+            self.y.append(torch.empty((c.N, c.B), dtype=torch.float32, device=device))
+        self.bytes_per_step = sum(c.algorithmic_bytes for c in self.calls)
+        self.weight_bytes_per_step = per_step
+
+    def launch(self, r: int, stream, variant: int):
+        for i, c in enumerate(self.calls):
+            self.qg.qg_gemv_variant(self.W[i][r], c.fmt, c.N, c.K, self.x[i], c.B, self.y[i],
+                                    stream, variant)
+
+    def launches_per_step(self, variant: int) -> int:
+        """Kernels one step launches (a split-K call adds its second pass)."""
+        import torch
+        n = 0
+        for i, c in enumerate(self.calls):
+            self.qg.qg_gemv_variant(self.W[i][0], c.fmt, c.N, c.K, self.x[i], c.B, self.y[i],
+                                    torch.cuda.current_stream(), variant)
+            n += 2 if self.qg.qg_last_splits() > 1 else 1
+        torch.cuda.synchronize()
+        return n
+
+
+def time_callset(cs: CallSet, steps: int, warmup: int, variant: int, clocks: ClockSampler | None):
+    """Time exactly `steps` steps (each: the call list on the next weight copy) replayed from CUDA
+    graphs; returns (seconds on this rank, per-step ms, kernels per step)."""
+    import torch
+    stream = torch.cuda.Stream(device=cs.device)
+    R = cs.copies
+    with torch.cuda.stream(stream):
+        for r in range(min(R, 2)):
+            cs.launch(r, stream, variant)  # allocates the workspace of this stream
+    stream.synchronize()
+    g_full = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_full, stream=stream):
+        for r in range(R):
+            cs.launch(r, stream, variant)
+    rem = steps % R
+    g_rem = None
+    if rem:
+        g_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rem, stream=stream):
+            for r in range(rem):
+                cs.launch(r, stream, variant)
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-warmup // R))):
+            g_full.replay()
+    stream.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    ctx = clocks if clocks is not None else _null()
+    with ctx:
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps // R):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            end.record(stream)
+        end.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+    secs = start.elapsed_time(end) / 1e3
+    del g_full, g_rem
+    return secs, secs * 1e3 / steps
+
+
+class _null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def time_e2e(cs: CallSet, steps: int, warmup: int, variant: int):
+    """End to end through the public Python API: per step, pinned host x -> device, qg_gemv,
+    y -> pinned host; returns (seconds, h2d bytes/step, d2h bytes/step)."""
+    import torch
+    xh = [torch.from_numpy(x.view(np.uint16)).pin_memory() for x in cs.x_host]
+    yh = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in cs.y]
+    stream = torch.cuda.current_stream()
+
+    def step(r):
+        for i, c in enumerate(cs.calls):
+            cs.x[i].copy_(xh[i], non_blocking=True)
+            cs.qg.qg_gemv_variant(cs.W[i][r], c.fmt, c.N, c.K, cs.x[i], c.B, cs.y[i], stream,
+                                  variant)
+            yh[i].copy_(cs.y[i], non_blocking=True)
+
+    for s in range(warmup):
+        step(s % cs.copies)
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.perf_counter()
+    for s in range(steps):
+        step(s % cs.copies)
+    torch.cuda.synchronize()
+    secs = time.perf_counter() - t0
+    barrier()
+    h2d = sum(x.nbytes for x in cs.x_host)
+    d2h = sum(c.N * c.B * 4 for c in cs.calls)
+    return secs, h2d, d2h
+
+
+def hbm_probe(device, nbytes=1 << 30, reps=10):
+    """Copy (read+write) and read-only bandwidth of this library's probe kernels, best of reps."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    src = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    out = torch.zeros(4096, dtype=torch.int32, device=device)
+    s = torch.cuda.current_stream()
+    res = {}
+    for name, fn, moved in [("copy", lambda: qg.qg_hbm_copy(src, dst, nbytes, s), 2 * nbytes),
+                            ("read", lambda: qg.qg_hbm_read(src, nbytes, out, s), nbytes)]:
+        fn()
+        torch.cuda.synchronize()
+        best = 1e9
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            best = min(best, a.elapsed_time(b) / 1e3)
+        res[name + "_gbs"] = round(moved / best / 1e9, 1)
+    del src, dst
+    torch.cuda.empty_cache()
+    return res
+
+
+def load_traffic(kernel_hash: str) -> dict | None:
+    """DRAM bytes per launch from a committed ncu capture summary, if it was taken on the current
+    kernel sources (same hash); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_hash") != kernel_hash:
+        return None
+    return d
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ------------------------------------------------------------------------------------------------
+def oracle_sample_rate(call: synth.Gemv, seed: int, seconds: float, rows_cap=None):
+    """Time the oracle on a bounded row sample of `call` for about `seconds`; returns
+    (GB/s on the call's algorithmic bytes per row, rows timed, seconds, bytes)."""
+    import oracle
+    oracle.build()
+    wl = synth.Workload("cpu", seed, (call,))
+    W, x = wl.inputs(call)
+    row_bytes = call.weight_bytes // call.N
+    rows, done_rows, t_total = 8, 0, 0.0
+    while t_total < seconds and done_rows < (rows_cap or call.N):
+        r0 = done_rows % call.N
+        sel = (np.arange(rows) + r0) % call.N
+        t0 = time.perf_counter()
+        oracle.gemv(W, call.fmt, call.N, call.K, x, call.B, rows=sel)
+        t_total += time.perf_counter() - t0
+        done_rows += rows
+        rows = min(rows * 2, 4096)
+    nbytes = done_rows * (row_bytes + 4 * call.B) + 2 * call.K * call.B
+    return nbytes / t_total / 1e9, done_rows, t_total, nbytes
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    call = HEADLINE
+    wl = synth.Workload("ref", HEADLINE_SEED, (call,))
+    W, x = wl.inputs(call)
+    row_bytes = call.weight_bytes // call.N
+    # rows per step so that warmup + steps take about a minute
+    t0 = time.perf_counter()
+    oracle.gemv(W, call.fmt, call.N, call.K, x, call.B, rows=np.arange(64))
+    per_row = (time.perf_counter() - t0) / 64
+    total = max(1, args.steps + args.warmup)
+    rows = int(max(1, min(call.N, 60.0 / total / per_row)))
+
+    def step(s):
+        sel = (np.arange(rows) + s * rows) % call.N
+        oracle.gemv(W, call.fmt, call.N, call.K, x, call.B, rows=sel)
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step(s)
+    secs = time.perf_counter() - t0
+    step_bytes = rows * (row_bytes + 4 * call.B) + 2 * call.K * call.B
+    value = step_bytes * args.steps / secs / 1e9
+    sample = (f"{rows} of {call.N} rows of the Q4_K N=17408 K=5120 B=1 GEMV per step "
+              f"(dequant + fp64 dot, single-threaded C)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs * 1e3 / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle dot; fp32 weights)",
+        "data": "synthetic (seeded Q4_K bytes, x ~ N(0,1) fp16)",
+        "config": {"workload": "ffn_gate Q4_K GEMV N=17408 K=5120 B=1 (CPU oracle, row sample)",
+                   "global_batch": 1, "seq_len": 1, "parallelism": "replicas"},
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(value, 4),
+                         "unit": UNIT},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="qg", choices=["qg", "reference"])
+    ap.add_argument("--variant", type=int, default=0, help="QG_VARIANT_* (0 = library default)")
+    ap.add_argument("--table-steps", type=int, default=4000)
+    ap.add_argument("--no-table", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+    from quant_dequant_gemv_q4_b200 import build as qbuild
+    qbuild.build()
+    import quant_dequant_gemv_q4_b200 as qg
+
+    peaks = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    props = torch.cuda.get_device_properties(device)
+    l2 = int(getattr(props, "L2_cache_size", 126 << 20))
+
+    # headline: B=1
+    cs = CallSet([HEADLINE], HEADLINE_SEED, device, l2)
+    launches = cs.launches_per_step(args.variant)
+    variant_used = qg.qg_last_variant()
+    sampler = ClockSampler(local)
+    secs, ms_local = time_callset(cs, args.steps, args.warmup, args.variant, sampler)
+    clocks = sampler.summary()
+    secs_max, bytes_total = aggregate(secs, float(cs.bytes_per_step * args.steps), device)
+    value = bytes_total / secs_max / 1e9
+    per_launch_s = secs / (args.steps * launches)
+    achieved = cs.bytes_per_step / launches / per_launch_s / 1e9
+    khash = kernel_source_hash()
+    traffic = load_traffic(khash)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4),
+                "traffic": (traffic or {}).get("bytes_per_launch"),
+                "peak_source": f"{peaks['source']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
+
+    # B = 8 on the same tensor
+    cs8 = CallSet([HEADLINE_B8], HEADLINE_SEED, device, l2)
+    steps8 = max(200, min(args.steps // 4, 20000))
+    secs8, ms8 = time_callset(cs8, steps8, args.warmup, args.variant, None)
+    secs8 = dist_max(secs8, device)
+    b8 = {"us_per_call": round(secs8 * 1e6 / steps8, 3),
+          "gbs": round(cs8.bytes_per_step * steps8 / secs8 / 1e9, 1),
+          "frac_of_hbm": round(cs8.bytes_per_step * steps8 / secs8 / 1e9 / hbm, 4),
+          "flops_tflops": round(2 * HEADLINE_B8.N * HEADLINE_B8.K * 8 * steps8 / secs8 / 1e12, 2),
+          "steps": steps8}
+    del cs8
+
+    # every workload of the suite, per call
+    table = {}
+    if not args.no_table:
+        for name, wl in synth.WORKLOADS.items():
+            cst = CallSet(list(wl.calls), wl.seed, device, l2)
+            st = max(args.table_steps, 3 * cst.copies)
+            s_t, _ = time_callset(cst, st, args.warmup, args.variant, None)
+            s_t = dist_max(s_t, device)
+            per_call = {}
+            for c in wl.calls:
+                csc = CallSet([c], wl.seed, device, l2)
+                s_c, _ = time_callset(csc, max(args.table_steps, 3 * csc.copies), args.warmup,
+                                      args.variant, None)
+                s_c = dist_max(s_c, device)
+                n_c = max(args.table_steps, 3 * csc.copies)
+                gbs = c.algorithmic_bytes * n_c / s_c / 1e9
+                per_call[c.name] = {"N": c.N, "K": c.K, "B": c.B,
+                                    "fmt": "Q4_K" if c.fmt == synth.Q4_K else "Q8_0",
+                                    "us": round(s_c * 1e6 / n_c, 3), "gbs": round(gbs, 1),
+                                    "frac": round(gbs / hbm, 4),
+                                    "splits": qg.qg_last_splits()}
+                del csc
+            table[name] = {"us_per_step": round(s_t * 1e6 / st, 3),
+                           "gbs": round(cst.bytes_per_step * st / s_t / 1e9, 1),
+                           "calls": per_call, "copies": cst.copies}
+            del cst
+            torch.cuda.empty_cache()
+
+    # end to end through the Python API with host buffers
+    e2e_steps = min(args.steps, 3000)
+    s_e, h2d, d2h = time_e2e(cs, e2e_steps, min(args.warmup, 50), args.variant)
+    s_e = dist_max(s_e, device)
+    e2e = {"value": round(cs.bytes_per_step * e2e_steps * world / s_e / 1e9, 2), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "us_per_step": round(s_e * 1e6 / e2e_steps, 2)}
+    probe = hbm_probe(device)
+    del cs
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, rows, t, nb = oracle_sample_rate(HEADLINE, HEADLINE_SEED, args.cpu_seconds)
+        cpu = {"value": round(rate, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{rows} rows ({nb / 1e6:.1f} MB) of the N=17408 K=5120 B=1 call in "
+                         f"{t:.1f} s, single-threaded C oracle (dequant + fp64 dot)",
+               "host_cores": os.cpu_count()}
+
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs_max * 1e3 / args.steps, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (Q4_K weights, f16 x, f32 accumulate)",
+        "data": "synthetic (seeded Q4_K bytes with the workload's d/dmin/sc/m/q distributions, "
+                "x ~ N(0,1) fp16)",
+        "config": {"workload": "ffn_gate Q4_K GEMV N=17408 K=5120 B=1 (one call per step); "
+                               "B=8 on the same tensor in 'b8'",
+                   "global_batch": 1, "seq_len": 1, "parallelism": f"replicas x{world}",
+                   "l2": f"{cs_copies_note(HEADLINE, l2)}; L2 {l2 >> 20} MiB",
+                   "timing": "CUDA graphs of one call per weight copy, CUDA events on the "
+                             "launching stream"},
+        "us_per_call": round(secs_max * 1e6 / args.steps, 3),
+        "frac_of_hbm": round(value / world / hbm, 4),
+        "variant": variant_used,
+        "roofline": roofline,
+        "b8": b8,
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": args.steps * launches,
+        "cpu_baseline": cpu,
+        "hbm_probe": probe,
+        "kernel_hash": khash,
+        "workloads": table,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cs_copies_note(call, l2):
+    copies = max(2, -(-4 * l2 // call.weight_bytes))
+    return (f"{copies} rotating weight copies ({copies * call.weight_bytes / 1e6:.0f} MB > 4x L2), "
+            "so every step reads its weights from HBM")
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,146 @@
+/*
+ * qg.h -- C ABI of libqg, a B200 (sm_100a) dequant GEMV over GGML block-quantized weights:
+ *
+ *     y[N,B] = dequant(W[N,K]) . x[K,B]      x fp16, accumulation fp32, y fp32, 1 <= B <= 8
+ *
+ * The operation is the mixed-quant GEMV of "HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle)"
+ * (second prompt, section "SPEC": y = dequant(W[N,K]) @ x[K], the format chosen by a tensor-type
+ * flag passed to the kernel; section "HARD CONSTRAINTS": x broadcast through shared memory, wide
+ * coalesced weight loads).  The Q4_K superblock and its dequantization w = d*(sc*q) - dmin*m are
+ * from the same dossier's "QUANTIZATION MIX"; "PHYSICS & CONTRACT" fixes fp32 accumulation and
+ * that each weight byte is read from DRAM at most once per token, which is what makes a batch of
+ * B <= 8 columns (speculative / MTP verify) share one pass over W.  The pages' fp16 y is replaced
+ * by fp32 y.
+ *
+ * Formats (GGML layouts; the pages name them but do not spell them out):
+ *   QG_FMT_Q4_K: 256 weights in 144 bytes {fp16 d; fp16 dmin; u8 scales[12]; u8 qs[128]},
+ *                w = d*sc_j*q - dmin*m_j with 6-bit (sc_j, m_j) of sub-block j = i/32 packed in
+ *                scales[12] (get_scale_min_k4 layout) and q the 4-bit nibble of weight i:
+ *                byte qs[32*(i/64) + i%32], low nibble if i%64 < 32 else high nibble.
+ *   QG_FMT_Q8_0: 32 weights in 34 bytes {fp16 d; i8 qs[32]}, w = d*q.
+ *   The flag values are GGML's type ids.
+ *
+ * Layouts: W row-major, row n = K/256 consecutive superblocks (Q4_K) or K/32 consecutive blocks
+ * (Q8_0); x[k*B + b] (fp16 bits); y[n*B + b] (fp32).  A caller holding activations [B][K] passes
+ * their transpose.
+ *
+ * Ownership: every pointer is the caller's; the library never frees caller memory.  The library
+ * owns one small workspace per (device, stream) for split rows (partial sums, arrival counters,
+ * an error word), allocated with cudaMalloc the first time a stream needs one of that size and
+ * kept until process exit.  Make the first call on a stream outside CUDA-graph capture.
+ *
+ * Errors: every call returns a qg_status.  Argument errors are found on the host before anything
+ * is enqueued.  Launch errors return QG_ERR_CUDA.  Faults of the asynchronous work surface at the
+ * caller's next synchronization.  Device-side timeouts (a copy that never lands) are recorded in
+ * the stream's error word, read with qg_device_error().  The library never aborts or prints.
+ *
+ * Determinism: for fixed inputs, device and library build, y is bitwise identical run to run
+ * (every reduction, including across thread blocks, sums in a fixed order).
+ *
+ * Thread safety: calls on different streams may run concurrently.  Calls on one stream are
+ * ordered by the stream.
+ */
+#ifndef QG_H
+#define QG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Block formats (GGML type ids). */
+enum { QG_FMT_Q8_0 = 8, QG_FMT_Q4_K = 12 };
+
+/* Status codes. */
+enum {
+    QG_OK = 0,
+    QG_ERR_NULL = 1,    /* a required pointer is NULL */
+    QG_ERR_FMT = 2,     /* unknown format flag */
+    QG_ERR_SHAPE = 3,   /* N < 0, K < 1, or K not a multiple of the block size */
+    QG_ERR_BATCH = 4,   /* B outside 1..8 */
+    QG_ERR_ALIGN = 5,   /* W not 16-byte aligned, x not 2-byte aligned or y not 4-byte aligned */
+    QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
+    QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
+    QG_ERR_RANGE = 8,   /* a packer field is out of range (sc, m > 63; Q4_K q > 15; Q8_0 q = -128) */
+    QG_ERR_VARIANT = 9  /* unknown kernel variant, or a variant that does not take this format */
+};
+
+/* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses. */
+enum {
+    QG_VARIANT_AUTO = 0,
+    /* Q4_K: each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m)
+     * (the dump's value) and multiplied by x: the error is bounded relative to sum|w*x|. */
+    QG_VARIANT_DIRECT = 1,
+    /* Q4_K: the scale and min are applied per 32-weight sub-block, y = sum_j (d*sc_j)*sum(q*x)
+     * - (dmin*m_j)*sum(x); fewer instructions per weight, error bounded relative to
+     * sum(|d*sc*q*x| + |dmin*m*x|). */
+    QG_VARIANT_FACTORED = 2,
+    /* Any format and shape: one warp per row, plain loads, no shared-memory staging.  Used by
+     * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0). */
+    QG_VARIANT_GENERIC = 3
+};
+
+/* Bytes of an N x K tensor in format fmt; 0 if fmt is unknown, N < 0, K < 1 or K is not a
+ * multiple of the block size (256 for Q4_K, 32 for Q8_0). */
+size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
+
+/* y = dequant(W) . x on the device.
+ *   W      device, qg_weight_bytes(fmt, N, K) bytes, 16-byte aligned, read only
+ *   fmt    QG_FMT_Q4_K or QG_FMT_Q8_0
+ *   N, K   rows and reduction length; N >= 0 (N == 0 does nothing); K >= 1, K % block == 0
+ *   x      device, fp16 bits [K][B], 2-byte aligned, read only
+ *   B      number of columns, 1..8
+ *   y      device, fp32 [N][B], 4-byte aligned, fully overwritten (not accumulated)
+ *   stream a cudaStream_t (NULL = the legacy default stream); the call is asynchronous
+ * Returns QG_OK once the work is enqueued. */
+int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
+            void *stream);
+
+/* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT if the variant does not
+ * take this format (DIRECT and FACTORED are Q4_K only; GENERIC takes both). */
+int qg_gemv_variant(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
+                    float *y, void *stream, int variant);
+
+/* Dump mode: out[n*K + k] = the fp32 dequantized weight w[n,k], correctly rounded from its exact
+ * value, computed by the same device unpacking code the GEMV uses.
+ *   W device as for qg_gemv; out device, fp32 [N][K], 4-byte aligned.  Asynchronous on stream. */
+int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, void *stream);
+
+/* Host-side bit packer (fields -> GGML bytes); it does not choose scales, it only places bits.
+ *   Q4_K: d[N*K/256], dmin[N*K/256] fp16 bits; sc[N*K/32], m[N*K/32] 6-bit values (<= 63);
+ *         q = uint8 [N*K] values 0..15, weight order.
+ *   Q8_0: d[N*K/32] fp16 bits; dmin, sc, m are ignored; q = int8 [N*K] in -127..127.
+ *   out   host, qg_weight_bytes(fmt, N, K) bytes.
+ * All pointers are host pointers.  QG_ERR_RANGE if a field is out of range (out is then
+ * unspecified). */
+int qg_pack_reference(int fmt, int64_t N, int64_t K, const uint16_t *d, const uint16_t *dmin,
+                      const uint8_t *sc, const uint8_t *m, const void *q, void *out);
+
+/* Kernel variant launched by the last successful qg_gemv / qg_gemv_variant of the calling host
+ * thread (a launch witness: QG_VARIANT_DIRECT, _FACTORED or _GENERIC), 0 if none yet. */
+int qg_last_variant(void);
+
+/* Number of K slices the last GEMV of the calling thread used (1 = no split-K second pass). */
+int qg_last_splits(void);
+
+/* Reads and clears the device error word of the workspace that (current device, stream) uses;
+ * synchronizes the stream.  *flag = 0 if no device-side timeout happened, else a nonzero code. */
+int qg_device_error(void *stream, int *flag);
+
+/* Bandwidth probes (for measurement): dst[i] = src[i] over `bytes` bytes (16-byte multiple,
+ * both 16-byte aligned), and a read-only pass that xor-folds `bytes` of src into out[i] for
+ * i < 4 * (SM count) (out: device, zero-initialised by the caller, at least 4096 uint32).
+ * Asynchronous on stream. */
+int qg_hbm_copy(const void *src, void *dst, size_t bytes, void *stream);
+int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
+
+/* Static text for a status code. */
+const char *qg_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QG_H */

@@ -1,0 +1,408 @@
+// qg_api.cu -- host side of libqg's C ABI: argument checks, launch planning, the per-stream
+// workspace, kernel dispatch.  Declarations and contracts: include/qg.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/qg.h"
+#include "qg_device.cuh"
+
+namespace {
+
+using namespace qg;
+
+struct DeviceInfo {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_dev;
+std::set<std::pair<int, const void *>> g_attr_set;
+
+thread_local int t_last_variant = 0;
+thread_local int t_last_splits = 0;
+
+int device_info(DeviceInfo *out, int *dev_out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QG_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess)
+            return QG_ERR_CUDA;
+        it = g_dev.emplace(dev, d).first;
+    }
+    *out = it->second;
+    *dev_out = dev;
+    return QG_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (device, kernel).
+int ensure_smem_attr(int dev, const void *func, int bytes)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_attr_set.count({dev, func})) return QG_OK;
+    }
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return QG_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_attr_set.insert({dev, func});
+    return QG_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Workspace: one per (device, stream).  Layout: [err int | pad to 256] [cnt uint[nw]]
+// [slots float[nw*2*8]] [part float[...]].  Counters are zeroed once at allocation; every
+// completed call leaves them at zero again (each counter wraps after its last arrival).
+// ---------------------------------------------------------------------------------------------
+struct Workspace {
+    uint8_t *base = nullptr;
+    size_t bytes = 0;
+    size_t nw = 0;       // warps covered by cnt / slots
+    size_t part_f = 0;   // floats of the split-K partial buffer
+};
+std::map<std::pair<int, void *>, Workspace> g_ws;
+
+struct WsView {
+    int *err;
+    unsigned *cnt;
+    float *slots;
+    float *part;
+};
+
+size_t ws_bytes_for(size_t nw, size_t part_f)
+{
+    return 256 + nw * sizeof(unsigned) + nw * 2 * 8 * sizeof(float) + part_f * sizeof(float) + 256;
+}
+
+WsView ws_view(const Workspace &w)
+{
+    WsView v;
+    v.err = reinterpret_cast<int *>(w.base);
+    v.cnt = reinterpret_cast<unsigned *>(w.base + 256);
+    v.slots = reinterpret_cast<float *>(w.base + 256 + w.nw * sizeof(unsigned));
+    v.part = v.slots + w.nw * 2 * 8;
+    return v;
+}
+
+int get_workspace(int dev, void *stream, size_t nw, size_t part_f, WsView *out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace &w = g_ws[{dev, stream}];
+    if (w.base && w.nw >= nw && w.part_f >= part_f) {
+        *out = ws_view(w);
+        return QG_OK;
+    }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap) != cudaSuccess)
+        return QG_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return QG_ERR_NOMEM;  // cannot grow while capturing
+    const size_t new_nw = std::max(nw, w.nw);
+    const size_t new_pf = std::max(part_f, w.part_f);
+    const size_t bytes = ws_bytes_for(new_nw, new_pf);
+    if (w.base) {
+        // the old buffer may still be read by work queued on this stream
+        if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return QG_ERR_CUDA;
+        cudaFree(w.base);
+        w.base = nullptr;
+    }
+    void *p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+        w = Workspace();
+        return QG_ERR_NOMEM;
+    }
+    if (cudaMemset(p, 0, bytes) != cudaSuccess) {
+        cudaFree(p);
+        w = Workspace();
+        return QG_ERR_CUDA;
+    }
+    w.base = static_cast<uint8_t *>(p);
+    w.bytes = bytes;
+    w.nw = new_nw;
+    w.part_f = new_pf;
+    *out = ws_view(w);
+    return QG_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Planning.
+// ---------------------------------------------------------------------------------------------
+int padded_cols(int B) { return B == 1 ? 1 : B == 2 ? 2 : B <= 4 ? 4 : 8; }
+
+struct Plan {
+    int BP, S, US, Gs, G, xs_floats;
+    size_t smem;
+};
+
+Plan make_plan(int fmt, int var, int64_t N, int64_t K, int B, const DeviceInfo &di)
+{
+    Plan p;
+    p.BP = padded_cols(B);
+    const int UB = (fmt == kFmtQ4_K) ? UnitFmt<kFmtQ4_K>::kBytes : UnitFmt<kFmtQ8_0>::kBytes;
+    const int CH = (fmt == kFmtQ4_K) ? UnitFmt<kFmtQ4_K>::kChunk : UnitFmt<kFmtQ8_0>::kChunk;
+    const size_t ring = (size_t)kWarps * kStages * CH * UB;
+    const size_t bars = (size_t)kWarps * kStages * 8;
+    const bool factored = (fmt == kFmtQ4_K && var == kVarFactored);
+    const size_t per_unit = (size_t)(256 * p.BP + (factored ? 8 * p.BP : 0)) * sizeof(float);
+    const size_t avail = (size_t)di.smem_optin - ring - bars - 128;
+    int64_t fit = (int64_t)(avail / per_unit);
+    fit -= fit & 1;  // staged x is allocated in pairs of units
+    if (fit < 2) fit = 2;
+    const int64_t UPR = K / 256;
+    int64_t S = (UPR + fit - 1) / fit;
+    const int64_t US = (UPR + S - 1) / S;
+    S = (UPR + US - 1) / US;
+    p.S = (int)S;
+    p.US = (int)US;
+    p.xs_floats = (int)(((US + 1) / 2) * 2 * 256 * p.BP);
+    const size_t xsum_f = factored ? (size_t)US * 8 * p.BP : 0;
+    p.smem = ring + (size_t)p.xs_floats * sizeof(float) + xsum_f * sizeof(float) + bars;
+    const int64_t items = N * US;
+    const int64_t want = std::max<int64_t>(1, (items + kWarps * 8 - 1) / (kWarps * 8));
+    const int64_t per_slice = std::max<int64_t>(1, di.sms / S);
+    p.Gs = (int)std::min(per_slice, want);
+    p.G = p.Gs * p.S;
+    return p;
+}
+
+const void *stream_kernel_ptr(int fmt, int BP, int var)
+{
+#define QG_PICK(F, V)                                                           \
+    switch (BP) {                                                              \
+    case 1: return reinterpret_cast<const void *>(&stream_gemv_kernel<F, 1, V>); \
+    case 2: return reinterpret_cast<const void *>(&stream_gemv_kernel<F, 2, V>); \
+    case 4: return reinterpret_cast<const void *>(&stream_gemv_kernel<F, 4, V>); \
+    default: return reinterpret_cast<const void *>(&stream_gemv_kernel<F, 8, V>); \
+    }
+    if (fmt == kFmtQ8_0) {
+        QG_PICK(kFmtQ8_0, kVarDirect)
+    } else if (var == kVarFactored) {
+        QG_PICK(kFmtQ4_K, kVarFactored)
+    } else {
+        QG_PICK(kFmtQ4_K, kVarDirect)
+    }
+#undef QG_PICK
+}
+
+int check_common(const void *W, int fmt, int64_t N, int64_t K)
+{
+    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_FMT;
+    const int64_t bw = (fmt == QG_FMT_Q4_K) ? 256 : 32;
+    if (N < 0 || K < 1 || K % bw != 0) return QG_ERR_SHAPE;
+    if (N > 0 && !W) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(W) % 16 != 0) return QG_ERR_ALIGN;
+    return QG_OK;
+}
+
+int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
+                   cudaStream_t st, const DeviceInfo &di)
+{
+    const int threads = 256;
+    const int64_t warps_needed = N;
+    const int64_t blocks = std::min<int64_t>((warps_needed + 7) / 8, (int64_t)di.sms * 8);
+    if (fmt == kFmtQ4_K)
+        rowwise_gemv_kernel<kFmtQ4_K><<<(unsigned)blocks, threads, 0, st>>>(
+            static_cast<const uint8_t *>(W), N, K, x, B, y);
+    else
+        rowwise_gemv_kernel<kFmtQ8_0><<<(unsigned)blocks, threads, 0, st>>>(
+            static_cast<const uint8_t *>(W), N, K, x, B, y);
+    return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
+              void *stream, int variant)
+{
+    int rc = check_common(W, fmt, N, K);
+    if (rc != QG_OK) return rc;
+    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_GENERIC) return QG_ERR_VARIANT;
+    if (fmt == QG_FMT_Q8_0 && variant == QG_VARIANT_FACTORED) return QG_ERR_VARIANT;
+    if (N == 0) return QG_OK;
+    if (!x || !y) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
+        return QG_ERR_ALIGN;
+    DeviceInfo di;
+    int dev = 0;
+    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // streaming kernel needs whole 16-byte-multiple units per row: always for Q4_K, K % 256 == 0
+    // for Q8_0
+    const bool streamable = (K % 256 == 0);
+    int var = variant;
+    if (var == QG_VARIANT_AUTO) var = streamable ? QG_VARIANT_DIRECT : QG_VARIANT_GENERIC;
+    if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
+    if (fmt == QG_FMT_Q8_0 && var != QG_VARIANT_GENERIC) var = QG_VARIANT_DIRECT;
+
+    if (var == QG_VARIANT_GENERIC) {
+        rc = launch_rowwise(W, fmt, N, K, x, B, y, st, di);
+        if (rc == QG_OK) {
+            t_last_variant = QG_VARIANT_GENERIC;
+            t_last_splits = 1;
+        }
+        return rc;
+    }
+
+    const int kvar = (var == QG_VARIANT_FACTORED) ? kVarFactored : kVarDirect;
+    const Plan p = make_plan(fmt, kvar, N, K, B, di);
+    const void *fn = stream_kernel_ptr(fmt, p.BP, kvar);
+    if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+    if ((rc = ensure_smem_attr(dev, fn, di.smem_optin)) != QG_OK) return rc;
+    WsView ws;
+    const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
+    if ((rc = get_workspace(dev, stream, (size_t)p.G * kWarps, part_f, &ws)) != QG_OK) return rc;
+
+    StreamArgs a;
+    a.W = static_cast<const uint8_t *>(W);
+    a.x = x;
+    a.out = (p.S > 1) ? ws.part : y;
+    a.slots = ws.slots;
+    a.cnt = ws.cnt;
+    a.err = ws.err;
+    a.N = N;
+    a.B = B;
+    a.UPR = (int)(K / 256);
+    a.US = p.US;
+    a.S = p.S;
+    a.Gs = p.Gs;
+    a.xs_floats = p.xs_floats;
+    void *args[] = {&a};
+    if (cudaLaunchKernel(fn, dim3(p.G), dim3(kWarps * 32), args, p.smem, st) != cudaSuccess)
+        return QG_ERR_CUDA;
+    if (p.S > 1) {
+        const int64_t NB = N * B;
+        const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
+        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(ws.part, y, NB, p.S);
+        if (cudaGetLastError() != cudaSuccess) return QG_ERR_CUDA;
+    }
+    t_last_variant = var;
+    t_last_splits = p.S;
+    return QG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
+            void *stream)
+{
+    return gemv_impl(W, fmt, N, K, x, B, y, stream, QG_VARIANT_AUTO);
+}
+
+int qg_gemv_variant(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
+                    float *y, void *stream, int variant)
+{
+    return gemv_impl(W, fmt, N, K, x, B, y, stream, variant);
+}
+
+int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, void *stream)
+{
+    int rc = check_common(W, fmt, N, K);
+    if (rc != QG_OK) return rc;
+    if (N == 0) return QG_OK;
+    if (!out) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(out) % 4 != 0) return QG_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (fmt == QG_FMT_Q4_K) {
+        const int64_t nsb = N * (K / 256);
+        const int64_t threads = nsb * 4;
+        dequant_q4k_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+            static_cast<const uint8_t *>(W), nsb, out);
+    } else {
+        const int64_t nblk = N * (K / 32);
+        dequant_q8_0_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(
+            static_cast<const uint8_t *>(W), nblk, out);
+    }
+    return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+int qg_last_variant(void) { return t_last_variant; }
+
+int qg_last_splits(void) { return t_last_splits; }
+
+int qg_device_error(void *stream, int *flag)
+{
+    if (!flag) return QG_ERR_NULL;
+    *flag = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QG_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Workspace w;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_ws.find({dev, stream});
+        if (it == g_ws.end()) return QG_OK;
+        w = it->second;
+    }
+    if (cudaStreamSynchronize(st) != cudaSuccess) return QG_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, w.base, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return QG_ERR_CUDA;
+    if (v != 0) {
+        // a warp that gave up left its rows unfinished: clear the error word and the counters
+        if (cudaMemset(w.base, 0, 256 + w.nw * sizeof(unsigned)) != cudaSuccess) return QG_ERR_CUDA;
+    }
+    *flag = v;
+    return QG_OK;
+}
+
+int qg_hbm_copy(const void *src, void *dst, size_t bytes, void *stream)
+{
+    if (!src || !dst) return QG_ERR_NULL;
+    if (bytes % 16 || reinterpret_cast<uintptr_t>(src) % 16 || reinterpret_cast<uintptr_t>(dst) % 16)
+        return QG_ERR_ALIGN;
+    DeviceInfo di;
+    int dev = 0;
+    int rc = device_info(&di, &dev);
+    if (rc != QG_OK) return rc;
+    hbm_copy_kernel<<<di.sms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), (int64_t)(bytes / 16));
+    return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream)
+{
+    if (!src || !out) return QG_ERR_NULL;
+    if (bytes % 16 || reinterpret_cast<uintptr_t>(src) % 16) return QG_ERR_ALIGN;
+    DeviceInfo di;
+    int dev = 0;
+    int rc = device_info(&di, &dev);
+    if (rc != QG_OK) return rc;
+    hbm_read_kernel<<<di.sms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(src), (int64_t)(bytes / 16), out);
+    return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+const char *qg_status_string(int status)
+{
+    switch (status) {
+    case QG_OK: return "ok";
+    case QG_ERR_NULL: return "a required pointer is NULL";
+    case QG_ERR_FMT: return "unknown format flag";
+    case QG_ERR_SHAPE: return "invalid shape (N < 0, K < 1 or K not a multiple of the block size)";
+    case QG_ERR_BATCH: return "B must be in 1..8";
+    case QG_ERR_ALIGN: return "misaligned pointer (W 16 B, x 2 B, y 4 B)";
+    case QG_ERR_CUDA: return "CUDA runtime error";
+    case QG_ERR_NOMEM: return "workspace allocation failed";
+    case QG_ERR_RANGE: return "packer field out of range";
+    case QG_ERR_VARIANT: return "kernel variant not available for this format/shape";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+"""Host-side tests of the C-ABI library (no GPU needed): it loads, exports every function that
+include/qg.h declares, computes sizes, packs bits exactly as the oracle unpacks them, and rejects
+bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import quant_dequant_gemv_q4_b200 as qg
+from quant_dequant_gemv_q4_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session")
+def L():
+    from quant_dequant_gemv_q4_b200 import build
+    build.build()
+    return qg.lib()
+
+
+def _declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(qg_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert "qg_gemv" in names and "qg_pack_reference" in names and "qg_weight_bytes" in names
+    for n in names:
+        assert hasattr(L, n), n
+        getattr(L, n)  # resolves the symbol
+
+
+def test_weight_bytes(L, orc):
+    for fmt, N, K in [(12, 17408, 5120), (12, 5120, 17408), (8, 12288, 5120), (12, 1024, 5120),
+                      (8, 3, 96), (12, 0, 256), (12, 1, 300), (8, 1, 33), (7, 1, 256),
+                      (12, -1, 256), (12, 1, 0)]:
+        assert qg.qg_weight_bytes(fmt, N, K) == max(orc.weight_bytes(fmt, N, K), 0), (fmt, N, K)
+
+
+def test_pack_q4k_roundtrips_through_oracle_unpack(L, orc):
+    """Random fields -> product packer -> oracle field view == the same fields."""
+    rng = np.random.default_rng(0)
+    N, K = 3, 768
+    nsb, nsub = N * K // 256, N * K // 32
+    d = rng.integers(0, 65536, nsb, dtype=np.uint16)
+    dmin = rng.integers(0, 65536, nsb, dtype=np.uint16)
+    sc = rng.integers(0, 64, nsub, dtype=np.uint8)
+    m = rng.integers(0, 64, nsub, dtype=np.uint8)
+    q = rng.integers(0, 16, N * K, dtype=np.uint8)
+    W = qg.qg_pack_reference(12, N, K, d, dmin, sc, m, q)
+    f = orc.unpack_q4k(W, nsb)
+    assert np.array_equal(f["d"], d) and np.array_equal(f["dmin"], dmin)
+    assert np.array_equal(f["sc"].reshape(-1), sc) and np.array_equal(f["m"].reshape(-1), m)
+    assert np.array_equal(f["q"].reshape(-1), q)
+
+
+def test_pack_q4k_bytes_roundtrip(L, orc):
+    """Random bytes -> oracle fields -> product packer == the same bytes (one-to-one format)."""
+    N, K = 2, 512
+    W = synth.q4k_weights(N, K, seed=3)
+    f = orc.unpack_q4k(W, N * K // 256)
+    W2 = qg.qg_pack_reference(12, N, K, f["d"], f["dmin"], f["sc"].reshape(-1),
+                              f["m"].reshape(-1), f["q"].reshape(-1))
+    assert np.array_equal(W, W2)
+
+
+def test_pack_q8_0_roundtrip(L, orc):
+    N, K = 4, 96
+    W = synth.q8_0_weights(N, K, seed=1)
+    f = orc.unpack_q8_0(W, N * K // 32)
+    W2 = qg.qg_pack_reference(8, N, K, f["d"], None, None, None, f["q"].reshape(-1))
+    assert np.array_equal(W, W2)
+
+
+def test_pack_range_checks(L):
+    N, K = 1, 256
+    ok = dict(d=np.zeros(1, np.uint16), dmin=np.zeros(1, np.uint16), sc=np.zeros(8, np.uint8),
+              m=np.zeros(8, np.uint8), q=np.zeros(256, np.uint8))
+    qg.qg_pack_reference(12, N, K, **ok)
+    for key, bad in [("sc", 64), ("m", 64), ("q", 16)]:
+        args = dict(ok)
+        args[key] = args[key].copy()
+        args[key][0] = bad
+        with pytest.raises(qg.QgError) as e:
+            qg.qg_pack_reference(12, N, K, **args)
+        assert e.value.status == qg.QG_ERR_RANGE
+    q8 = np.zeros(32, np.int8)
+    q8[5] = -128
+    with pytest.raises(qg.QgError) as e:
+        qg.qg_pack_reference(8, 1, 32, np.zeros(1, np.uint16), None, None, None, q8)
+    assert e.value.status == qg.QG_ERR_RANGE
+
+
+# Argument validation happens on the host before any CUDA call, so these run without a GPU.
+FAKE = 0x10000  # a 16-byte-aligned non-null pointer value that is never dereferenced
+
+
+@pytest.mark.parametrize("args,status", [
+    ((FAKE, 99, 4, 256, FAKE, 1, FAKE), qg.QG_ERR_FMT),
+    ((FAKE, 12, 4, 300, FAKE, 1, FAKE), qg.QG_ERR_SHAPE),
+    ((FAKE, 12, 4, 0, FAKE, 1, FAKE), qg.QG_ERR_SHAPE),
+    ((FAKE, 12, -1, 256, FAKE, 1, FAKE), qg.QG_ERR_SHAPE),
+    ((FAKE, 8, 4, 48, FAKE, 1, FAKE), qg.QG_ERR_SHAPE),
+    ((FAKE, 12, 4, 256, FAKE, 0, FAKE), qg.QG_ERR_BATCH),
+    ((FAKE, 12, 4, 256, FAKE, 9, FAKE), qg.QG_ERR_BATCH),
+    ((0, 12, 4, 256, FAKE, 1, FAKE), qg.QG_ERR_NULL),
+    ((FAKE, 12, 4, 256, 0, 1, FAKE), qg.QG_ERR_NULL),
+    ((FAKE, 12, 4, 256, FAKE, 1, 0), qg.QG_ERR_NULL),
+    ((FAKE + 8, 12, 4, 256, FAKE, 1, FAKE), qg.QG_ERR_ALIGN),
+    ((FAKE, 12, 4, 256, FAKE + 1, 1, FAKE), qg.QG_ERR_ALIGN),
+    ((FAKE, 12, 4, 256, FAKE, 1, FAKE + 2), qg.QG_ERR_ALIGN),
+])
+def test_gemv_rejects_bad_arguments(L, args, status):
+    assert L.qg_gemv(*args, None) == status
+
+
+def test_gemv_zero_rows_is_a_noop(L):
+    assert L.qg_gemv(None, 12, 0, 256, None, 1, None, None) == qg.QG_OK
+
+
+def test_variant_checks(L):
+    # FACTORED is Q4_K only; unknown variants are rejected
+    assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_FACTORED) == \
+        qg.QG_ERR_VARIANT
+    assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 7) == qg.QG_ERR_VARIANT
+
+
+def test_dequant_rejects_bad_arguments(L):
+    assert L.qg_dequant_f32(FAKE, 5, 1, 256, FAKE, None) == qg.QG_ERR_FMT
+    assert L.qg_dequant_f32(FAKE, 12, 1, 255, FAKE, None) == qg.QG_ERR_SHAPE
+    assert L.qg_dequant_f32(FAKE, 12, 1, 256, 0, None) == qg.QG_ERR_NULL
+    assert L.qg_dequant_f32(FAKE, 12, 1, 256, FAKE + 1, None) == qg.QG_ERR_ALIGN
+
+
+def test_status_strings(L):
+    for s in range(10):
+        assert qg.status_string(s) and qg.status_string(s) != "unknown status"
+    assert qg.status_string(1234) == "unknown status"
+
+
+def test_probe_argument_checks(L):
+    assert L.qg_hbm_copy(FAKE, FAKE, 17, None) == qg.QG_ERR_ALIGN
+    assert L.qg_hbm_read(0, 16, FAKE, None) == qg.QG_ERR_NULL
