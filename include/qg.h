@@ -64,7 +64,8 @@ enum {
     QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
     QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
     QG_ERR_RANGE = 8,   /* a packer field is out of range (sc, m > 63; Q4_K q > 15; Q8_0 q = -128) */
-    QG_ERR_VARIANT = 9  /* unknown kernel variant, or a variant that does not take this format */
+    QG_ERR_VARIANT = 9, /* unknown kernel variant, or a variant that does not take this format */
+    QG_ERR_SCRATCH = 10 /* qg_gemv_noalloc: the call needs more scratch than its fixed array holds */
 };
 
 /* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses. */
@@ -135,6 +136,32 @@ int qg_device_error(void *stream, int *flag);
  * Asynchronous on stream. */
 int qg_hbm_copy(const void *src, void *dst, size_t bytes, void *stream);
 int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
+
+/* Size of the fixed device array qg_gemv_noalloc uses as scratch (per GPU, held until exit). */
+#define QG_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/* qg_gemv without any allocation.  The pages have no counterpart of this entry point; it exists
+ * for callers that cannot let a library call cudaMalloc: a host framework or plugin interface
+ * that owns all device memory through its own pool, a decode loop that cannot afford the
+ * device-wide synchronization an allocation may cause, or code recorded into a CUDA graph (an
+ * allocation during capture is an error).  The caller passes inputs and outputs exactly as for
+ * qg_gemv (same arguments, layouts, preconditions and results, default kernel variant); the
+ * kernel's scratch (arrival counters, partial sums of rows split between warps, split-K partial
+ * rows) lives in one file-scope device array of QG_NOALLOC_SCRATCH_BYTES per GPU.
+ *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library routine.  Each call
+ *     clears the counters it uses with cudaMemsetAsync on `stream`, since the array keeps what
+ *     the previous call left.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current) and caches it; make that first call before any stream capture.
+ *   - Every call on every stream shares the one array: calls that overlap on the GPU race and give
+ *     wrong results.  Serialize them (one stream, or events between streams).
+ *   - QG_ERR_SCRATCH if the call needs more scratch than the array holds (this happens only when
+ *     x for the whole of K does not fit in shared memory and N*B is large: the split-K partial
+ *     rows need S*N*B*4 bytes); nothing is enqueued then.
+ *   - Device-side copy timeouts are not reported by this entry point (qg_device_error reads the
+ *     allocating path's workspaces only). */
+int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
+                    float *y, void *stream);
 
 /* Static text for a status code. */
 const char *qg_status_string(int status);

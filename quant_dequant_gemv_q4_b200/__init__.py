@@ -33,6 +33,10 @@ QG_ERR_CUDA = 6
 QG_ERR_NOMEM = 7
 QG_ERR_RANGE = 8
 QG_ERR_VARIANT = 9
+QG_ERR_SCRATCH = 10
+
+# bytes of the fixed device array qg_gemv_noalloc uses as scratch
+QG_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqg.so")
@@ -61,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.qg_gemv.restype = I
         L.qg_gemv_variant.argtypes = [P, I, I64, I64, P, I, P, P, I]
         L.qg_gemv_variant.restype = I
+        L.qg_gemv_noalloc.argtypes = [P, I, I64, I64, P, I, P, P]
+        L.qg_gemv_noalloc.restype = I
         L.qg_dequant_f32.argtypes = [P, I, I64, I64, P, P]
         L.qg_dequant_f32.restype = I
         L.qg_pack_reference.argtypes = [I, I64, I64, P, P, P, P, P, P]
@@ -129,6 +135,13 @@ def qg_gemv_variant(W, fmt: int, N: int, K: int, x, B: int, y, stream=None,
                     variant: int = QG_VARIANT_AUTO) -> None:
     _ok(lib().qg_gemv_variant(_ptr(W), int(fmt), int(N), int(K), _ptr(x), int(B), _ptr(y),
                               _stream(stream), int(variant)), "qg_gemv_variant")
+
+
+def qg_gemv_noalloc(W, fmt: int, N: int, K: int, x, B: int, y, stream=None) -> None:
+    """qg_gemv that allocates nothing: scratch in the library's fixed device array (for callers
+    that cannot let the library call cudaMalloc; calls that overlap on the GPU race)."""
+    _ok(lib().qg_gemv_noalloc(_ptr(W), int(fmt), int(N), int(K), _ptr(x), int(B), _ptr(y),
+                              _stream(stream)), "qg_gemv_noalloc")
 
 
 def qg_dequant_f32(W, fmt: int, N: int, K: int, out, stream=None) -> None:

@@ -401,8 +401,105 @@ const char *qg_status_string(int status)
     case QG_ERR_NOMEM: return "workspace allocation failed";
     case QG_ERR_RANGE: return "packer field out of range";
     case QG_ERR_VARIANT: return "kernel variant not available for this format/shape";
+    case QG_ERR_SCRATCH: return "call needs more scratch than the fixed no-allocation array holds";
     default: return "unknown status";
     }
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free entry point.  Some callers cannot let a library call cudaMalloc: a host
+// framework or plugin interface that owns every device allocation through its own pool, a
+// decode loop that cannot afford the device-wide synchronization cudaMalloc may cause, code
+// recorded into a CUDA graph (allocating during capture is an error).  qg_gemv_noalloc runs
+// the same streaming kernel with its scratch (arrival counters, split-row partial sums, split-K
+// partial rows) in the fixed file-scope device array below instead of a cudaMalloc'd workspace.
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+// Every GPU that loads this library holds this array until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QG_NOALLOC_SCRATCH_BYTES];
+
+std::map<int, uint8_t *> g_noalloc_base;  // device address of the array, per device
+
+// The array's name is only a host-side stand-in in host code: its device address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(int dev, uint8_t **out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_noalloc_base.find(dev);
+    if (it != g_noalloc_base.end()) {
+        *out = it->second;
+        return QG_OK;
+    }
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return QG_ERR_CUDA;
+    g_noalloc_base.emplace(dev, static_cast<uint8_t *>(p));
+    *out = static_cast<uint8_t *>(p);
+    return QG_OK;
+}
+
+}  // namespace
+
+extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
+                               int B, float *y, void *stream)
+{
+    int rc = check_common(W, fmt, N, K);
+    if (rc != QG_OK) return rc;
+    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (N == 0) return QG_OK;
+    if (!x || !y) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
+        return QG_ERR_ALIGN;
+    DeviceInfo di;
+    int dev = 0;
+    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K % 256 != 0) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // needs no scratch
+
+    const int kvar = kVarDirect;
+    const Plan p = make_plan(fmt, kvar, N, K, B, di);
+    if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+    const size_t nw = (size_t)p.G * kWarps;
+    const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
+    if (ws_bytes_for(nw, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
+    const void *fn = stream_kernel_ptr(fmt, p.BP, kvar);
+    if ((rc = ensure_smem_attr(dev, fn, di.smem_optin)) != QG_OK) return rc;
+    uint8_t *base = nullptr;
+    if ((rc = noalloc_scratch(dev, &base)) != QG_OK) return rc;
+    Workspace w;
+    w.base = base;
+    w.bytes = QG_NOALLOC_SCRATCH_BYTES;
+    w.nw = nw;
+    w.part_f = part_f;
+    const WsView ws = ws_view(w);
+    // The array keeps whatever the previous call left; the arrival counters must start at zero.
+    if (cudaMemsetAsync(ws.cnt, 0, nw * sizeof(unsigned), st) != cudaSuccess) return QG_ERR_CUDA;
+
+    StreamArgs a;
+    a.W = static_cast<const uint8_t *>(W);
+    a.x = x;
+    a.out = (p.S > 1) ? ws.part : y;
+    a.slots = ws.slots;
+    a.cnt = ws.cnt;
+    a.err = ws.err;
+    a.N = N;
+    a.B = B;
+    a.UPR = (int)(K / 256);
+    a.US = p.US;
+    a.S = p.S;
+    a.Gs = p.Gs;
+    a.xs_floats = p.xs_floats;
+    void *args[] = {&a};
+    if (cudaLaunchKernel(fn, dim3(p.G), dim3(kWarps * 32), args, p.smem, st) != cudaSuccess)
+        return QG_ERR_CUDA;
+    if (p.S > 1) {
+        const int64_t NB = N * B;
+        const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
+        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(ws.part, y, NB, p.S);
+        if (cudaGetLastError() != cudaSuccess) return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}

@@ -143,7 +143,7 @@ def test_dequant_rejects_bad_arguments(L):
 
 
 def test_status_strings(L):
-    for s in range(10):
+    for s in range(11):
         assert qg.status_string(s) and qg.status_string(s) != "unknown status"
     assert qg.status_string(1234) == "unknown status"
 
