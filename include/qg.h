@@ -68,15 +68,19 @@ enum {
     QG_ERR_SCRATCH = 10 /* qg_gemv_noalloc: the call needs more scratch than its fixed array holds */
 };
 
-/* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses. */
+/* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses:
+ * FACTORED when K % 256 == 0, else GENERIC. */
 enum {
     QG_VARIANT_AUTO = 0,
-    /* Q4_K: each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m)
-     * (the dump's value) and multiplied by x: the error is bounded relative to sum|w*x|. */
+    /* Each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m) (Q4_K; the
+     * dump's value) or w = d*q (Q8_0) and multiplied by x: the error is bounded relative to
+     * sum|w*x| for any input.  Four lanes per 256-weight unit; slower. */
     QG_VARIANT_DIRECT = 1,
-    /* Q4_K: the scale and min are applied per 32-weight sub-block, y = sum_j (d*sc_j)*sum(q*x)
-     * - (dmin*m_j)*sum(x); fewer instructions per weight, error bounded relative to
-     * sum(|d*sc*q*x| + |dmin*m*x|). */
+    /* One lane per row.  Q4_K: the scale and min are applied per 32-weight sub-block,
+     * y = sum_j (d*sc_j)*sum(q*x) - (dmin*m_j)*sum(x), with every q*x product exact; the error is
+     * bounded relative to sum(|d*sc*q*x| + |dmin*m*x|), which exceeds sum|w*x| only when
+     * d*sc*q and dmin*m nearly cancel.  Q8_0: the block scale d is applied per 32 weights (error
+     * relative to sum|w*x|).  Requires K % 256 == 0. */
     QG_VARIANT_FACTORED = 2,
     /* Any format and shape: one warp per row, plain loads, no shared-memory staging.  Used by
      * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0). */
@@ -99,8 +103,8 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
 int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
             void *stream);
 
-/* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT if the variant does not
- * take this format (DIRECT and FACTORED are Q4_K only; GENERIC takes both). */
+/* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant or
+ * for DIRECT / FACTORED when K % 256 != 0.  Every variant takes both formats. */
 int qg_gemv_variant(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
                     float *y, void *stream, int variant);
 
@@ -138,7 +142,7 @@ int qg_hbm_copy(const void *src, void *dst, size_t bytes, void *stream);
 int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
 
 /* Size of the fixed device array qg_gemv_noalloc uses as scratch (per GPU, held until exit). */
-#define QG_NOALLOC_SCRATCH_BYTES (2u << 20)
+#define QG_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /* qg_gemv without any allocation.  The pages have no counterpart of this entry point; it exists
  * for callers that cannot let a library call cudaMalloc: a host framework or plugin interface

@@ -36,7 +36,7 @@ QG_ERR_VARIANT = 9
 QG_ERR_SCRATCH = 10
 
 # bytes of the fixed device array qg_gemv_noalloc uses as scratch
-QG_NOALLOC_SCRATCH_BYTES = 2 << 20
+QG_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqg.so")

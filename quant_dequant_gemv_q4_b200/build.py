@@ -13,7 +13,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libqg.so")
 SOURCES = [os.path.join(CSRC, "qg_api.cu"), os.path.join(CSRC, "qg_pack.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, "qg_device.cuh"), os.path.join(INCLUDE, "qg.h")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cuh", ".h"))] \
+    + [os.path.join(INCLUDE, "qg.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -12,6 +12,9 @@
 
 #include "../../include/qg.h"
 #include "qg_device.cuh"
+#include "qg_rows.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace {
 
@@ -71,7 +74,8 @@ int ensure_smem_attr(int dev, const void *func, int bytes)
 struct Workspace {
     uint8_t *base = nullptr;
     size_t bytes = 0;
-    size_t nw = 0;       // warps covered by cnt / slots
+    size_t nw = 0;       // warps covered by cnt
+    size_t slot_f = 0;   // floats of split-row partial sums
     size_t part_f = 0;   // floats of the split-K partial buffer
 };
 std::map<std::pair<int, void *>, Workspace> g_ws;
@@ -83,26 +87,30 @@ struct WsView {
     float *part;
 };
 
-size_t ws_bytes_for(size_t nw, size_t part_f)
+size_t ws_bytes_for(size_t nw, size_t slot_f, size_t part_f)
 {
-    return 256 + nw * sizeof(unsigned) + nw * 2 * 8 * sizeof(float) + part_f * sizeof(float) + 256;
+    const size_t cnt_b = ((nw * sizeof(unsigned) + 255) / 256) * 256;
+    const size_t slot_b = ((slot_f * sizeof(float) + 255) / 256) * 256;
+    return 256 + cnt_b + slot_b + part_f * sizeof(float) + 256;
 }
 
 WsView ws_view(const Workspace &w)
 {
     WsView v;
+    const size_t cnt_b = ((w.nw * sizeof(unsigned) + 255) / 256) * 256;
+    const size_t slot_b = ((w.slot_f * sizeof(float) + 255) / 256) * 256;
     v.err = reinterpret_cast<int *>(w.base);
     v.cnt = reinterpret_cast<unsigned *>(w.base + 256);
-    v.slots = reinterpret_cast<float *>(w.base + 256 + w.nw * sizeof(unsigned));
-    v.part = v.slots + w.nw * 2 * 8;
+    v.slots = reinterpret_cast<float *>(w.base + 256 + cnt_b);
+    v.part = reinterpret_cast<float *>(w.base + 256 + cnt_b + slot_b);
     return v;
 }
 
-int get_workspace(int dev, void *stream, size_t nw, size_t part_f, WsView *out)
+int get_workspace(int dev, void *stream, size_t nw, size_t slot_f, size_t part_f, WsView *out)
 {
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace &w = g_ws[{dev, stream}];
-    if (w.base && w.nw >= nw && w.part_f >= part_f) {
+    if (w.base && w.nw >= nw && w.slot_f >= slot_f && w.part_f >= part_f) {
         *out = ws_view(w);
         return QG_OK;
     }
@@ -111,8 +119,9 @@ int get_workspace(int dev, void *stream, size_t nw, size_t part_f, WsView *out)
         return QG_ERR_CUDA;
     if (cap != cudaStreamCaptureStatusNone) return QG_ERR_NOMEM;  // cannot grow while capturing
     const size_t new_nw = std::max(nw, w.nw);
+    const size_t new_sf = std::max(slot_f, w.slot_f);
     const size_t new_pf = std::max(part_f, w.part_f);
-    const size_t bytes = ws_bytes_for(new_nw, new_pf);
+    const size_t bytes = ws_bytes_for(new_nw, new_sf, new_pf);
     if (w.base) {
         // the old buffer may still be read by work queued on this stream
         if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -133,6 +142,7 @@ int get_workspace(int dev, void *stream, size_t nw, size_t part_f, WsView *out)
     w.base = static_cast<uint8_t *>(p);
     w.bytes = bytes;
     w.nw = new_nw;
+    w.slot_f = new_sf;
     w.part_f = new_pf;
     *out = ws_view(w);
     return QG_OK;
@@ -188,15 +198,144 @@ const void *stream_kernel_ptr(int fmt, int BP, int var)
     case 4: return reinterpret_cast<const void *>(&stream_gemv_kernel<F, 4, V>); \
     default: return reinterpret_cast<const void *>(&stream_gemv_kernel<F, 8, V>); \
     }
+    (void)var;
     if (fmt == kFmtQ8_0) {
         QG_PICK(kFmtQ8_0, kVarDirect)
-    } else if (var == kVarFactored) {
-        QG_PICK(kFmtQ4_K, kVarFactored)
     } else {
         QG_PICK(kFmtQ4_K, kVarDirect)
     }
 #undef QG_PICK
 }
+
+// Plan of the row-per-lane kernel.
+struct RowsPlan {
+    int BP, NW, S, US, Gs, G;
+    size_t smem;
+};
+
+RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di)
+{
+    RowsPlan p;
+    p.BP = padded_cols(B);
+    const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
+    if (fmt == kFmtQ4_K)
+        p.NW = p.BP >= 8 ? RowsWarps<kFmtQ4_K, 8>::value : RowsWarps<kFmtQ4_K, 1>::value;
+    else
+        p.NW = p.BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
+    const size_t ring = (size_t)p.NW * kRowsStages * 32 * UB;
+    const size_t bars = (size_t)p.NW * kRowsStages * 8;
+    const size_t per_unit = (size_t)(512 + 32) * p.BP;  // fp16 x + fp32 sub-block sums
+    const size_t avail = (size_t)di.smem_optin - ring - bars - 128;
+    int64_t fit = (int64_t)(avail / per_unit);
+    if (fit < 1) fit = 1;
+    const int64_t UPR = K / 256;
+    int64_t S = (UPR + fit - 1) / fit;
+    const int64_t US = (UPR + S - 1) / S;
+    S = (UPR + US - 1) / US;
+    p.S = (int)S;
+    p.US = (int)US;
+    p.smem = ring + (size_t)US * per_unit + bars;
+    const int64_t items = ((N + 31) / 32) * US;
+    const int64_t want = std::max<int64_t>(1, (items + p.NW - 1) / p.NW);
+    const int64_t per_slice = std::max<int64_t>(1, di.sms / S);
+    p.Gs = (int)std::min(per_slice, want);
+    p.G = p.Gs * p.S;
+    return p;
+}
+
+const void *rows_kernel_ptr(int fmt, int BP)
+{
+#define QG_PICKR(F)                                                            \
+    switch (BP) {                                                              \
+    case 1: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 1>);    \
+    case 2: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 2>);    \
+    case 4: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 4>);    \
+    default: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 8>);   \
+    }
+    if (fmt == kFmtQ8_0) {
+        QG_PICKR(kFmtQ8_0)
+    } else {
+        QG_PICKR(kFmtQ4_K)
+    }
+#undef QG_PICKR
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link needed).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D view of W for the TMA: rows of K/256 units, u32 elements; a box is 32 rows x one unit.
+int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *map)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return QG_ERR_CUDA;
+    const int inner = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kBoxInner : RowsFmt<kFmtQ8_0>::kBoxInner;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 256) * inner, (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 256) * inner * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)inner, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(W), dims, strides,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
+}
+
+// Launch the row-per-lane kernel (+ the split-K second pass when S > 1) with a given workspace.
+int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
+                cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, const WsView &ws,
+                bool pdl)
+{
+    const void *fn = rows_kernel_ptr(fmt, p.BP);
+    int rc = ensure_smem_attr(dev, fn, di.smem_optin);
+    if (rc != QG_OK) return rc;
+    CUtensorMap map;
+    if ((rc = make_weight_map(W, fmt, N, K, &map)) != QG_OK) return rc;
+    RowsArgs a;
+    a.x = x;
+    a.out = (p.S > 1) ? ws.part : y;
+    a.slots = ws.slots;
+    a.cnt = ws.cnt;
+    a.err = ws.err;
+    a.N = N;
+    a.B = B;
+    a.UPR = (int)(K / 256);
+    a.US = p.US;
+    a.S = p.S;
+    a.Gs = p.Gs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.G);
+    cfg.blockDim = dim3(p.NW * 32);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *args[] = {&a, &map};
+    if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return QG_ERR_CUDA;
+    if (p.S > 1) {
+        const int64_t NB = N * B;
+        const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
+        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(ws.part, y, NB, p.S);
+        if (cudaGetLastError() != cudaSuccess) return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+size_t rows_slot_floats(const RowsPlan &p) { return (size_t)p.G * p.NW * 2 * 32 * p.BP; }
 
 int check_common(const void *W, int fmt, int64_t N, int64_t K)
 {
@@ -230,7 +369,6 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     if (rc != QG_OK) return rc;
     if (B < 1 || B > 8) return QG_ERR_BATCH;
     if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_GENERIC) return QG_ERR_VARIANT;
-    if (fmt == QG_FMT_Q8_0 && variant == QG_VARIANT_FACTORED) return QG_ERR_VARIANT;
     if (N == 0) return QG_OK;
     if (!x || !y) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
@@ -240,13 +378,12 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // streaming kernel needs whole 16-byte-multiple units per row: always for Q4_K, K % 256 == 0
-    // for Q8_0
+    // the streaming kernels need rows of whole 256-weight units (16-byte multiples): always for
+    // Q4_K, K % 256 == 0 for Q8_0
     const bool streamable = (K % 256 == 0);
     int var = variant;
-    if (var == QG_VARIANT_AUTO) var = streamable ? QG_VARIANT_DIRECT : QG_VARIANT_GENERIC;
+    if (var == QG_VARIANT_AUTO) var = streamable ? QG_VARIANT_FACTORED : QG_VARIANT_GENERIC;
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
-    if (fmt == QG_FMT_Q8_0 && var != QG_VARIANT_GENERIC) var = QG_VARIANT_DIRECT;
 
     if (var == QG_VARIANT_GENERIC) {
         rc = launch_rowwise(W, fmt, N, K, x, B, y, st, di);
@@ -257,14 +394,31 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
         return rc;
     }
 
-    const int kvar = (var == QG_VARIANT_FACTORED) ? kVarFactored : kVarDirect;
+    if (var == QG_VARIANT_FACTORED) {
+        const RowsPlan p = make_rows_plan(fmt, N, K, B, di);
+        if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+        WsView ws;
+        const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
+        if ((rc = get_workspace(dev, stream, (size_t)p.G * p.NW, rows_slot_floats(p), part_f, &ws)) !=
+            QG_OK)
+            return rc;
+        if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws, true)) != QG_OK) return rc;
+        t_last_variant = var;
+        t_last_splits = p.S;
+        return QG_OK;
+    }
+
+    // QG_VARIANT_DIRECT: four lanes per unit, correctly rounded fp32 weights
+    const int kvar = kVarDirect;
     const Plan p = make_plan(fmt, kvar, N, K, B, di);
     const void *fn = stream_kernel_ptr(fmt, p.BP, kvar);
     if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     if ((rc = ensure_smem_attr(dev, fn, di.smem_optin)) != QG_OK) return rc;
     WsView ws;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-    if ((rc = get_workspace(dev, stream, (size_t)p.G * kWarps, part_f, &ws)) != QG_OK) return rc;
+    if ((rc = get_workspace(dev, stream, (size_t)p.G * kWarps, (size_t)p.G * kWarps * 2 * 8, part_f,
+                            &ws)) != QG_OK)
+        return rc;
 
     StreamArgs a;
     a.W = static_cast<const uint8_t *>(W);
@@ -280,9 +434,20 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     a.S = p.S;
     a.Gs = p.Gs;
     a.xs_floats = p.xs_floats;
+    // Programmatic dependent launch: the kernel prefetches weights, then waits for the previous
+    // kernel on the stream (griddepcontrol.wait) before it reads x or writes y / the workspace.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.G);
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     void *args[] = {&a};
-    if (cudaLaunchKernel(fn, dim3(p.G), dim3(kWarps * 32), args, p.smem, st) != cudaSuccess)
-        return QG_ERR_CUDA;
+    if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return QG_ERR_CUDA;
     if (p.S > 1) {
         const int64_t NB = N * B;
         const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
@@ -459,47 +624,23 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (K % 256 != 0) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // needs no scratch
 
-    const int kvar = kVarDirect;
-    const Plan p = make_plan(fmt, kvar, N, K, B, di);
+    const RowsPlan p = make_rows_plan(fmt, N, K, B, di);
     if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
-    const size_t nw = (size_t)p.G * kWarps;
+    const size_t nw = (size_t)p.G * p.NW;
+    const size_t slot_f = rows_slot_floats(p);
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-    if (ws_bytes_for(nw, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
-    const void *fn = stream_kernel_ptr(fmt, p.BP, kvar);
-    if ((rc = ensure_smem_attr(dev, fn, di.smem_optin)) != QG_OK) return rc;
+    if (ws_bytes_for(nw, slot_f, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
     uint8_t *base = nullptr;
     if ((rc = noalloc_scratch(dev, &base)) != QG_OK) return rc;
     Workspace w;
     w.base = base;
     w.bytes = QG_NOALLOC_SCRATCH_BYTES;
     w.nw = nw;
+    w.slot_f = slot_f;
     w.part_f = part_f;
     const WsView ws = ws_view(w);
     // The array keeps whatever the previous call left; the arrival counters must start at zero.
     if (cudaMemsetAsync(ws.cnt, 0, nw * sizeof(unsigned), st) != cudaSuccess) return QG_ERR_CUDA;
-
-    StreamArgs a;
-    a.W = static_cast<const uint8_t *>(W);
-    a.x = x;
-    a.out = (p.S > 1) ? ws.part : y;
-    a.slots = ws.slots;
-    a.cnt = ws.cnt;
-    a.err = ws.err;
-    a.N = N;
-    a.B = B;
-    a.UPR = (int)(K / 256);
-    a.US = p.US;
-    a.S = p.S;
-    a.Gs = p.Gs;
-    a.xs_floats = p.xs_floats;
-    void *args[] = {&a};
-    if (cudaLaunchKernel(fn, dim3(p.G), dim3(kWarps * 32), args, p.smem, st) != cudaSuccess)
-        return QG_ERR_CUDA;
-    if (p.S > 1) {
-        const int64_t NB = N * B;
-        const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
-        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(ws.part, y, NB, p.S);
-        if (cudaGetLastError() != cudaSuccess) return QG_ERR_CUDA;
-    }
+    if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws, false)) != QG_OK) return rc;
     return QG_OK;
 }

@@ -274,46 +274,82 @@ __device__ __forceinline__ int xs_index(int j, int c, int iota)
     return ((((j >> 1) * 16 * BP + iota) * 2 + (j & 1)) * 4 + c) * 4;
 }
 
+// Shared-memory position of x[k_local][b] (k_local = 256 j + 64 c + e within the slice).
+template <int BP>
+__device__ __forceinline__ int xs_pos(int k_local, int b)
+{
+    const int j = k_local >> 8, r = k_local & 255;
+    const int c = r >> 6, e = r & 63;
+    const int e4 = e & 3;
+    const int el = ((e4 & 1) << 1) | (e4 >> 1);  // group order (e, e+2, e+1, e+3)
+    return xs_index<BP>(j, c, (e >> 2) * BP + b) + el;
+}
+
+// Scale applied to x in the factored form: 2^(64 - 4k) for the nibble position k its weight is
+// read at (k = 2 * (byte & 1) + high-nibble, byte = the weight's byte within its qs word).
+__device__ __forceinline__ float factored_x_scale(int k_local)
+{
+    const int e = k_local & 63;
+    const int kk = 2 * (e & 1) + (e >> 5);
+    return __uint_as_float((uint32_t)(127 + 64 - 4 * kk) << 23);
+}
+
 template <int FMT, int BP, int VAR>
 __device__ __forceinline__ void stage_x(const StreamArgs &a, int s, int US_s, float *xs, float *xsum)
 {
-    const int nfl = a.xs_floats;
     const int64_t kbase = (int64_t)s * a.US * 256;
-    for (int p = threadIdx.x; p < nfl; p += blockDim.x) {
-        const int el = p & 3;
-        const int c = (p >> 2) & 3;
-        const int jpar = (p >> 4) & 1;
-        const int rest = p >> 5;
-        const int iota = rest % (16 * BP);
-        const int j = (rest / (16 * BP)) * 2 + jpar;
-        const int g = iota / BP;
-        const int b = iota % BP;
-        const int e = 4 * g + ((el & 1) << 1) + (el >> 1);
-        float v = 0.0f;
-        if (j < US_s && b < a.B) {
-            const int64_t k = kbase + (int64_t)j * 256 + 64 * c + e;
-            v = __half2float(__ushort_as_half(a.x[k * a.B + b]));
-            if (VAR == kVarFactored) {
-                const int l = e & 31, half_hi = e >> 5;
-                const int kk = 2 * (l & 1) + half_hi;
-                v *= __uint_as_float((uint32_t)(127 + 64 - 4 * kk) << 23);
+    const int KS = US_s * 256;
+    const int nfl = a.xs_floats;
+    // zero the padding (columns b >= B and the odd unit of the last pair) first
+    if (a.B != BP || (US_s & 1)) {
+        for (int p = threadIdx.x; p < nfl; p += blockDim.x) xs[p] = 0.0f;
+        __syncthreads();
+    }
+    const uint16_t *xsl = a.x + kbase * a.B;
+    const int nh = KS * a.B;  // halves of this slice, a multiple of 8
+    if ((reinterpret_cast<uintptr_t>(xsl) & 15) == 0) {
+        // 16-byte loads: two per thread in flight
+        const int nv = nh >> 3;
+        for (int v0 = threadIdx.x; v0 < nv; v0 += 2 * blockDim.x) {
+            uint4 q[2];
+            const int v1 = v0 + blockDim.x;
+            q[0] = reinterpret_cast<const uint4 *>(xsl)[v0];
+            if (v1 < nv) q[1] = reinterpret_cast<const uint4 *>(xsl)[v1];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int v = u ? v1 : v0;
+                if (v >= nv) break;
+                const uint32_t w4[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    const int flat = 8 * v + h;
+                    const int kl = flat / a.B, b = flat - kl * a.B;
+                    float f = __half2float(__ushort_as_half(
+                        (unsigned short)((h & 1) ? (w4[h >> 1] >> 16) : (w4[h >> 1] & 0xFFFFu))));
+                    if (VAR == kVarFactored) f *= factored_x_scale(kl);
+                    xs[xs_pos<BP>(kl, b)] = f;
+                }
             }
         }
-        xs[p] = v;
+    } else {
+        for (int flat = threadIdx.x; flat < nh; flat += blockDim.x) {
+            const int kl = flat / a.B, b = flat - kl * a.B;
+            float f = __half2float(__ushort_as_half(xsl[flat]));
+            if (VAR == kVarFactored) f *= factored_x_scale(kl);
+            xs[xs_pos<BP>(kl, b)] = f;
+        }
     }
     if (VAR == kVarFactored) {
         // xsum[((j*4 + c)*2 + h)*BP + b] = sum of the 32 unscaled x of sub-block 2c+h of unit j
         const int nsum = US_s * 8 * BP;
         for (int t = threadIdx.x; t < nsum; t += blockDim.x) {
             const int b = t % BP;
-            const int h = (t / BP) & 1;
-            const int c = (t / (2 * BP)) & 3;
-            const int j = t / (8 * BP);
+            const int hc = t / BP;  // (j*4 + c)*2 + h
             float acc = 0.0f;
             if (b < a.B) {
-                const int64_t k0 = kbase + (int64_t)j * 256 + 64 * c + 32 * h;
-                for (int i = 0; i < 32; ++i)
-                    acc += __half2float(__ushort_as_half(a.x[(k0 + i) * a.B + b]));
+                const uint16_t *xp = xsl + (int64_t)(32 * hc) * a.B + b;
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) acc += __half2float(__ushort_as_half(xp[i * a.B]));
             }
             xsum[t] = acc;
         }
@@ -450,7 +486,7 @@ __device__ __forceinline__ int64_t warp_of_item(int64_t t, int64_t Ws, int64_t I
 
 template <int BP>
 __device__ void finish_row(const StreamArgs &a, int s, int64_t row, const float (&tot)[BP],
-                           bool complete, int64_t t0, int64_t w, int64_t Ws, int64_t Is, int US_s)
+                           bool complete, int64_t row0, int64_t w, int64_t Ws, int64_t Is, int US_s)
 {
     float *dst = a.out + ((int64_t)s * a.N + row) * a.B;
     if (complete) {
@@ -458,7 +494,7 @@ __device__ void finish_row(const StreamArgs &a, int s, int64_t row, const float 
         return;
     }
     const int64_t base = (int64_t)s * a.Gs * kWarps;
-    const int side = (row == t0 / US_s) ? 0 : 1;
+    const int side = (row == row0) ? 0 : 1;  // row0: the first row of this warp's range
     float *mine = a.slots + ((base + w) * 2 + side) * BP;
     for (int b = 0; b < BP; ++b) __stcg(mine + b, tot[b]);
     const int64_t wlo = warp_of_item(row * US_s, Ws, Is);
@@ -501,22 +537,24 @@ __global__ void __launch_bounds__(kWarps * 32, 1) stream_gemv_kernel(const Strea
     const int64_t Ws = min((int64_t)a.Gs * kWarps, Is);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t w = (int64_t)cta * kWarps + warp;
+    const bool active = w < Ws;
 
-    stage_x<FMT, BP, VAR>(a, s, US_s, xs, xsum);
-    __syncthreads();
-    if (w >= Ws) return;
-
-    const int64_t t0 = (w * Is) / Ws, t1 = ((w + 1) * Is) / Ws;
-    const int nch = (int)((t1 - t0 + CH - 1) / CH);
+    int64_t t0 = 0, t1 = 0;
+    if (active) {
+        t0 = (w * Is) / Ws;
+        t1 = ((w + 1) * Is) / Ws;
+    }
+    const int L = (int)(t1 - t0);  // units of this warp's range
+    const int nch = (L + CH - 1) / CH;
     uint8_t *myring = ring + warp * kStages * CHB;
     const uint32_t bar0 = smem_u32(bars + warp * kStages);
-    const uint64_t policy = evict_first_policy();
 
     auto issue = [&](int i) {
         const int64_t ta = t0 + (int64_t)i * CH;
         const int64_t tb = min(ta + CH, t1);
         const uint32_t bar = bar0 + 8 * (i % kStages);
         const uint32_t dst0 = smem_u32(myring + (i % kStages) * CHB);
+        const uint64_t policy = evict_first_policy();
         mbar_arrive_expect_tx(bar, (uint32_t)((tb - ta) * UB));
         if (a.S == 1) {
             bulk_g2s(dst0, a.W + ta * UB, (uint32_t)((tb - ta) * UB), bar, policy);
@@ -532,21 +570,41 @@ __global__ void __launch_bounds__(kWarps * 32, 1) stream_gemv_kernel(const Strea
         }
     };
 
-    if (lane == 0) {
+    // 1. Weight prefetch: fill the ring.  W does not depend on the kernel before this one on the
+    //    stream, so this may overlap that kernel's tail (programmatic dependent launch).
+    if (active && lane == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         for (int i = 0; i < kStages && i < nch; ++i) issue(i);
     }
+    // 2. Let the next kernel on the stream begin its own prefetch as SMs free up, then wait for
+    //    the previous kernel's results (x) before reading x or writing y / the workspace.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // 3. x for this slice -> shared memory (fp32, consumer order)
+    stage_x<FMT, BP, VAR>(a, s, US_s, xs, xsum);
+    __syncthreads();
+    if (!active) return;
     __syncwarp();
 
     const int c = lane & 3;
-    const int usub = lane >> 2;  // unit of this lane within a pass of 8 units
+    const int g = lane >> 2;  // unit of this lane within a pass of 8 units
+    const int64_t row0 = t0 / US_s;
+    int64_t row = row0;
+    int j = (int)(t0 - row0 * US_s);  // position of the next pass's first unit within its row
+    bool row_started_here = (j == 0);
     float acc[BP];
 #pragma unroll
     for (int b = 0; b < BP; ++b) acc[b] = 0.0f;
-    int64_t cur_row = t0 / US_s;
-    int64_t row_first = cur_row * US_s, row_end = row_first + US_s;
-    int pj = (int)(t0 - row_first);  // unit (within its virtual row) of the pass's first item
+
+    auto flush = [&](bool complete) {
+        float tot[BP];
+#pragma unroll
+        for (int b = 0; b < BP; ++b) tot[b] = warp_sum(acc[b]);
+        if (lane == 0) finish_row<BP>(a, s, row, tot, complete, row0, w, Ws, Is, US_s);
+#pragma unroll
+        for (int b = 0; b < BP; ++b) acc[b] = 0.0f;
+    };
 
     for (int i = 0; i < nch; ++i) {
         const bool ok = mbar_wait_bounded(bar0 + 8 * (i % kStages), (uint32_t)((i / kStages) & 1));
@@ -560,57 +618,54 @@ __global__ void __launch_bounds__(kWarps * 32, 1) stream_gemv_kernel(const Strea
             __syncwarp();
             return;
         }
-        const int64_t ta = t0 + (int64_t)i * CH;
-        const int64_t tb = min(ta + CH, t1);
         const uint8_t *stage = myring + (i % kStages) * CHB;
-        for (int64_t pa = ta; pa < tb; pa += 8) {
-            const int64_t pe = min(pa + 8, tb);
-            const int64_t t = pa + usub;
+        const int nu = min(CH, L - i * CH);  // units in this chunk
+        for (int p = 0; p < nu; p += 8) {
+            const int pn = min(8, nu - p);  // units in this pass (8 except at the range's end)
+            // the lane's unit position within its row, and how many rows past the current one
+            int jj = j + g, rel = 0;
+            while (jj >= US_s) {
+                jj -= US_s;
+                ++rel;
+            }
             float v[BP];
 #pragma unroll
             for (int b = 0; b < BP; ++b) v[b] = 0.0f;
-            // unit index of this lane's item within its virtual row, and how many rows it is
-            // past the pass's first row
-            int tj = pj + usub, rel = 0;
-            while (tj >= US_s) {
-                tj -= US_s;
-                ++rel;
-            }
-            if (t < pe) {
-                const uint8_t *u = stage + (t - ta) * UB;
+            if (g < pn) {
+                const uint8_t *u = stage + (p + g) * UB;
                 if (FMT == kFmtQ4_K)
-                    q4k_unit<BP, VAR>(u, c, xs, xsum, tj, v);
+                    q4k_unit<BP, VAR>(u, c, xs, xsum, jj, v);
                 else
-                    q8_0_unit<BP>(u, c, xs, tj, v);
+                    q8_0_unit<BP>(u, c, xs, jj, v);
             }
-            if (pe < row_end) {
+            if (j + pn < US_s) {
+                // the current row continues past this pass
 #pragma unroll
                 for (int b = 0; b < BP; ++b) acc[b] += v[b];
+                j += pn;
             } else {
-                // the current row ends inside this pass: hand out contributions row by row
-                int r = 0;
+                // the current row ends inside this pass: hand contributions out row by row
+                int k = 0, end = US_s - j;  // pass offset where row k ends
                 while (true) {
-                    if (rel == r) {
+                    if (rel == k) {
 #pragma unroll
                         for (int b = 0; b < BP; ++b) acc[b] += v[b];
                     }
-                    if (row_end > pe) break;
-                    float tot[BP];
-#pragma unroll
-                    for (int b = 0; b < BP; ++b) tot[b] = warp_sum(acc[b]);
-                    if (lane == 0)
-                        finish_row<BP>(a, s, cur_row, tot, row_first >= t0, t0, w, Ws, Is, US_s);
-#pragma unroll
-                    for (int b = 0; b < BP; ++b) acc[b] = 0.0f;
-                    ++cur_row;
-                    ++r;
-                    row_first = row_end;
-                    row_end += US_s;
-                    if (row_first >= pe) break;
+                    if (end > pn) {
+                        j = pn - (end - US_s);
+                        break;
+                    }
+                    flush(row_started_here);
+                    ++row;
+                    row_started_here = true;
+                    ++k;
+                    if (end == pn) {
+                        j = 0;
+                        break;
+                    }
+                    end += US_s;
                 }
             }
-            pj += 8;
-            while (pj >= US_s) pj -= US_s;
         }
         __syncwarp();
         if (lane == 0 && i + kStages < nch) {
@@ -618,13 +673,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) stream_gemv_kernel(const Strea
             issue(i + kStages);
         }
     }
-    if (row_first < t1) {
-        // the warp's range ends inside cur_row: hand its partial to the row's last arriver
-        float tot[BP];
-#pragma unroll
-        for (int b = 0; b < BP; ++b) tot[b] = warp_sum(acc[b]);
-        if (lane == 0) finish_row<BP>(a, s, cur_row, tot, false, t0, w, Ws, Is, US_s);
-    }
+    // the warp's range ends inside the current row: hand its partial to the row's last arriver
+    if (j > 0) flush(false);
 }
 
 // Second pass of split-K: y[n][b] = sum over slices s = 0..S-1 (in that order) of part[s][n][b].

@@ -129,10 +129,9 @@ def test_gemv_zero_rows_is_a_noop(L):
 
 
 def test_variant_checks(L):
-    # FACTORED is Q4_K only; unknown variants are rejected
-    assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_FACTORED) == \
-        qg.QG_ERR_VARIANT
+    # unknown variants are rejected; the streaming variants need rows of whole 256-weight units
     assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 7) == qg.QG_ERR_VARIANT
+    assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, -1) == qg.QG_ERR_VARIANT
 
 
 def test_dequant_rejects_bad_arguments(L):

@@ -305,3 +305,23 @@ def test_streams_do_not_interfere(dev, orc):
     for W, x, y, N, K, B in outs:
         yref, A = orc.gemv(W, Q4_K, N, K, x, B)
         assert_within(y.cpu().numpy(), yref, A, "two streams")
+
+
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_x_not_16_byte_aligned(dev, orc, B):
+    """x only 2-byte aligned: the staging falls back to element loads; results unchanged."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    N, K = 150, 2560
+    W = synth.q4k_weights(N, K, seed=B)
+    x = synth.activations(K, B, seed=B)
+    buf = torch.zeros(K * B + 8, dtype=torch.int16, device=dev)
+    buf[1:1 + K * B] = torch.from_numpy(x.view(np.int16).reshape(-1)).to(dev)
+    xd = buf[1:1 + K * B]
+    assert xd.data_ptr() % 16 != 0
+    yref, A = orc.gemv(W, Q4_K, N, K, x, B)
+    for v in (1, 2):
+        y = torch.empty((N, B), dtype=torch.float32, device=dev)
+        qg.qg_gemv_variant(_t(W, dev), Q4_K, N, K, xd, B, y, None, v)
+        torch.cuda.synchronize()
+        assert_within(y.cpu().numpy(), yref, A, f"unaligned x v{v}")

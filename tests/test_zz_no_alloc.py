@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 CASES = [
     (12, 17408, 5120, 1),   # FFN gate at B=1, rows split between warps
-    (12, 300, 5120, 8),     # x for the whole K does not fit: split-K partial rows in scratch
+    (12, 300, 17408, 8),    # x for the whole K does not fit: split-K partial rows in scratch
     (12, 5120, 17408, 1),   # long-K down projection
     (8, 1000, 5120, 2),     # Q8_0
 ]
@@ -56,5 +56,5 @@ def test_noalloc_rejects_oversized_call(dev):
     """A call whose split-K partial rows exceed the fixed array is refused before any launch."""
     import quant_dequant_gemv_q4_b200 as qg
     fake = 1 << 20  # aligned, never dereferenced: the size check happens first
-    rc = qg.lib().qg_gemv_noalloc(fake, 12, 400000, 5120, fake, 8, fake, None)
+    rc = qg.lib().qg_gemv_noalloc(fake, 12, 400000, 17408, fake, 8, fake, None)
     assert rc == qg.QG_ERR_SCRATCH
