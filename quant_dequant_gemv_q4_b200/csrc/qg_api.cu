@@ -207,40 +207,55 @@ const void *stream_kernel_ptr(int fmt, int BP, int var)
 #undef QG_PICK
 }
 
-// Plan of the row-per-lane kernel.
+// Plan of the row-band kernel.
 struct RowsPlan {
-    int BP, NW, S, US, Gs, G;
+    int BP, NW, S, US, Gs, G, red_floats;
     size_t smem;
 };
 
 RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di)
 {
-    RowsPlan p;
-    p.BP = padded_cols(B);
+    RowsPlan best{};
+    double best_util = -1.0;
+    const int BP = padded_cols(B);
     const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
+    int NW;
     if (fmt == kFmtQ4_K)
-        p.NW = p.BP >= 8 ? RowsWarps<kFmtQ4_K, 8>::value : RowsWarps<kFmtQ4_K, 1>::value;
+        NW = BP >= 8 ? RowsWarps<kFmtQ4_K, 8>::value : RowsWarps<kFmtQ4_K, 1>::value;
     else
-        p.NW = p.BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
-    const size_t ring = (size_t)p.NW * kRowsStages * 32 * UB;
-    const size_t bars = (size_t)p.NW * kRowsStages * 8;
-    const size_t per_unit = (size_t)(512 + 32) * p.BP;  // fp16 x + fp32 sub-block sums
-    const size_t avail = (size_t)di.smem_optin - ring - bars - 128;
-    int64_t fit = (int64_t)(avail / per_unit);
-    if (fit < 1) fit = 1;
+        NW = BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
+    const size_t ring = (size_t)NW * kRowsStages * 32 * UB;
+    const size_t bars = (size_t)NW * kRowsStages * 8;
     const int64_t UPR = K / 256;
-    int64_t S = (UPR + fit - 1) / fit;
-    const int64_t US = (UPR + S - 1) / S;
-    S = (UPR + US - 1) / US;
-    p.S = (int)S;
-    p.US = (int)US;
-    p.smem = ring + (size_t)US * per_unit + bars;
-    const int64_t items = ((N + 31) / 32) * US;
-    const int64_t want = std::max<int64_t>(1, (items + p.NW - 1) / p.NW);
-    const int64_t per_slice = std::max<int64_t>(1, di.sms / S);
-    p.Gs = (int)std::min(per_slice, want);
-    p.G = p.Gs * p.S;
-    return p;
+    // K slices: the fewest for which x fits in shared memory and the row bands keep at least 85%
+    // of their 32-row lanes busy (bands of N*S/SMs rows); otherwise the best such fraction
+    for (int64_t S0 = 1; S0 <= std::min<int64_t>(UPR, 64); ++S0) {
+        const int64_t US = (UPR + S0 - 1) / S0;
+        const int64_t S = (UPR + US - 1) / US;
+        if (S != S0) continue;  // the same slicing as a smaller S0
+        const int64_t Gs = std::max<int64_t>(1, std::min<int64_t>(di.sms / S, N));
+        // partial rows are kept in shared memory only when a band has several K parts, and then
+        // there is at most one (row group, part) pair per warp
+        const int red = NW * 32 * BP;
+        const size_t smem = ring + (size_t)US * (512 + 32) * BP + (size_t)red * sizeof(float) + bars;
+        if (smem + 128 > (size_t)di.smem_optin) continue;
+        const double util = ((double)N / (double)Gs) / (32.0 * (double)((N / Gs + 31) / 32 > 0 ? (N / Gs + 31) / 32 : 1));
+        RowsPlan p;
+        p.BP = BP;
+        p.NW = NW;
+        p.S = (int)S;
+        p.US = (int)US;
+        p.Gs = (int)Gs;
+        p.G = (int)(Gs * S);
+        p.red_floats = red;
+        p.smem = smem;
+        if (util >= 0.85) return p;
+        if (util > best_util) {
+            best_util = util;
+            best = p;
+        }
+    }
+    return best;  // smem == 0 if nothing fits
 }
 
 const void *rows_kernel_ptr(int fmt, int BP)
@@ -276,15 +291,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 2-D view of W for the TMA: rows of K/256 units, u32 elements; a box is 32 rows x one unit.
+// 2-D view of W for the TMA: N rows of K/256 units in u32 elements; a box is 32 rows x one unit.
 int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *map)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return QG_ERR_CUDA;
-    const int inner = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kBoxInner : RowsFmt<kFmtQ8_0>::kBoxInner;
-    const cuuint64_t dims[2] = {(cuuint64_t)(K / 256) * inner, (cuuint64_t)N};
-    const cuuint64_t strides[1] = {(cuuint64_t)(K / 256) * inner * 4};
-    const cuuint32_t box[2] = {(cuuint32_t)inner, 32};
+    const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 256) * (UB / 4), (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 256) * UB};
+    const cuuint32_t box[2] = {(cuuint32_t)(UB / 4), 32};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(W), dims, strides,
                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -292,10 +307,11 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
     return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
 }
 
-// Launch the row-per-lane kernel (+ the split-K second pass when S > 1) with a given workspace.
+// Launch the row-band kernel (+ the split-K second pass when S > 1).  `err` is the device error
+// word; `part` holds S*N*B floats when S > 1.
 int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
-                cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, const WsView &ws,
-                bool pdl)
+                cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, int *err,
+                float *part, bool pdl)
 {
     const void *fn = rows_kernel_ptr(fmt, p.BP);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
@@ -304,16 +320,15 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     if ((rc = make_weight_map(W, fmt, N, K, &map)) != QG_OK) return rc;
     RowsArgs a;
     a.x = x;
-    a.out = (p.S > 1) ? ws.part : y;
-    a.slots = ws.slots;
-    a.cnt = ws.cnt;
-    a.err = ws.err;
+    a.out = (p.S > 1) ? part : y;
+    a.err = err;
     a.N = N;
     a.B = B;
     a.UPR = (int)(K / 256);
     a.US = p.US;
     a.S = p.S;
     a.Gs = p.Gs;
+    a.red_floats = p.red_floats;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
     cfg.blockDim = dim3(p.NW * 32);
@@ -329,13 +344,11 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     if (p.S > 1) {
         const int64_t NB = N * B;
         const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
-        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(ws.part, y, NB, p.S);
+        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(part, y, NB, p.S);
         if (cudaGetLastError() != cudaSuccess) return QG_ERR_CUDA;
     }
     return QG_OK;
 }
-
-size_t rows_slot_floats(const RowsPlan &p) { return (size_t)p.G * p.NW * 2 * 32 * p.BP; }
 
 int check_common(const void *W, int fmt, int64_t N, int64_t K)
 {
@@ -396,13 +409,12 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
 
     if (var == QG_VARIANT_FACTORED) {
         const RowsPlan p = make_rows_plan(fmt, N, K, B, di);
-        if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+        if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
         WsView ws;
         const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-        if ((rc = get_workspace(dev, stream, (size_t)p.G * p.NW, rows_slot_floats(p), part_f, &ws)) !=
-            QG_OK)
+        if ((rc = get_workspace(dev, stream, 0, 0, part_f, &ws)) != QG_OK) return rc;
+        if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.part, true)) != QG_OK)
             return rc;
-        if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws, true)) != QG_OK) return rc;
         t_last_variant = var;
         t_last_splits = p.S;
         return QG_OK;
@@ -625,22 +637,18 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     if (K % 256 != 0) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // needs no scratch
 
     const RowsPlan p = make_rows_plan(fmt, N, K, B, di);
-    if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
-    const size_t nw = (size_t)p.G * p.NW;
-    const size_t slot_f = rows_slot_floats(p);
+    if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-    if (ws_bytes_for(nw, slot_f, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
+    if (ws_bytes_for(0, 0, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
     uint8_t *base = nullptr;
     if ((rc = noalloc_scratch(dev, &base)) != QG_OK) return rc;
     Workspace w;
     w.base = base;
     w.bytes = QG_NOALLOC_SCRATCH_BYTES;
-    w.nw = nw;
-    w.slot_f = slot_f;
-    w.part_f = part_f;
     const WsView ws = ws_view(w);
-    // The array keeps whatever the previous call left; the arrival counters must start at zero.
-    if (cudaMemsetAsync(ws.cnt, 0, nw * sizeof(unsigned), st) != cudaSuccess) return QG_ERR_CUDA;
-    if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws, false)) != QG_OK) return rc;
+    // Every element of the split-K partial rows is written before it is read, so nothing in the
+    // array has to be cleared between calls.
+    if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.part, false)) != QG_OK)
+        return rc;
     return QG_OK;
 }
