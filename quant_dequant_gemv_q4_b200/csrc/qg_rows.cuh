@@ -354,7 +354,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         }
     };
 
-    // 1. weight prefetch (independent of the previous kernel on the stream)
+    // 1. weight prefetch (independent of the previous kernel on the stream): the first steps
+    //    into the ring
     if (nsteps > 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
