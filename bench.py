@@ -35,7 +35,7 @@ import numpy as np  # noqa: E402
 
 from quant_dequant_gemv_q4_b200 import synth  # noqa: E402
 
-METRIC = "Q4_K GEMV effective HBM GB/s and % of B200 HBM roofline (us/call), B=1 and B=8"
+METRIC = "Q4_K GEMV effective HBM GB/s and % of B200 HBM roofline (\u00b5s/call), B=1 and B=8"
 UNIT = "GB/s"
 HEADLINE = synth.Gemv("ffn_gate", synth.Q4_K, 17408, 5120, 1, 0)
 HEADLINE_B8 = synth.Gemv("ffn_gate_b8", synth.Q4_K, 17408, 5120, 8, 0)
@@ -49,6 +49,12 @@ def kernel_source_hash() -> str:
         with open(os.path.join(ROOT, "quant_dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def bench_config(world: int) -> dict:
+    """The workload both arms (this library and the CPU oracle) report on."""
+    return {"workload": "ffn_gate Q4_K GEMV N=17408 K=5120 B=1, one call per step",
+            "global_batch": 1, "seq_len": 1, "parallelism": f"replicas x{world}"}
 
 
 def load_peaks() -> dict:
@@ -374,7 +380,7 @@ def run_reference(args):
     oracle.gemv(W, call.fmt, call.N, call.K, x, call.B, rows=np.arange(64))
     per_row = (time.perf_counter() - t0) / 64
     total = max(1, args.steps + args.warmup)
-    rows = int(max(1, min(call.N, 60.0 / total / per_row)))
+    rows = int(max(1, min(call.N, args.ref_seconds / total / per_row)))
 
     def step(s):
         sel = (np.arange(rows) + s * rows) % call.N
@@ -396,14 +402,36 @@ def run_reference(args):
         "ms_per_step": round(secs * 1e3 / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle dot; fp32 weights)",
         "data": "synthetic (seeded Q4_K bytes, x ~ N(0,1) fp16)",
-        "config": {"workload": "ffn_gate Q4_K GEMV N=17408 K=5120 B=1 (CPU oracle, row sample)",
-                   "global_batch": 1, "seq_len": 1, "parallelism": "replicas"},
+        "config": bench_config(world),
         "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(value, 4),
                          "unit": UNIT},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ncu_case(args):
+    """The headline tensor, one copy on the device: 3 launches at B=1, then 3 at B=8."""
+    import torch
+    from quant_dequant_gemv_q4_b200 import build as qbuild
+    qbuild.build()
+    import quant_dequant_gemv_q4_b200 as qg
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    for call in (HEADLINE, HEADLINE_B8):
+        wl = synth.Workload("ncu", HEADLINE_SEED, (call,))
+        W, x = wl.inputs(call)
+        Wd = torch.from_numpy(W).to(device)
+        xd = torch.from_numpy(x.view(np.uint16)).to(device)
+        yd = torch.empty((call.N, call.B), dtype=torch.float32, device=device)
+        s = torch.cuda.current_stream()
+        for _ in range(3):
+            qg.qg_gemv_variant(Wd, call.fmt, call.N, call.K, xd, call.B, yd, s, args.variant)
+        torch.cuda.synchronize()
+        del Wd, xd, yd
+    print(json.dumps({"ncu_case": "done", "kernel_hash": kernel_source_hash()}), flush=True)
     return 0
 
 
@@ -419,11 +447,18 @@ def main(argv=None):
     ap.add_argument("--no-table", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: CPU seconds the whole warm-up + timed run takes")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="launch the headline call 3x at B=1 then 3x at B=8 on one weight copy "
+                         "and exit (the small case an ncu capture runs; nothing is timed)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
         return run_reference(args)
+    if args.ncu_case:
+        return run_ncu_case(args)
 
     import torch
     import torch.distributed as dist
@@ -533,12 +568,10 @@ def main(argv=None):
         "dtype": "f32 (Q4_K weights, f16 x, f32 accumulate)",
         "data": "synthetic (seeded Q4_K bytes with the workload's d/dmin/sc/m/q distributions, "
                 "x ~ N(0,1) fp16)",
-        "config": {"workload": "ffn_gate Q4_K GEMV N=17408 K=5120 B=1 (one call per step); "
-                               "B=8 on the same tensor in 'b8'",
-                   "global_batch": 1, "seq_len": 1, "parallelism": f"replicas x{world}",
-                   "l2": f"{cs_copies_note(HEADLINE, l2)}; L2 {l2 >> 20} MiB",
-                   "timing": "CUDA graphs of one call per weight copy, CUDA events on the "
-                             "launching stream"},
+        "config": bench_config(world),
+        "timing": {"l2": f"{cs_copies_note(HEADLINE, l2)}; L2 {l2 >> 20} MiB",
+                   "how": "CUDA graphs of one call per weight copy, CUDA events on the "
+                          "launching stream; B=8 on the same tensor in 'b8'"},
         "us_per_call": round(secs_max * 1e6 / args.steps, 3),
         "frac_of_hbm": round(value / world / hbm, 4),
         "variant": variant_used,
