@@ -45,9 +45,11 @@ FALLBACK_HBM_GBS = 6650.0
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("qg_device.cuh", "qg_rows.cuh", "qg_api.cu"):
-        with open(os.path.join(ROOT, "quant_dequant_gemv_q4_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "quant_dequant_gemv_q4_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".cpp", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
     return h.hexdigest()[:16]
 
 

@@ -68,8 +68,8 @@ enum {
     QG_ERR_SCRATCH = 10 /* qg_gemv_noalloc: the call needs more scratch than its fixed array holds */
 };
 
-/* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses:
- * FACTORED when K % 256 == 0, else GENERIC. */
+/* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses: when
+ * K % 256 == 0, TENSOR for Q4_K with B >= 2 and FACTORED otherwise; GENERIC when K % 256 != 0. */
 enum {
     QG_VARIANT_AUTO = 0,
     /* Each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m) (Q4_K; the
@@ -84,7 +84,12 @@ enum {
     QG_VARIANT_FACTORED = 2,
     /* Any format and shape: one warp per row, plain loads, no shared-memory staging.  Used by
      * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0). */
-    QG_VARIANT_GENERIC = 3
+    QG_VARIANT_GENERIC = 3,
+    /* Q4_K only: the FACTORED arithmetic with the q*x products on the tensor cores
+     * (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the instruction are
+     * the B columns of x), so B = 1..8 cost the same.  Same error bound as FACTORED.  Requires
+     * K % 256 == 0. */
+    QG_VARIANT_TENSOR = 4
 };
 
 /* Bytes of an N x K tensor in format fmt; 0 if fmt is unknown, N < 0, K < 1 or K is not a
@@ -103,8 +108,9 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
 int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
             void *stream);
 
-/* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant or
- * for DIRECT / FACTORED when K % 256 != 0.  Every variant takes both formats. */
+/* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant,
+ * for DIRECT / FACTORED / TENSOR when K % 256 != 0, and for TENSOR with Q8_0.  The other variants
+ * take both formats. */
 int qg_gemv_variant(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
                     float *y, void *stream, int variant);
 
@@ -124,7 +130,7 @@ int qg_pack_reference(int fmt, int64_t N, int64_t K, const uint16_t *d, const ui
                       const uint8_t *sc, const uint8_t *m, const void *q, void *out);
 
 /* Kernel variant launched by the last successful qg_gemv / qg_gemv_variant of the calling host
- * thread (a launch witness: QG_VARIANT_DIRECT, _FACTORED or _GENERIC), 0 if none yet. */
+ * thread (a launch witness: QG_VARIANT_DIRECT, _FACTORED, _GENERIC or _TENSOR), 0 if none yet. */
 int qg_last_variant(void);
 
 /* Number of K slices the last GEMV of the calling thread used (1 = no split-K second pass). */

@@ -13,6 +13,7 @@
 #include "../../include/qg.h"
 #include "qg_device.cuh"
 #include "qg_rows.cuh"
+#include "qg_mma.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -211,20 +212,24 @@ const void *stream_kernel_ptr(int fmt, int BP, int var)
 struct RowsPlan {
     int BP, NW, S, US, Gs, G, red_floats;
     size_t smem;
+    bool tensor;  // mma_gemv_kernel instead of rows_gemv_kernel
 };
 
-RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di)
+RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di, bool tensor)
 {
     RowsPlan best{};
     double best_util = -1.0;
     const int BP = padded_cols(B);
     const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
     int NW;
-    if (fmt == kFmtQ4_K)
+    if (tensor)
+        NW = BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
+    else if (fmt == kFmtQ4_K)
         NW = BP >= 8 ? RowsWarps<kFmtQ4_K, 8>::value : RowsWarps<kFmtQ4_K, 1>::value;
     else
         NW = BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
     const size_t ring = (size_t)NW * kRowsStages * 32 * UB;
+    const size_t tabs = tensor ? (size_t)NW * 256 * sizeof(float) : 0;  // per-warp scale tables
     const size_t bars = (size_t)NW * kRowsStages * 8;
     const int64_t UPR = K / 256;
     // K slices: the fewest for which x fits in shared memory and the row bands keep at least 85%
@@ -237,7 +242,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         // partial rows are kept in shared memory only when a band has several K parts, and then
         // there is at most one (row group, part) pair per warp
         const int red = NW * 32 * BP;
-        const size_t smem = ring + (size_t)US * (512 + 32) * BP + (size_t)red * sizeof(float) + bars;
+        const size_t smem = ring + (size_t)US * (512 + 32) * BP + tabs + (size_t)red * sizeof(float) + bars;
         if (smem + 128 > (size_t)di.smem_optin) continue;
         const double util = ((double)N / (double)Gs) / (32.0 * (double)((N / Gs + 31) / 32 > 0 ? (N / Gs + 31) / 32 : 1));
         RowsPlan p;
@@ -249,6 +254,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         p.G = (int)(Gs * S);
         p.red_floats = red;
         p.smem = smem;
+        p.tensor = tensor;
         if (util >= 0.85) return p;
         if (util > best_util) {
             best_util = util;
@@ -258,8 +264,16 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     return best;  // smem == 0 if nothing fits
 }
 
-const void *rows_kernel_ptr(int fmt, int BP)
+const void *rows_kernel_ptr(int fmt, int BP, bool tensor)
 {
+    if (tensor) {
+        switch (BP) {
+        case 1: return reinterpret_cast<const void *>(&mma_gemv_kernel<1>);
+        case 2: return reinterpret_cast<const void *>(&mma_gemv_kernel<2>);
+        case 4: return reinterpret_cast<const void *>(&mma_gemv_kernel<4>);
+        default: return reinterpret_cast<const void *>(&mma_gemv_kernel<8>);
+        }
+    }
 #define QG_PICKR(F)                                                            \
     switch (BP) {                                                              \
     case 1: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 1>);    \
@@ -313,7 +327,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
                 cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, int *err,
                 float *part, bool pdl)
 {
-    const void *fn = rows_kernel_ptr(fmt, p.BP);
+    const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
     if (rc != QG_OK) return rc;
     CUtensorMap map;
@@ -375,28 +389,38 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
     return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
+// The variant qg_gemv takes: the tensor-core kernel for Q4_K with B >= 2 (the CUDA-core kernel
+// spends one FMA per weight and column, so its cost grows with B while the tensor-core kernel's
+// does not; at B = 1 the CUDA-core kernel is faster), the CUDA-core row kernel otherwise, and the
+// generic kernel for rows that are not whole 256-weight units.
+int auto_variant(int fmt, int64_t K, int B)
+{
+    if (K % 256 != 0) return QG_VARIANT_GENERIC;
+    return (fmt == QG_FMT_Q4_K && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
+}
+
 int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
               void *stream, int variant)
 {
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
     if (B < 1 || B > 8) return QG_ERR_BATCH;
-    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_GENERIC) return QG_ERR_VARIANT;
+    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TENSOR) return QG_ERR_VARIANT;
     if (N == 0) return QG_OK;
     if (!x || !y) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
         return QG_ERR_ALIGN;
-    DeviceInfo di;
-    int dev = 0;
-    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-
     // the streaming kernels need rows of whole 256-weight units (16-byte multiples): always for
     // Q4_K, K % 256 == 0 for Q8_0
     const bool streamable = (K % 256 == 0);
     int var = variant;
-    if (var == QG_VARIANT_AUTO) var = streamable ? QG_VARIANT_FACTORED : QG_VARIANT_GENERIC;
+    if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
+    if (var == QG_VARIANT_TENSOR && fmt != QG_FMT_Q4_K) return QG_ERR_VARIANT;
+    DeviceInfo di;
+    int dev = 0;
+    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     if (var == QG_VARIANT_GENERIC) {
         rc = launch_rowwise(W, fmt, N, K, x, B, y, st, di);
@@ -407,8 +431,8 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
         return rc;
     }
 
-    if (var == QG_VARIANT_FACTORED) {
-        const RowsPlan p = make_rows_plan(fmt, N, K, B, di);
+    if (var == QG_VARIANT_FACTORED || var == QG_VARIANT_TENSOR) {
+        const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
         if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
         WsView ws;
         const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
@@ -634,9 +658,10 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (K % 256 != 0) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // needs no scratch
+    const int var = auto_variant(fmt, K, B);
+    if (var == QG_VARIANT_GENERIC) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // no scratch
 
-    const RowsPlan p = make_rows_plan(fmt, N, K, B, di);
+    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
     if (ws_bytes_for(0, 0, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;

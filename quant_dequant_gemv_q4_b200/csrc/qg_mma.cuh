@@ -1,0 +1,331 @@
+// qg_mma.cuh -- the tensor-core streaming GEMV of libqg (sm_100a) for Q4_K, B = 1..8 columns.
+//
+// Operation (HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle), second prompt, "SPEC"):
+//   y[n,b] = sum_k dequant(W)[n,k] * x[k,b], fp32 accumulation ("PHYSICS & CONTRACT"), Q4_K
+//   w = d*sc*q - dmin*m ("QUANTIZATION MIX").
+//
+// Why tensor cores here.  With B columns, the CUDA-core kernel spends one fp32 FMA per weight and
+// column, so at B = 8 the FMA pipe, not HBM, bounds it.  mma.sync.m16n8k16 (f16 x f16 -> f32)
+// multiplies a 16-row x 16-weight tile of 4-bit integers by a 16 x 8 tile of x in one
+// instruction: the 8 columns of the instruction are the B <= 8 columns of x, so B = 1..8 cost the
+// same tensor work, and the weights are unpacked once for all columns.  Products are exact
+// (integers up to 15 times fp16 x) and the sums are fp32, so the arithmetic is the factored form
+// of the CUDA-core kernel:
+//   sum_i w_i x_i = sum_j [ D_j * sum_{i in j} q_i x_i  -  M_j * sum_{i in j} x_i ],
+//   D_j = d*sc_j, M_j = dmin*m_j (exact in fp32), j = 32-weight sub-block.
+//
+// Mapping.  The grid, row bands, (row group, K part) pairs and the per-warp ring of 2-D TMA
+// boxes (32 rows x one 144-byte superblock) are those of the CUDA-core kernel (qg_rows.cuh).  Per
+// step a warp multiplies its 32 rows as two 16-row tiles:
+//   A fragment (rows g and g+8 of a tile, lane = 4g + t): word 2t+h of the 32-byte chunk c of the
+//     row; (word & 0x000F000F) holds the low nibbles of bytes 0 and 2 as fp16 subnormals q*2^-24
+//     (sub-block 2c), (word & 0x00F000F0) the high nibbles as q*2^-20 (sub-block 2c+1), and the
+//     same masks on word >> 8 give bytes 1 and 3.  So one 32-bit word feeds four A registers.
+//   B fragment: x in the matching order, staged once per CTA (mma_stage_x).
+//   C fragment: rows g, g+8 x columns 2t, 2t+1, fresh per (chunk, tile, nibble half), then scaled
+//     by D_j of its row and added to the warp's accumulators.
+// The scales come from a per-warp table: lane l decodes row l's header (as in the CUDA-core
+// kernel), writes D_j for its row, and folds -M_j * sum(x over j) into its own per-row sum.
+#pragma once
+
+#include "qg_rows.cuh"
+
+namespace qg {
+
+// warps per CTA of the tensor-core kernel (shared memory: ring + x fragments + tables)
+template <int BP> struct MmaWarps {
+    static constexpr int value = BP >= 8 ? 12 : 16;
+};
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// x fragments.  For unit j of the slice, chunk c, nibble half lh (0 low, 1 high), k-step h,
+// column col < BP and t = lane % 4, one uint2 holds
+//   { (x[e], x[e+2]), (x[e+1], x[e+3]) },  e = 256j + 64c + 32lh + 8t + 4h,
+// the weights that word 2t+h of chunk c contributes in that nibble half, in the order the masks
+// produce them.  Index (in uint2):
+__device__ __forceinline__ int mma_xf_idx(int j, int c, int lh, int h, int col, int t, int BP)
+{
+    return ((((j * 4 + c) * 2 + lh) * 2 + h) * BP + col) * 4 + t;
+}
+
+template <int BP>
+__device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, uint2 *xf,
+                                            float *xsum)
+{
+    const uint16_t *xsl = a.x + (int64_t)s * a.US * 256 * a.B;
+    const int nfrag = a.US * 16 * BP * 4;
+    for (int idx = threadIdx.x; idx < nfrag; idx += blockDim.x) {
+        const int t = idx & 3;
+        int r = idx >> 2;
+        const int col = r % BP;
+        r /= BP;
+        const int h = r & 1, lh = (r >> 1) & 1, c = (r >> 2) & 3, j = r >> 4;
+        uint32_t v[4] = {0u, 0u, 0u, 0u};
+        if (j < US_s && col < a.B) {
+            const int e = j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = xsl[(int64_t)(e + i) * a.B + col];
+        }
+        xf[idx] = make_uint2(v[0] | (v[2] << 16), v[1] | (v[3] << 16));
+    }
+    __syncthreads();
+    // per-sub-block sums: sub-block 2c+lh of unit j = the 32 halves of its 8 fragments (h, t)
+    const int nsum = a.US * 8 * BP;
+    for (int idx = threadIdx.x; idx < nsum; idx += blockDim.x) {
+        const int col = idx % BP;
+        const int js = idx / BP;
+        const int sub = js & 7, j = js >> 3;
+        const int c = sub >> 1, lh = sub & 1;
+        float acc = 0.0f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint2 v = xf[mma_xf_idx(j, c, lh, h, col, t, BP)];
+                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
+                const float2 q = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
+                acc += (p.x + p.y) + (q.x + q.y);
+            }
+        xsum[rows_xsum_off<BP>(a.US, j, sub, col)] = acc;
+    }
+}
+
+// One step: 32 rows (two 16-row tiles) x one superblock (unit j of the slice) at u0 (row stride
+// 144 B).  acc: C-fragment accumulators of the warp's rows; accM: this lane's row (row = lane),
+// the min term.  dtab: the warp's [8][32] table of D_j (scaled by 2^24 / 2^20 for the low /
+// high nibble halves), position (row % 8) * 4 + row / 8 so that rows g, g+8, g+16, g+24 are one
+// float4.
+template <int BP>
+__device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
+                                             int US, int j, float *dtab, float (&acc)[2][4],
+                                             float (&accM)[BP], int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    {
+        // header of row `lane`: the GGML get_scale_min_k4 table decoded with 32-bit masks (byte k
+        // of each word = sub-block k or k+4), d and dmin exact in fp32
+        const uint4 hdr = *reinterpret_cast<const uint4 *>(u0 + lane * 144);
+        const uint32_t SC_lo = hdr.y & 0x3F3F3F3Fu;
+        const uint32_t MM_lo = hdr.z & 0x3F3F3F3Fu;
+        const uint32_t SC_hi = (hdr.w & 0x0F0F0F0Fu) | ((hdr.y >> 2) & 0x30303030u);
+        const uint32_t MM_hi = ((hdr.w >> 4) & 0x0F0F0F0Fu) | ((hdr.z >> 2) & 0x30303030u);
+        __half2 dd;
+        *reinterpret_cast<uint32_t *>(&dd) = hdr.x;
+        const float2 dm = __half22float2(dd);
+        const float2 dscale = f2(dm.x * 16777216.0f, dm.x * 1048576.0f);
+        const int pos = (lane & 7) * 4 + (lane >> 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t scw = c < 2 ? SC_lo : SC_hi;
+            const uint32_t mmw = c < 2 ? MM_lo : MM_hi;
+            const uint32_t sel = 0x7650u + 2u * (c & 1);
+            // 6-bit integers to float through the 2^23 mantissa: (2^23 + v) - 2^23
+            const float2 sc = __fadd2_rn(f2(__uint_as_float(__byte_perm(scw, 0x4B000000u, sel)),
+                                            __uint_as_float(__byte_perm(scw, 0x4B000000u, sel + 1))),
+                                         f2(-8388608.0f, -8388608.0f));
+            const float2 mm = __fadd2_rn(f2(__uint_as_float(__byte_perm(mmw, 0x4B000000u, sel)),
+                                            __uint_as_float(__byte_perm(mmw, 0x4B000000u, sel + 1))),
+                                         f2(-8388608.0f, -8388608.0f));
+            const float2 D = __fmul2_rn(dscale, sc);
+            const float2 M = __fmul2_rn(f2(dm.y, dm.y), mm);
+            dtab[(2 * c) * 32 + pos] = D.x;
+            dtab[(2 * c + 1) * 32 + pos] = D.y;
+#pragma unroll
+            for (int b = 0; b < BP; ++b) {
+                accM[b] = fmaf(-M.x, xsum[rows_xsum_off<BP>(US, j, 2 * c, b)], accM[b]);
+                accM[b] = fmaf(-M.y, xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)], accM[b]);
+            }
+        }
+    }
+    __syncwarp();
+    const int col = g % BP;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint2 xb[2][2];
+#pragma unroll
+        for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) xb[lh][h] = xf[mma_xf_idx(j, c, lh, h, col, t, BP)];
+        const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * g);
+        const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * g);
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const uint8_t *rowA = u0 + (tile * 16 + g) * 144 + 16 + 32 * c + 8 * t;
+            const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);            // row tile*16 + g
+            const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * 144);  // row tile*16 + g + 8
+            float cl[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ch[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t wa = h ? wA.y : wA.x, wb = h ? wB.y : wB.x;
+                const uint32_t sa = __umulhi(wa, 1u << 24), sb = __umulhi(wb, 1u << 24);  // >> 8
+                mma_16816(cl, wa & 0x000F000Fu, wb & 0x000F000Fu, sa & 0x000F000Fu,
+                          sb & 0x000F000Fu, xb[0][h].x, xb[0][h].y);
+                mma_16816(ch, wa & 0x00F000F0u, wb & 0x00F000F0u, sa & 0x00F000F0u,
+                          sb & 0x00F000F0u, xb[1][h].x, xb[1][h].y);
+            }
+            const float la = tile ? Dlo.z : Dlo.x, lb = tile ? Dlo.w : Dlo.y;
+            const float ha = tile ? Dhi.z : Dhi.x, hb = tile ? Dhi.w : Dhi.y;
+            acc[tile][0] = fmaf(ha, ch[0], fmaf(la, cl[0], acc[tile][0]));
+            acc[tile][2] = fmaf(hb, ch[2], fmaf(lb, cl[2], acc[tile][2]));
+            if (BP > 1) {
+                acc[tile][1] = fmaf(ha, ch[1], fmaf(la, cl[1], acc[tile][1]));
+                acc[tile][3] = fmaf(hb, ch[3], fmaf(lb, cl[3], acc[tile][3]));
+            }
+        }
+    }
+}
+
+// Shared memory of the tensor-core kernel, in order: ring [NW][2][32 x 144 B], x fragments
+// [US][16][BP][4] uint2, x sums [US][8][BP], per-warp tables [NW][256] floats, partial rows
+// [red_floats], mbarriers [NW][2].
+template <int BP>
+__global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
+    mma_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap)
+{
+    constexpr int NW = MmaWarps<BP>::value;
+    constexpr int UB = 144;
+    constexpr int BOX = 32 * UB;
+    constexpr int INNER = UB / 4;
+    static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *ring = smem;
+    uint2 *xf = reinterpret_cast<uint2 *>(smem + NW * kRowsStages * BOX);
+    float *xsum = reinterpret_cast<float *>(xf + (size_t)a.US * 16 * BP * 4);
+    float *tabs = xsum + a.US * 8 * BP;
+    float *red = tabs + NW * 256;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(red + a.red_floats);
+
+    const int s = blockIdx.x / a.Gs;
+    const int cta = blockIdx.x % a.Gs;
+    const int US_s = min(a.US, a.UPR - s * a.US);
+    const int64_t R0 = ((int64_t)cta * a.N) / a.Gs, R1 = ((int64_t)(cta + 1) * a.N) / a.Gs;
+    const int rows = (int)(R1 - R0);
+    const BandShape bs = band_shape(rows, US_s, NW);
+    const int npairs = bs.G * bs.P;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ucol0 = s * a.US;
+    float *dtab = tabs + warp * 256;
+
+    auto pair_units = [&](int q, int &ua, int &ub) {
+        const int p = q % bs.P;
+        ua = (p * US_s) / bs.P;
+        ub = ((p + 1) * US_s) / bs.P;
+    };
+    int nsteps = 0;
+    for (int q = warp; q < npairs; q += NW) {
+        int ua, ub;
+        pair_units(q, ua, ub);
+        nsteps += ub - ua;
+    }
+    uint8_t *myring = ring + warp * kRowsStages * BOX;
+    const uint32_t bar0 = smem_u32(bars + warp * kRowsStages);
+    int iq = warp, iu = 0, iub = 0;
+    if (iq < npairs) pair_units(iq, iu, iub);
+    auto issue = [&](int i) {
+        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+        mbar_arrive_expect_tx(bar, BOX);
+        const int g = iq / bs.P;
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &tmap, (ucol0 + iu) * INNER,
+                    (int)(R0 + 32 * g), bar);
+        if (++iu == iub) {
+            iq += NW;
+            if (iq < npairs) pair_units(iq, iu, iub);
+        }
+    };
+
+    // 1. weight prefetch (independent of the previous kernel on the stream)
+    if (nsteps > 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+        for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
+        mbar_init_fence();
+        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+    }
+    // 2. programmatic dependent launch: let the next kernel start prefetching, then wait for the
+    //    previous kernel's results before reading x or writing y
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // 3. x fragments and sub-block sums of this slice
+    mma_stage_x<BP>(a, s, US_s, xf, xsum);
+    __syncthreads();
+
+    int step = 0;
+    bool failed = false;
+    for (int q = warp; q < npairs && !failed; q += NW) {
+        int ua, ub;
+        pair_units(q, ua, ub);
+        float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+        float accM[BP];
+#pragma unroll
+        for (int b = 0; b < BP; ++b) accM[b] = 0.0f;
+        for (int j = ua; j < ub; ++j, ++step) {
+            const bool ok = mbar_wait_bounded(bar0 + 8 * (step % kRowsStages),
+                                              (uint32_t)((step / kRowsStages) & 1));
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) {
+                    atomicExch(a.err, kErrCopyTimeout);
+                    for (int r = step + 1; r < nsteps && r < step + kRowsStages; ++r)
+                        (void)mbar_wait_bounded(bar0 + 8 * (r % kRowsStages), (uint32_t)((r / kRowsStages) & 1));
+                }
+                failed = true;
+                break;
+            }
+            mma_q4k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
+                             lane);
+            __syncwarp();
+            if (lane == 0 && step + kRowsStages < nsteps) {
+                fence_proxy_async_smem();
+                issue(step + kRowsStages);
+            }
+        }
+        if (failed) break;
+        // C fragments -> rows (row = lane) through the warp's table, plus the lane's min term
+        {
+            const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+            for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int col = 2 * t + (i & 1);
+                    if (col < BP) dtab[(tile * 16 + g + 8 * (i >> 1)) * BP + col] = acc[tile][i];
+                }
+        }
+        __syncwarp();
+        float v[BP];
+#pragma unroll
+        for (int b = 0; b < BP; ++b) v[b] = dtab[lane * BP + b] + accM[b];
+        __syncwarp();
+        if (bs.P == 1) {
+            const int rr = (q / bs.P) * 32 + lane;
+            if (rr < rows) {
+                float *dst = a.out + ((int64_t)s * a.N + R0 + rr) * a.B;
+                for (int b = 0; b < a.B; ++b) dst[b] = v[b];
+            }
+        } else {
+            float *r = red + ((size_t)q * 32 + lane) * BP;
+#pragma unroll
+            for (int b = 0; b < BP; ++b) r[b] = v[b];
+        }
+    }
+    if (__syncthreads_or(failed ? 1 : 0) || bs.P == 1) return;
+    // 4. rows of the band: sum the K parts in part order, write once
+    float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
+    for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
+        const int rr = t / a.B, b = t - rr * a.B;
+        const int g = rr >> 5, l = rr & 31;
+        float sum = 0.0f;
+        for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
+        outb[t] = sum;
+    }
+}
+
+}  // namespace qg

@@ -307,6 +307,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     constexpr int UB = RowsFmt<FMT>::kUnitBytes;
     constexpr int BOX = 32 * UB;  // bytes of one step: 32 rows x one unit
     constexpr int INNER = UB / 4; // u32 elements of one unit
+    static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;

@@ -132,6 +132,11 @@ def test_variant_checks(L):
     # unknown variants are rejected; the streaming variants need rows of whole 256-weight units
     assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 7) == qg.QG_ERR_VARIANT
     assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, -1) == qg.QG_ERR_VARIANT
+    assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 5) == qg.QG_ERR_VARIANT
+    # the tensor-core variant takes Q4_K only; every streaming variant needs K % 256 == 0
+    assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
+    for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_TENSOR):
+        assert L.qg_gemv_variant(FAKE, 8, 4, 96, FAKE, 1, FAKE, None, v) == qg.QG_ERR_VARIANT
 
 
 def test_dequant_rejects_bad_arguments(L):

@@ -106,7 +106,7 @@ def test_dequant_dump_golden_superblock(dev, orc):
 # GEMV parity on shapes the oracle finishes quickly (several tiles, ragged tails)
 # ------------------------------------------------------------------------------------------------
 
-Q4K_VARIANTS = [1, 2, 3]  # direct, factored, generic
+Q4K_VARIANTS = [1, 2, 3, 4]  # direct, factored, generic, tensor
 SMALL_SHAPES = [(1, 256), (2, 512), (7, 1280), (33, 5120), (300, 768), (129, 2560)]
 
 
@@ -137,6 +137,8 @@ def test_q8_0_gemv_small(dev, orc, variant, N, K, B):
     (Q4_K, 2, 96, 17408, 8),
     (Q4_K, 1, 40, 65536, 1),
     (Q4_K, 2, 17, 65536, 2),
+    (Q4_K, 4, 96, 17408, 8),
+    (Q4_K, 4, 17, 65536, 2),
     (Q8_0, 0, 64, 17408, 8),
 ])
 def test_split_k(dev, orc, fmt, variant, N, K, B):
@@ -207,12 +209,13 @@ def test_near_cancellation_direct_meets_strict_bound(dev, orc):
     yref, A = orc.gemv(W, Q4_K, N, K, x, B)
     y = gpu_gemv(dev, W, Q4_K, N, K, x, 1)
     assert_within(y, yref, A, "direct, near-cancellation")
-    yf = gpu_gemv(dev, W, Q4_K, N, K, x, 2)
     # magnitude of the factored terms: |d*sc*q*x| + |dmin*m*x| summed
     Dq = (np.repeat(sc.astype(np.float64) * 2.0 ** -7, 32) * q).reshape(N, K)
     Mm = np.repeat(m.astype(np.float64) * 2.0 ** -7, 32).reshape(N, K)
     Af = (Dq + Mm) @ np.abs(x.astype(np.float64))
-    assert_within(yf, yref, Af, "factored, near-cancellation (factored bound)")
+    for v in (2, 4):
+        yf = gpu_gemv(dev, W, Q4_K, N, K, x, v)
+        assert_within(yf, yref, Af, f"variant {v}, near-cancellation (factored bound)")
 
 
 # ------------------------------------------------------------------------------------------------
@@ -225,12 +228,12 @@ def _sample_rows(N, rng, k=192):
 
 
 @pytest.mark.parametrize("wl", sorted(synth.WORKLOADS))
-@pytest.mark.parametrize("variant", [0, 1, 2])
+@pytest.mark.parametrize("variant", [0, 1, 2, 4])
 def test_full_size_workloads_sampled(dev, orc, wl, variant):
     w = synth.WORKLOADS[wl]
     rng = np.random.default_rng(0)
     for call in w.calls:
-        if call.fmt == Q8_0 and variant == 2:
+        if call.fmt == Q8_0 and variant in (2, 4):
             continue
         W, x = w.inputs(call)
         v = variant if call.fmt == Q4_K else 0
@@ -254,11 +257,15 @@ def test_launch_witness_and_no_device_error(dev):
     W = _t(synth.q4k_weights(N, K, seed=1), dev)
     x = _t(synth.activations(K, 1, seed=1).view(np.uint16), dev)
     y = torch.empty((N, 1), dtype=torch.float32, device=dev)
-    for v in (1, 2, 3):
+    for v in (1, 2, 3, 4):
         qg.qg_gemv_variant(W, Q4_K, N, K, x, 1, y, None, v)
         assert qg.qg_last_variant() == v
     qg.qg_gemv(W, Q4_K, N, K, x, 1, y)
-    assert qg.qg_last_variant() in (1, 2)
+    assert qg.qg_last_variant() == qg.QG_VARIANT_FACTORED
+    x2 = _t(synth.activations(K, 2, seed=1).view(np.uint16), dev)
+    y2 = torch.empty((N, 2), dtype=torch.float32, device=dev)
+    qg.qg_gemv(W, Q4_K, N, K, x2, 2, y2)
+    assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
     assert qg.qg_device_error() == 0
     Wq8 = _t(synth.q8_0_weights(N, 96, seed=1), dev)
     x96 = _t(synth.activations(96, 1, seed=1).view(np.uint16), dev)
