@@ -57,45 +57,59 @@ __device__ __forceinline__ int mma_xf_idx(int j, int c, int lh, int h, int col, 
     return ((((j * 4 + c) * 2 + lh) * 2 + h) * BP + col) * 4 + t;
 }
 
+// Thread g stages the 4 consecutive x rows e..e+3 of group g = ((j*4 + c)*2 + lh)*8 + 2t + h
+// (all B columns, one contiguous run of 4*B halves, read with the widest aligned loads), writes
+// their BP fragments, and the 8 groups of one sub-block (8 consecutive lanes) add up its x sums.
 template <int BP>
 __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, uint2 *xf,
                                             float *xsum)
 {
-    const uint16_t *xsl = a.x + (int64_t)s * a.US * 256 * a.B;
-    const int nfrag = a.US * 16 * BP * 4;
-    for (int idx = threadIdx.x; idx < nfrag; idx += blockDim.x) {
-        const int t = idx & 3;
-        int r = idx >> 2;
-        const int col = r % BP;
-        r /= BP;
-        const int h = r & 1, lh = (r >> 1) & 1, c = (r >> 2) & 3, j = r >> 4;
-        uint32_t v[4] = {0u, 0u, 0u, 0u};
-        if (j < US_s && col < a.B) {
+    const int B = a.B;
+    const uint16_t *xsl = a.x + (int64_t)s * a.US * 256 * B;
+    const int ngroups = a.US * 64;  // a multiple of 32: every lane of a warp takes part
+    for (int gi = threadIdx.x; gi < ngroups; gi += blockDim.x) {
+        const int th = gi & 7, t = th >> 1, h = th & 1;
+        const int lh = (gi >> 3) & 1, c = (gi >> 4) & 3, j = gi >> 6;
+        uint32_t xv[4 * BP];  // x[e + r][col] at r * BP + col (fp16 bits), zero when absent
+#pragma unroll
+        for (int q = 0; q < 4 * BP; ++q) xv[q] = 0u;
+        if (j < US_s) {
             const int e = j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
+            const uint16_t *src = xsl + (int64_t)e * B;  // 4 * B contiguous halves
+            const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
+            if (B == BP && (8 * BP) % 16 == 0 && (addr & 15) == 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = xsl[(int64_t)(e + i) * a.B + col];
-        }
-        xf[idx] = make_uint2(v[0] | (v[2] << 16), v[1] | (v[3] << 16));
-    }
-    __syncthreads();
-    // per-sub-block sums: sub-block 2c+lh of unit j = the 32 halves of its 8 fragments (h, t)
-    const int nsum = a.US * 8 * BP;
-    for (int idx = threadIdx.x; idx < nsum; idx += blockDim.x) {
-        const int col = idx % BP;
-        const int js = idx / BP;
-        const int sub = js & 7, j = js >> 3;
-        const int c = sub >> 1, lh = sub & 1;
-        float acc = 0.0f;
+                for (int q = 0; q < (8 * BP) / 16; ++q) {
+                    const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
+                    xv[8 * q + 0] = v.x & 0xFFFFu; xv[8 * q + 1] = v.x >> 16;
+                    xv[8 * q + 2] = v.y & 0xFFFFu; xv[8 * q + 3] = v.y >> 16;
+                    xv[8 * q + 4] = v.z & 0xFFFFu; xv[8 * q + 5] = v.z >> 16;
+                    xv[8 * q + 6] = v.w & 0xFFFFu; xv[8 * q + 7] = v.w >> 16;
+                }
+            } else if (B == BP && BP == 1 && (addr & 7) == 0) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(src);
+                xv[0] = v.x & 0xFFFFu; xv[1] = v.x >> 16; xv[2] = v.y & 0xFFFFu; xv[3] = v.y >> 16;
+            } else {
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+                for (int r = 0; r < 4; ++r)
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const uint2 v = xf[mma_xf_idx(j, c, lh, h, col, t, BP)];
-                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
-                const float2 q = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
-                acc += (p.x + p.y) + (q.x + q.y);
+                    for (int col = 0; col < BP; ++col)
+                        if (col < B) xv[r * BP + col] = src[r * B + col];
             }
-        xsum[rows_xsum_off<BP>(a.US, j, sub, col)] = acc;
+        }
+#pragma unroll
+        for (int col = 0; col < BP; ++col) {
+            xf[mma_xf_idx(j, c, lh, h, col, t, BP)] =
+                make_uint2(xv[0 * BP + col] | (xv[2 * BP + col] << 16),
+                           xv[1 * BP + col] | (xv[3 * BP + col] << 16));
+            float sum = (__half2float(__ushort_as_half((unsigned short)xv[0 * BP + col])) +
+                         __half2float(__ushort_as_half((unsigned short)xv[1 * BP + col]))) +
+                        (__half2float(__ushort_as_half((unsigned short)xv[2 * BP + col])) +
+                         __half2float(__ushort_as_half((unsigned short)xv[3 * BP + col])));
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (th == 0) xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, col)] = sum;
+        }
     }
 }
 

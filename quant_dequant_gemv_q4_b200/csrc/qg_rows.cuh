@@ -105,12 +105,16 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
     const int US = a.US;
     const int64_t kbase = (int64_t)s * US * 256;
     const uint16_t *xsl = a.x + kbase * a.B;
-    const int nchunk = 32 * BP * US;  // 16-byte chunks (j, c, i, b), b fastest
+    // thread t stages word i = t % 8 of chunk (j, c) for column b; the 8 words of one chunk are 8
+    // consecutive lanes, which then add their halves into the chunk's two sub-block sums
+    const int nchunk = 32 * BP * US;  // a multiple of 32: every lane of a warp takes part
     const bool vec = (BP == 1) && ((reinterpret_cast<uintptr_t>(xsl) & 7) == 0);
     for (int t = threadIdx.x; t < nchunk; t += blockDim.x) {
-        const int b = t % BP;
-        const int jci = t / BP;
-        const int i = jci & 7, c = (jci >> 3) & 3, j = jci >> 5;
+        const int i = t & 7;
+        const int jcb = t >> 3;
+        const int b = jcb % BP;
+        const int jc = jcb / BP;
+        const int c = jc & 3, j = jc >> 2;
         uint32_t h[8];  // x[e0 .. e0+3], x[e0+32 .. e0+35] in natural order
         if (j < US_s && b < a.B) {
             const int e0 = j * 256 + c * 64 + 4 * i;
@@ -135,25 +139,26 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
         v.y = h[1] | (h[3] << 16);
         v.z = h[4] | (h[6] << 16);
         v.w = h[5] | (h[7] << 16);
-        *reinterpret_cast<uint4 *>(xs + (int64_t)t * 8) = v;
-    }
-    __syncthreads();
-    // sub-block 2c+h of unit j = halves 4h..4h+3 of the 8 words of chunk c, summed in fixed order
-    const int nsum = 8 * BP * US;
-    for (int t = threadIdx.x; t < nsum; t += blockDim.x) {
-        const int b = t % BP;
-        const int js = t / BP;
-        const int sub = js & 7, j = js >> 3;
-        const int c = sub >> 1, hsel = sub & 1;
-        float acc = 0.0f;
+        *reinterpret_cast<uint4 *>(xs + rows_x_off<BP>(US, j, c, i, b)) = v;
+        // sub-block sums of the chunk: low half (sub-block 2c) and high half (2c+1), fp32, the
+        // same xor-butterfly order on every lane
+        float lo = (__half2float(__ushort_as_half((unsigned short)h[0])) +
+                    __half2float(__ushort_as_half((unsigned short)h[1]))) +
+                   (__half2float(__ushort_as_half((unsigned short)h[2])) +
+                    __half2float(__ushort_as_half((unsigned short)h[3])));
+        float hi = (__half2float(__ushort_as_half((unsigned short)h[4])) +
+                    __half2float(__ushort_as_half((unsigned short)h[5]))) +
+                   (__half2float(__ushort_as_half((unsigned short)h[6])) +
+                    __half2float(__ushort_as_half((unsigned short)h[7])));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(xs + rows_x_off<BP>(US, j, c, i, b) + 4 * hsel);
-            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
-            const float2 q = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
-            acc += (p.x + p.y) + (q.x + q.y);
+        for (int off = 1; off < 8; off <<= 1) {
+            lo += __shfl_xor_sync(0xffffffffu, lo, off);
+            hi += __shfl_xor_sync(0xffffffffu, hi, off);
         }
-        xsum[t] = acc;
+        if (i == 0) {
+            xsum[rows_xsum_off<BP>(US, j, 2 * c, b)] = lo;
+            xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)] = hi;
+        }
     }
 }
 
