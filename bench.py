@@ -208,13 +208,15 @@ class CallSet:
                                     stream, variant)
 
     def launches_per_step(self, variant: int) -> int:
-        """Kernels one step launches (a split-K call adds its second pass)."""
+        """Kernels one step launches (a split-K call of the DIRECT kernel adds its second pass;
+        the streaming kernels add the K slices inside the same launch)."""
         import torch
         n = 0
         for i, c in enumerate(self.calls):
             self.qg.qg_gemv_variant(self.W[i][0], c.fmt, c.N, c.K, self.x[i], c.B, self.y[i],
                                     torch.cuda.current_stream(), variant)
-            n += 2 if self.qg.qg_last_splits() > 1 else 1
+            two = self.qg.qg_last_splits() > 1 and self.qg.qg_last_variant() == self.qg.QG_VARIANT_DIRECT
+            n += 2 if two else 1
         torch.cuda.synchronize()
         return n
 

@@ -59,8 +59,12 @@ int ensure_smem_attr(int dev, const void *func, int bytes)
         std::lock_guard<std::mutex> lk(g_mu);
         if (g_attr_set.count({dev, func})) return QG_OK;
     }
-    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess)
+    // static and dynamic shared memory together must fit the per-block limit
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, func) != cudaSuccess) return QG_ERR_CUDA;
+    const int dyn = bytes - (int)fa.sharedSizeBytes;
+    if (dyn <= 0 ||
+        cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess)
         return QG_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
     g_attr_set.insert({dev, func});
@@ -325,7 +329,7 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
 // word; `part` holds S*N*B floats when S > 1.
 int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
                 cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, int *err,
-                float *part, bool pdl)
+                unsigned *cnt, float *part, bool pdl)
 {
     const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
@@ -335,6 +339,8 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     RowsArgs a;
     a.x = x;
     a.out = (p.S > 1) ? part : y;
+    a.y = y;
+    a.cnt = cnt;
     a.err = err;
     a.N = N;
     a.B = B;
@@ -355,12 +361,6 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     cfg.numAttrs = 1;
     void *args[] = {&a, &map};
     if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return QG_ERR_CUDA;
-    if (p.S > 1) {
-        const int64_t NB = N * B;
-        const int64_t blocks = std::min<int64_t>((NB + 255) / 256, (int64_t)di.sms * 4);
-        splitk_sum_kernel<<<(unsigned)blocks, 256, 0, st>>>(part, y, NB, p.S);
-        if (cudaGetLastError() != cudaSuccess) return QG_ERR_CUDA;
-    }
     return QG_OK;
 }
 
@@ -436,8 +436,10 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
         if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
         WsView ws;
         const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-        if ((rc = get_workspace(dev, stream, 0, 0, part_f, &ws)) != QG_OK) return rc;
-        if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.part, true)) != QG_OK)
+        const size_t ncnt = (p.S > 1) ? (size_t)p.Gs : 0;
+        if ((rc = get_workspace(dev, stream, ncnt, 0, part_f, &ws)) != QG_OK) return rc;
+        if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.cnt, ws.part, true)) !=
+            QG_OK)
             return rc;
         t_last_variant = var;
         t_last_splits = p.S;
@@ -644,6 +646,10 @@ int noalloc_scratch(int dev, uint8_t **out)
 
 }  // namespace
 
+// band counters reserved at the start of the fixed scratch array (a band per CTA of a slice, at
+// most one per SM)
+constexpr size_t kNoallocCounters = 1024;
+
 extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
                                int B, float *y, void *stream)
 {
@@ -664,16 +670,22 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-    if (ws_bytes_for(0, 0, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
+    // one fixed layout for every call: kNoallocCounters band counters, then the partial rows
+    const size_t ncnt = kNoallocCounters;
+    if ((size_t)p.Gs > kNoallocCounters) return QG_ERR_SCRATCH;
+    if (ws_bytes_for(ncnt, 0, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
     uint8_t *base = nullptr;
     if ((rc = noalloc_scratch(dev, &base)) != QG_OK) return rc;
     Workspace w;
     w.base = base;
     w.bytes = QG_NOALLOC_SCRATCH_BYTES;
+    w.nw = ncnt;
     const WsView ws = ws_view(w);
-    // Every element of the split-K partial rows is written before it is read, so nothing in the
-    // array has to be cleared between calls.
-    if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.part, false)) != QG_OK)
+    // Every element of the split-K partial rows is written before it is read, and the kernel
+    // returns every band counter to zero (the array starts zeroed), so nothing has to be cleared
+    // between calls.
+    if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.cnt, ws.part, false)) !=
+        QG_OK)
         return rc;
     return QG_OK;
 }

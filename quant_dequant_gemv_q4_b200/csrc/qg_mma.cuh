@@ -330,16 +330,20 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
             for (int b = 0; b < BP; ++b) r[b] = v[b];
         }
     }
-    if (__syncthreads_or(failed ? 1 : 0) || bs.P == 1) return;
+    const bool any_failed = __syncthreads_or(failed ? 1 : 0);
     // 4. rows of the band: sum the K parts in part order, write once
-    float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
-    for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
-        const int rr = t / a.B, b = t - rr * a.B;
-        const int g = rr >> 5, l = rr & 31;
-        float sum = 0.0f;
-        for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
-        outb[t] = sum;
+    if (!any_failed && bs.P > 1) {
+        float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
+        for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
+            const int rr = t / a.B, b = t - rr * a.B;
+            const int g = rr >> 5, l = rr & 31;
+            float sum = 0.0f;
+            for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
+            outb[t] = sum;
+        }
     }
+    // 5. K slices: the last CTA of the band adds them up
+    if (a.S > 1) splitk_fixup(a, cta, R0, rows);
 }
 
 }  // namespace qg

@@ -49,6 +49,8 @@ constexpr int kRowsStages = 2;  // ring stages per warp (double buffering)
 struct RowsArgs {
     const uint16_t *x;  // fp16 bits [K][B]
     float *out;         // y [N][B] when S == 1, else per-slice partial rows [S][N][B]
+    float *y;           // y [N][B] (the split-K result when S > 1)
+    unsigned *cnt;      // S > 1: arrival counter per row band, zero between calls
     int *err;           // device error word
     int64_t N;
     int B;
@@ -304,6 +306,33 @@ __device__ __forceinline__ BandShape band_shape(int rows, int US_s, int NW)
     return b;
 }
 
+// Split-K across CTAs without a second kernel.  CTA (slice s, band) has written its band's
+// partial rows to out = part[s][N][B]; each makes its writes visible and bumps the band's
+// counter, and the last of the S CTAs to arrive adds the S slices in slice order (so y does not
+// depend on arrival order), writes y and resets the counter for the next call.  Every CTA
+// arrives, also after a copy timeout, so the counters always return to zero.
+__device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_t R0, int rows)
+{
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned prev = atomicAdd(a.cnt + band, 1u);
+        s_last = (prev == (unsigned)(a.S - 1)) ? 1 : 0;
+        if (s_last) a.cnt[band] = 0u;  // all S arrivals of this call are in
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int64_t NB = a.N * a.B;
+    for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
+        const int64_t idx = R0 * a.B + t;
+        float sum = 0.0f;
+        for (int s2 = 0; s2 < a.S; ++s2) sum += __ldcg(a.out + s2 * NB + idx);
+        a.y[idx] = sum;
+    }
+}
+
 template <int FMT, int BP>
 __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     rows_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap)
@@ -423,16 +452,20 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
             for (int b = 0; b < BP; ++b) r[b] = acc[b];
         }
     }
-    if (__syncthreads_or(failed ? 1 : 0) || bs.P == 1) return;
+    const bool any_failed = __syncthreads_or(failed ? 1 : 0);
     // 4. rows of the band: sum the K parts in part order, write once
-    float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
-    for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
-        const int rr = t / a.B, b = t - rr * a.B;
-        const int g = rr >> 5, l = rr & 31;
-        float sum = 0.0f;
-        for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
-        outb[t] = sum;
+    if (!any_failed && bs.P > 1) {
+        float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
+        for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
+            const int rr = t / a.B, b = t - rr * a.B;
+            const int g = rr >> 5, l = rr & 31;
+            float sum = 0.0f;
+            for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
+            outb[t] = sum;
+        }
     }
+    // 5. K slices: the last CTA of the band adds them up
+    if (a.S > 1) splitk_fixup(a, cta, R0, rows);
 }
 
 }  // namespace qg
