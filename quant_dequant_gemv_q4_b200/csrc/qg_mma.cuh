@@ -56,6 +56,13 @@ __device__ __forceinline__ int mma_xf_idx(int j, int c, int lh, int h, int col, 
 {
     return ((((j * 4 + c) * 2 + lh) * 2 + h) * BP + col) * 4 + t;
 }
+// Columns are stored XOR-swizzled per block, col ^ mma_xf_swz(c, lh, h): the staging lanes that
+// differ only in (h, lh, chunk) then write different banks (with BP >= 4 a block spans a multiple
+// of 32 words, so unswizzled they would all hit one bank).
+__device__ __forceinline__ int mma_xf_swz(int c, int lh, int h, int BP)
+{
+    return BP >= 4 ? ((h + 2 * lh + 4 * (c & 1)) & (BP - 1)) : 0;
+}
 
 // Thread g stages the 4 consecutive x rows e..e+3 of group g = ((j*4 + c)*2 + lh)*8 + 2t + h
 // (all B columns, one contiguous run of 4*B halves, read with the widest aligned loads), writes
@@ -99,9 +106,6 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
         }
 #pragma unroll
         for (int col = 0; col < BP; ++col) {
-            xf[mma_xf_idx(j, c, lh, h, col, t, BP)] =
-                make_uint2(xv[0 * BP + col] | (xv[2 * BP + col] << 16),
-                           xv[1 * BP + col] | (xv[3 * BP + col] << 16));
             float sum = (__half2float(__ushort_as_half((unsigned short)xv[0 * BP + col])) +
                          __half2float(__ushort_as_half((unsigned short)xv[1 * BP + col]))) +
                         (__half2float(__ushort_as_half((unsigned short)xv[2 * BP + col])) +
@@ -110,6 +114,12 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
             for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
             if (th == 0) xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, col)] = sum;
         }
+        const int swz = mma_xf_swz(c, lh, h, BP);
+#pragma unroll
+        for (int col = 0; col < BP; ++col)
+            xf[mma_xf_idx(j, c, lh, h, col ^ swz, t, BP)] =
+                make_uint2(xv[0 * BP + col] | (xv[2 * BP + col] << 16),
+                           xv[1 * BP + col] | (xv[3 * BP + col] << 16));
     }
 }
 
@@ -168,7 +178,7 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 #pragma unroll
         for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) xb[lh][h] = xf[mma_xf_idx(j, c, lh, h, col, t, BP)];
+            for (int h = 0; h < 2; ++h) xb[lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
         const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * g);
         const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * g);
 #pragma unroll
