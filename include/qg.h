@@ -156,11 +156,12 @@ int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
  * device-wide synchronization an allocation may cause, or code recorded into a CUDA graph (an
  * allocation during capture is an error).  The caller passes inputs and outputs exactly as for
  * qg_gemv (same arguments, layouts, preconditions and results, default kernel variant); the
- * kernel's scratch (arrival counters, partial sums of rows split between warps, split-K partial
- * rows) lives in one file-scope device array of QG_NOALLOC_SCRATCH_BYTES per GPU.
- *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library routine.  Each call
- *     clears the counters it uses with cudaMemsetAsync on `stream`, since the array keeps what
- *     the previous call left.
+ * kernel's scratch (an error word, one arrival counter per row band when K is split, the split-K
+ * partial rows) lives in one file-scope device array of QG_NOALLOC_SCRATCH_BYTES per GPU.
+ *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library routine.  The counters
+ *     start at zero (the array is zero-initialized) and every call leaves them at zero again (the
+ *     last CTA of a band resets its counter); the partial rows are written before they are read.
+ *     So nothing is cleared between calls.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current) and caches it; make that first call before any stream capture.
  *   - Every call on every stream shares the one array: calls that overlap on the GPU race and give
