@@ -275,6 +275,61 @@ class _null:
         return False
 
 
+def time_gate_up(device, B: int, steps: int, warmup: int, l2_bytes: int) -> dict:
+    """The fused FFN gate/up pair (two Q4_K 17408 x 5120 tensors on one x, h = silu(g) * u) per
+    call, replayed from CUDA graphs over rotating copies of both tensors."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    N, K = HEADLINE.N, HEADLINE.K
+    g_call = synth.Gemv("ffn_gate", synth.Q4_K, N, K, B, 0)
+    u_call = synth.Gemv("ffn_up", synth.Q4_K, N, K, B, 1)
+    wl = synth.Workload("gate_up", HEADLINE_SEED, (g_call, u_call))
+    Wg, x = wl.inputs(g_call)
+    Wu, _ = wl.inputs(u_call)
+    pair_bytes = 2 * g_call.weight_bytes
+    copies = int(max(2, -(-4 * l2_bytes // pair_bytes)))
+    Wgs = [torch.from_numpy(Wg).to(device)]
+    Wus = [torch.from_numpy(Wu).to(device)]
+    for _ in range(copies - 1):
+        Wgs.append(Wgs[0].clone())
+        Wus.append(Wus[0].clone())
+    xd = torch.from_numpy(x.view(np.uint16)).to(device)
+    h = torch.empty((N, B), dtype=torch.float32, device=device)
+    stream = torch.cuda.Stream(device=device)
+
+    def launch(r):
+        qg.qg_gemv_gate_up_silu(Wgs[r], Wus[r], synth.Q4_K, N, K, xd, B, h, stream)
+
+    with torch.cuda.stream(stream):
+        launch(0)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for r in range(copies):
+            launch(r)
+    reps = max(1, steps // copies)
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-warmup // copies))):
+            graph.replay()
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        b.record(stream)
+    b.synchronize()
+    secs = a.elapsed_time(b) / 1e3
+    secs = dist_max(secs, device)
+    calls = reps * copies
+    nbytes = pair_bytes + 2 * K * B + 4 * N * B
+    del graph
+    return {"B": B, "us_per_call": round(secs * 1e6 / calls, 3),
+            "gbs": round(nbytes * calls / secs / 1e9, 1),
+            "bytes_per_call": nbytes, "calls": calls, "variant": qg.qg_last_variant(),
+            "splits": qg.qg_last_splits()}
+
+
 def time_e2e(cs: CallSet, steps: int, warmup: int, variant: int):
     """End to end through the public Python API: per step, pinned host x -> device, qg_gemv,
     y -> pinned host; returns (seconds, h2d bytes/step, d2h bytes/step)."""
@@ -513,6 +568,14 @@ def main(argv=None):
           "steps": steps8}
     del cs8
 
+    # the fused FFN gate/up pair (one launch, two weight streams, h = silu(g) * u)
+    gate_up = []
+    for Bg in (1, 8):
+        r = time_gate_up(device, Bg, max(500, min(args.steps // 8, 20000)), args.warmup, l2)
+        r["frac_of_hbm"] = round(r["gbs"] / hbm, 4)
+        gate_up.append(r)
+    torch.cuda.empty_cache()
+
     # every workload of the suite, per call
     table = {}
     if not args.no_table:
@@ -582,6 +645,7 @@ def main(argv=None):
         "variant": variant_used,
         "roofline": roofline,
         "b8": b8,
+        "gate_up_silu": gate_up,
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": args.steps * launches,

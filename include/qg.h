@@ -108,6 +108,22 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
 int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
             void *stream);
 
+/* The FFN gate/up pair on one x, fused with its activation:
+ *     h[n,b] = silu(gate[n,b]) * up[n,b],  gate = dequant(Wg) . x,  up = dequant(Wu) . x,
+ *     silu(v) = v / (1 + e^-v)
+ * as "Qwen3.6 27B Single-B70 Maximum-Speed Requirements And Execution Plan", "Phase 3: Maximum
+ * Useful Fusion" names it first among the fusion families (the gate+up projection pair and its
+ * SiLU-mul epilogue).  One launch streams both weight tensors, stages x once and writes only h;
+ * gate and up never reach HBM.
+ *   Wg, Wu   device, two N x K tensors of format fmt (each qg_weight_bytes(fmt, N, K) bytes,
+ *            16-byte aligned), read only
+ *   x, B     as for qg_gemv; h: device, fp32 [N][B], 4-byte aligned, fully overwritten
+ * The products and sums are those of qg_gemv's default kernels for (fmt, B); silu is evaluated in
+ * fp32 with expf.  Errors as qg_gemv, plus QG_ERR_SHAPE when K % 256 != 0 (the fused path needs rows
+ * of whole 256-weight units). */
+int qg_gemv_gate_up_silu(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K,
+                         const uint16_t *x, int B, float *h, void *stream);
+
 /* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant,
  * for DIRECT / FACTORED / TENSOR when K % 256 != 0, and for TENSOR with Q8_0.  The other variants
  * take both formats. */

@@ -6,7 +6,10 @@ numpy; it shares no code with the CUDA library and never imports it.
 
 What it computes, and the page passages it follows, is stated in the header of ``qg_oracle.c``:
 fp32 weights dequantized exactly and rounded once, then ``y = sum_k w*x`` and
-``A = sum_k |w*x|`` in fp64.
+``A = sum_k |w*x|`` in fp64.  ``gate_up_silu`` adds the FFN gate/up pair's activation,
+``h = silu(gate) * up`` with ``silu(v) = v / (1 + e^-v)``, in fp64 on the two GEMVs ("Qwen3.6 27B
+Single-B70 Maximum-Speed Requirements And Execution Plan", "Phase 3: Maximum Useful Fusion": the
+gate+up pair and its SiLU-mul epilogue).
 """
 from __future__ import annotations
 
@@ -116,6 +119,22 @@ def gemv(W: np.ndarray, fmt: int, N: int, K: int, x: np.ndarray, B: int,
         _check(lib().orc_gemv_rows(int(fmt), _ptr(W), N, K, _ptr(xb), B, _ptr(r), r.size,
                                    _ptr(y), _ptr(A)), "gemv_rows")
     return y, A
+
+
+def silu(v) -> np.ndarray:
+    """silu(v) = v / (1 + e^-v) = v * sigmoid(v), in fp64."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return v / (1.0 + np.exp(-v))
+
+
+def gate_up_silu(Wg: np.ndarray, Wu: np.ndarray, fmt: int, N: int, K: int, x: np.ndarray, B: int,
+                 rows: np.ndarray | None = None):
+    """(h, g, Ag, u, Au) in fp64: g = W_g x and u = W_u x with their sum|w*x| (as ``gemv``), and
+    h = silu(g) * u."""
+    g, Ag = gemv(Wg, fmt, N, K, x, B, rows)
+    u, Au = gemv(Wu, fmt, N, K, x, B, rows)
+    return silu(g) * u, g, Ag, u, Au
 
 
 def unpack_q4k(W: np.ndarray, nsb: int) -> dict:

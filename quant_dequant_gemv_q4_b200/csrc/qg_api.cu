@@ -219,7 +219,8 @@ struct RowsPlan {
     bool tensor;  // mma_gemv_kernel instead of rows_gemv_kernel
 };
 
-RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di, bool tensor)
+RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di, bool tensor,
+                        int mats = 1)
 {
     RowsPlan best{};
     double best_util = -1.0;
@@ -245,7 +246,11 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         const int64_t Gs = std::max<int64_t>(1, std::min<int64_t>(di.sms / S, N));
         // partial rows are kept in shared memory only when a band has several K parts, and then
         // there is at most one (row group, part) pair per warp
-        const int red = NW * 32 * BP;
+        // partial rows: one (group, part) pair per warp, or, for the gate/up pair, every group of
+        // both matrices when there are more groups than warps
+        const int64_t band_rows = (N + Gs - 1) / Gs;
+        const int64_t groups = (int64_t)mats * ((band_rows + 31) / 32);
+        const int red = (int)((mats == 1 ? NW : std::max<int64_t>(NW, groups)) * 32 * BP);
         const size_t smem = ring + (size_t)US * (512 + 32) * BP + tabs + (size_t)red * sizeof(float) + bars;
         if (smem + 128 > (size_t)di.smem_optin) continue;
         const double util = ((double)N / (double)Gs) / (32.0 * (double)((N / Gs + 31) / 32 > 0 ? (N / Gs + 31) / 32 : 1));
@@ -329,13 +334,18 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
 // word; `part` holds S*N*B floats when S > 1.
 int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
                 cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, int *err,
-                unsigned *cnt, float *part, bool pdl)
+                unsigned *cnt, float *part, bool pdl, const void *W2 = nullptr, int act = 0)
 {
     const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
     if (rc != QG_OK) return rc;
-    CUtensorMap map;
+    CUtensorMap map, map2;
     if ((rc = make_weight_map(W, fmt, N, K, &map)) != QG_OK) return rc;
+    if (W2) {
+        if ((rc = make_weight_map(W2, fmt, N, K, &map2)) != QG_OK) return rc;
+    } else {
+        map2 = map;
+    }
     RowsArgs a;
     a.x = x;
     a.out = (p.S > 1) ? part : y;
@@ -349,6 +359,8 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     a.S = p.S;
     a.Gs = p.Gs;
     a.red_floats = p.red_floats;
+    a.mats = W2 ? 2 : 1;
+    a.act = act;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
     cfg.blockDim = dim3(p.NW * 32);
@@ -359,7 +371,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void *args[] = {&a, &map};
+    void *args[] = {&a, &map, &map2};
     if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return QG_ERR_CUDA;
     return QG_OK;
 }
@@ -497,9 +509,47 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     return QG_OK;
 }
 
+// The FFN gate/up pair on one x, h = silu(Wg x) * (Wu x): the streaming kernels with both
+// matrices in one launch (x staged once, the two rows of h's entry meet in shared memory).
+int gate_up_impl(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K, const uint16_t *x,
+                 int B, float *h, void *stream)
+{
+    int rc = check_common(Wg, fmt, N, K);
+    if (rc != QG_OK) return rc;
+    if ((rc = check_common(Wu, fmt, N, K)) != QG_OK) return rc;
+    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (N == 0) return QG_OK;
+    if (!x || !h) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(h) % 4 != 0)
+        return QG_ERR_ALIGN;
+    if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
+    DeviceInfo di;
+    int dev = 0;
+    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    const int var = auto_variant(fmt, K, B);
+    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR, 2);
+    if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+    WsView ws;
+    const size_t part_f = (p.S > 1) ? (size_t)p.S * 2 * (size_t)N * (size_t)B : 0;
+    const size_t ncnt = (p.S > 1) ? (size_t)p.Gs : 0;
+    if ((rc = get_workspace(dev, stream, ncnt, 0, part_f, &ws)) != QG_OK) return rc;
+    if ((rc = launch_rows(Wg, fmt, N, K, x, B, h, static_cast<cudaStream_t>(stream), di, dev, p, ws.err,
+                          ws.cnt, ws.part, true, Wu, 1)) != QG_OK)
+        return rc;
+    t_last_variant = var;
+    t_last_splits = p.S;
+    return QG_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int qg_gemv_gate_up_silu(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K,
+                         const uint16_t *x, int B, float *h, void *stream)
+{
+    return gate_up_impl(Wg, Wu, fmt, N, K, x, B, h, stream);
+}
 
 int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
             void *stream)

@@ -213,7 +213,8 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 // [red_floats], mbarriers [NW][2].
 template <int BP>
 __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
-    mma_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap)
+    mma_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap,
+                    const __grid_constant__ CUtensorMap tmap2)
 {
     constexpr int NW = MmaWarps<BP>::value;
     constexpr int UB = 144;
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     const int US_s = min(a.US, a.UPR - s * a.US);
     const int64_t R0 = ((int64_t)cta * a.N) / a.Gs, R1 = ((int64_t)(cta + 1) * a.N) / a.Gs;
     const int rows = (int)(R1 - R0);
-    const BandShape bs = band_shape(rows, US_s, NW);
+    const BandShape bs = band_shape(rows, US_s, NW, a.mats);
     const int npairs = bs.G * bs.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;
@@ -258,9 +259,9 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     auto issue = [&](int i) {
         const uint32_t bar = bar0 + 8 * (i % kRowsStages);
         mbar_arrive_expect_tx(bar, BOX);
-        const int g = iq / bs.P;
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &tmap, (ucol0 + iu) * INNER,
-                    (int)(R0 + 32 * g), bar);
+        const int g = iq / bs.P;  // matrix g / Gm, row group g % Gm
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), g < bs.Gm ? &tmap : &tmap2,
+                    (ucol0 + iu) * INNER, (int)(R0 + 32 * (g % bs.Gm)), bar);
         if (++iu == iub) {
             iq += NW;
             if (iq < npairs) pair_units(iq, iu, iub);
@@ -270,6 +271,8 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     // 1. weight prefetch (independent of the previous kernel on the stream)
     if (nsteps > 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+        if (a.mats > 1)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap2)) : "memory");
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
@@ -328,7 +331,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
 #pragma unroll
         for (int b = 0; b < BP; ++b) v[b] = dtab[lane * BP + b] + accM[b];
         __syncwarp();
-        if (bs.P == 1) {
+        if (bs.P == 1 && a.mats == 1) {
             const int rr = (q / bs.P) * 32 + lane;
             if (rr < rows) {
                 float *dst = a.out + ((int64_t)s * a.N + R0 + rr) * a.B;
@@ -341,17 +344,8 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
         }
     }
     const bool any_failed = __syncthreads_or(failed ? 1 : 0);
-    // 4. rows of the band: sum the K parts in part order, write once
-    if (!any_failed && bs.P > 1) {
-        float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
-        for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
-            const int rr = t / a.B, b = t - rr * a.B;
-            const int g = rr >> 5, l = rr & 31;
-            float sum = 0.0f;
-            for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
-            outb[t] = sum;
-        }
-    }
+    // 4. rows of the band: sum the K parts (and combine the pair) in part order, write once
+    if (!any_failed && (bs.P > 1 || a.mats > 1)) band_finish<BP>(a, bs, red, s, R0, rows);
     // 5. K slices: the last CTA of the band adds them up
     if (a.S > 1) splitk_fixup(a, cta, R0, rows);
 }

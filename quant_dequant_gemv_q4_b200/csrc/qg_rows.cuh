@@ -59,7 +59,12 @@ struct RowsArgs {
     int S;           // slices
     int Gs;          // CTAs per slice (row bands)
     int red_floats;  // floats of the per-CTA partial-row buffer
+    int mats;        // 1: y = W x; 2: the gate/up pair, two matrices (the second tensor map) on x
+    int act;         // mats == 2: 1 writes h = silu(gate) * up
 };
+
+// silu(v) * u, the FFN activation of the gate/up pair (silu(v) = v / (1 + e^-v))
+__device__ __forceinline__ float silu_mul(float v, float u) { return v / (1.0f + expf(-v)) * u; }
 
 // acc += lo(q)*lo(x) + hi(q)*hi(x), halves of q and x as fp16, products exact, sums fp32
 __device__ __forceinline__ void mfma2(float &acc, uint32_t q, uint32_t x)
@@ -295,19 +300,49 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 }
 
 // Pair layout of a band: G row groups of 32 rows, P K parts; pair q = g * P + p.
+// Pair layout of a band: Gm row groups of 32 rows per matrix, G = mats * Gm groups (matrix-major),
+// P K parts; pair q = g * P + p.
 struct BandShape {
-    int G, P;
+    int Gm, G, P;
 };
-__device__ __forceinline__ BandShape band_shape(int rows, int US_s, int NW)
+__device__ __forceinline__ BandShape band_shape(int rows, int US_s, int NW, int mats)
 {
     BandShape b;
-    b.G = (rows + 31) / 32;
+    b.Gm = (rows + 31) / 32;
+    b.G = mats * b.Gm;
     b.P = max(1, min(NW / max(b.G, 1), US_s));
     return b;
 }
 
+// The band's finished rows: sum the K parts of every matrix in part order from the partial rows
+// red[pair][32][BP] and write y (one slice: y itself, through the pair's activation) or this
+// slice's partial rows part[s][mats][N][B].
+template <int BP>
+__device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &bs, const float *red,
+                                            int s, int64_t R0, int rows)
+{
+    const int64_t NB = a.N * a.B;
+    for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
+        const int rr = t / a.B, b = t - rr * a.B;
+        const int g = rr >> 5, l = rr & 31;
+        float v[2] = {0.0f, 0.0f};
+        for (int m = 0; m < a.mats; ++m) {
+            float sum = 0.0f;
+            for (int p = 0; p < bs.P; ++p)
+                sum += red[((size_t)((m * bs.Gm + g) * bs.P + p) * 32 + l) * BP + b];
+            v[m] = sum;
+        }
+        const int64_t idx = R0 * a.B + t;
+        if (a.S == 1) {
+            a.out[idx] = (a.mats == 2 && a.act) ? silu_mul(v[0], v[1]) : v[0];
+        } else {
+            for (int m = 0; m < a.mats; ++m) a.out[((int64_t)s * a.mats + m) * NB + idx] = v[m];
+        }
+    }
+}
+
 // Split-K across CTAs without a second kernel.  CTA (slice s, band) has written its band's
-// partial rows to out = part[s][N][B]; each makes its writes visible and bumps the band's
+// partial rows to out = part[s][mats][N][B]; each makes its writes visible and bumps the band's
 // counter, and the last of the S CTAs to arrive adds the S slices in slice order (so y does not
 // depend on arrival order), writes y and resets the counter for the next call.  Every CTA
 // arrives, also after a copy timeout, so the counters always return to zero.
@@ -327,15 +362,20 @@ __device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_
     const int64_t NB = a.N * a.B;
     for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
         const int64_t idx = R0 * a.B + t;
-        float sum = 0.0f;
-        for (int s2 = 0; s2 < a.S; ++s2) sum += __ldcg(a.out + s2 * NB + idx);
-        a.y[idx] = sum;
+        float v[2] = {0.0f, 0.0f};
+        for (int m = 0; m < a.mats; ++m) {
+            float sum = 0.0f;
+            for (int s2 = 0; s2 < a.S; ++s2) sum += __ldcg(a.out + ((int64_t)s2 * a.mats + m) * NB + idx);
+            v[m] = sum;
+        }
+        a.y[idx] = (a.mats == 2 && a.act) ? silu_mul(v[0], v[1]) : v[0];
     }
 }
 
 template <int FMT, int BP>
 __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
-    rows_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap)
+    rows_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap,
+                     const __grid_constant__ CUtensorMap tmap2)
 {
     constexpr int NW = RowsWarps<FMT, BP>::value;
     constexpr int UB = RowsFmt<FMT>::kUnitBytes;
@@ -355,7 +395,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     const int US_s = min(a.US, a.UPR - s * a.US);
     const int64_t R0 = ((int64_t)cta * a.N) / a.Gs, R1 = ((int64_t)(cta + 1) * a.N) / a.Gs;
     const int rows = (int)(R1 - R0);
-    const BandShape bs = band_shape(rows, US_s, NW);
+    const BandShape bs = band_shape(rows, US_s, NW, a.mats);
     const int npairs = bs.G * bs.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;  // first unit column of this slice
@@ -380,9 +420,9 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     auto issue = [&](int i) {
         const uint32_t bar = bar0 + 8 * (i % kRowsStages);
         mbar_arrive_expect_tx(bar, BOX);
-        const int g = iq / bs.P;
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &tmap, (ucol0 + iu) * INNER,
-                    (int)(R0 + 32 * g), bar);
+        const int g = iq / bs.P;  // matrix g / Gm, row group g % Gm
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), g < bs.Gm ? &tmap : &tmap2,
+                    (ucol0 + iu) * INNER, (int)(R0 + 32 * (g % bs.Gm)), bar);
         if (++iu == iub) {
             iq += NW;
             if (iq < npairs) pair_units(iq, iu, iub);
@@ -393,6 +433,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     //    into the ring
     if (nsteps > 0 && lane == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+        if (a.mats > 1)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap2)) : "memory");
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
@@ -439,8 +481,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
                 issue(step + kRowsStages);
             }
         }
-        if (bs.P == 1) {
-            // a single K part: the row is complete, write it
+        if (bs.P == 1 && a.mats == 1) {
+            // a single K part of a single matrix: the row is complete, write it
             const int rr = (q / bs.P) * 32 + lane;
             if (rr < rows) {
                 float *dst = a.out + ((int64_t)s * a.N + R0 + rr) * a.B;
@@ -453,17 +495,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         }
     }
     const bool any_failed = __syncthreads_or(failed ? 1 : 0);
-    // 4. rows of the band: sum the K parts in part order, write once
-    if (!any_failed && bs.P > 1) {
-        float *outb = a.out + ((int64_t)s * a.N + R0) * a.B;
-        for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
-            const int rr = t / a.B, b = t - rr * a.B;
-            const int g = rr >> 5, l = rr & 31;
-            float sum = 0.0f;
-            for (int p = 0; p < bs.P; ++p) sum += red[((size_t)(g * bs.P + p) * 32 + l) * BP + b];
-            outb[t] = sum;
-        }
-    }
+    // 4. rows of the band: sum the K parts (and combine the pair) in part order, write once
+    if (!any_failed && (bs.P > 1 || a.mats > 1)) band_finish<BP>(a, bs, red, s, R0, rows);
     // 5. K slices: the last CTA of the band adds them up
     if (a.S > 1) splitk_fixup(a, cta, R0, rows);
 }

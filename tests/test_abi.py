@@ -155,3 +155,19 @@ def test_status_strings(L):
 def test_probe_argument_checks(L):
     assert L.qg_hbm_copy(FAKE, FAKE, 17, None) == qg.QG_ERR_ALIGN
     assert L.qg_hbm_read(0, 16, FAKE, None) == qg.QG_ERR_NULL
+
+
+def test_gate_up_rejects_bad_arguments(L):
+    f = L.qg_gemv_gate_up_silu
+    assert f(FAKE, FAKE, 5, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_FMT
+    assert f(FAKE, FAKE, 12, 4, 255, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
+    assert f(FAKE, None, 12, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_NULL
+    assert f(None, FAKE, 12, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_NULL
+    assert f(FAKE, FAKE + 8, 12, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_ALIGN
+    assert f(FAKE, FAKE, 12, 4, 256, FAKE, 0, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, FAKE, 12, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, FAKE, 12, 4, 256, None, 1, FAKE, None) == qg.QG_ERR_NULL
+    assert f(FAKE, FAKE, 12, 4, 256, FAKE, 1, FAKE + 2, None) == qg.QG_ERR_ALIGN
+    # the fused path needs whole 256-weight units per row (Q8_0 K = 96 is a valid tensor)
+    assert f(FAKE, FAKE, 8, 4, 96, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
+    assert f(None, None, 12, 0, 256, None, 1, None, None) == qg.QG_OK

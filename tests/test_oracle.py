@@ -291,3 +291,44 @@ def test_invalid_arguments_raise(orc):
     x = synth.activations(256, 1, seed=0)
     with pytest.raises(ValueError):
         orc.gemv(W, Q4_K, 1, 256, x, 1, rows=np.array([1]))
+
+
+# ------------------------------------------------------------------------------------------------
+# The gate/up pair's activation (B70 plan, "Phase 3: Maximum Useful Fusion": SiLU-mul epilogue)
+# ------------------------------------------------------------------------------------------------
+
+def test_silu_closed_forms(orc):
+    """silu(v) = v / (1 + e^-v): silu(0) = 0, silu(1) = e/(1+e), silu(-1) = 1/(1+e) - 1 ... and the
+    odd-part identity silu(v) - silu(-v) = v."""
+    e = np.e
+    assert orc.silu(0.0) == 0.0
+    assert abs(orc.silu(1.0) - e / (1.0 + e)) < 1e-15
+    assert abs(orc.silu(-1.0) - (-1.0 / (1.0 + e))) < 1e-15
+    v = np.linspace(-30, 30, 1201)
+    assert np.allclose(orc.silu(v) - orc.silu(-v), v, rtol=0, atol=1e-12)
+    # asymptotes: silu(v) -> v for large v, -> 0 (from below) for very negative v
+    assert orc.silu(40.0) == 40.0
+    assert -1e-15 < orc.silu(-40.0) < 0.0
+    assert orc.silu(-1000.0) == 0.0  # e^1000 overflows to inf: v / inf
+    # derivative 1/2 at 0 (central difference)
+    hstep = 1e-6
+    assert abs((orc.silu(hstep) - orc.silu(-hstep)) / (2 * hstep) - 0.5) < 1e-9
+
+
+def test_gate_up_silu_composition(orc):
+    """h is silu of the first GEMV times the second, row by row, and a row subset agrees."""
+    N, K, B = 12, 512, 3
+    Wg = synth.q4k_weights(N, K, seed=21)
+    Wu = synth.q4k_weights(N, K, seed=22)
+    x = synth.activations(K, B, seed=23)
+    h, g, Ag, u, Au = orc.gate_up_silu(Wg, Wu, Q4_K, N, K, x, B)
+    g2, _ = orc.gemv(Wg, Q4_K, N, K, x, B)
+    u2, _ = orc.gemv(Wu, Q4_K, N, K, x, B)
+    assert np.array_equal(g, g2) and np.array_equal(u, u2)
+    assert np.array_equal(h, g2 / (1.0 + np.exp(-g2)) * u2)
+    rows = np.array([0, 5, 11])
+    hr, *_ = orc.gate_up_silu(Wg, Wu, Q4_K, N, K, x, B, rows=rows)
+    assert np.array_equal(hr, h[rows])
+    # with W_u = W_g, h = silu(g) * g >= 0 wherever g >= 0
+    hs, gs, *_ = orc.gate_up_silu(Wg, Wg, Q4_K, N, K, x, B)
+    assert np.all(hs[gs >= 0] >= 0)
