@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <map>
@@ -273,29 +274,38 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     return best;  // smem == 0 if nothing fits
 }
 
-const void *rows_kernel_ptr(int fmt, int BP, bool tensor)
+const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 {
-    if (tensor) {
-        switch (BP) {
-        case 1: return reinterpret_cast<const void *>(&mma_gemv_kernel<1>);
-        case 2: return reinterpret_cast<const void *>(&mma_gemv_kernel<2>);
-        case 4: return reinterpret_cast<const void *>(&mma_gemv_kernel<4>);
-        default: return reinterpret_cast<const void *>(&mma_gemv_kernel<8>);
-        }
-    }
-#define QG_PICKR(F)                                                            \
+#define QG_BP_SWITCH(KERNEL)                                                   \
     switch (BP) {                                                              \
-    case 1: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 1>);    \
-    case 2: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 2>);    \
-    case 4: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 4>);    \
-    default: return reinterpret_cast<const void *>(&rows_gemv_kernel<F, 8>);   \
+    case 1: return reinterpret_cast<const void *>(&KERNEL(1));                 \
+    case 2: return reinterpret_cast<const void *>(&KERNEL(2));                 \
+    case 4: return reinterpret_cast<const void *>(&KERNEL(4));                 \
+    default: return reinterpret_cast<const void *>(&KERNEL(8));                \
+    }
+#define QG_MMA1(bp) mma_gemv_kernel<bp, 1>
+#define QG_MMA2(bp) mma_gemv_kernel<bp, 2>
+#define QG_ROWS_Q4K1(bp) rows_gemv_kernel<kFmtQ4_K, bp, 1>
+#define QG_ROWS_Q4K2(bp) rows_gemv_kernel<kFmtQ4_K, bp, 2>
+#define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
+#define QG_ROWS_Q802(bp) rows_gemv_kernel<kFmtQ8_0, bp, 2>
+    if (tensor) {
+        if (mats == 2) { QG_BP_SWITCH(QG_MMA2) }
+        QG_BP_SWITCH(QG_MMA1)
     }
     if (fmt == kFmtQ8_0) {
-        QG_PICKR(kFmtQ8_0)
-    } else {
-        QG_PICKR(kFmtQ4_K)
+        if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q802) }
+        QG_BP_SWITCH(QG_ROWS_Q801)
     }
-#undef QG_PICKR
+    if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q4K2) }
+    QG_BP_SWITCH(QG_ROWS_Q4K1)
+#undef QG_ROWS_Q802
+#undef QG_ROWS_Q801
+#undef QG_ROWS_Q4K2
+#undef QG_ROWS_Q4K1
+#undef QG_MMA2
+#undef QG_MMA1
+#undef QG_BP_SWITCH
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link needed).
@@ -336,16 +346,14 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
                 cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, int *err,
                 unsigned *cnt, float *part, bool pdl, const void *W2 = nullptr, int act = 0)
 {
-    const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor);
+    const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor, W2 ? 2 : 1);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
     if (rc != QG_OK) return rc;
-    CUtensorMap map, map2;
-    if ((rc = make_weight_map(W, fmt, N, K, &map)) != QG_OK) return rc;
-    if (W2) {
-        if ((rc = make_weight_map(W2, fmt, N, K, &map2)) != QG_OK) return rc;
-    } else {
-        map2 = map;
-    }
+    WeightMaps<2> maps;  // the first map alone is the WeightMaps<1> of a single matrix
+    static_assert(offsetof(WeightMaps<2>, m) == 0 && sizeof(WeightMaps<1>) == sizeof(CUtensorMap),
+                  "WeightMaps<1> is a prefix of WeightMaps<2>");
+    if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
+    if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
     RowsArgs a;
     a.x = x;
     a.out = (p.S > 1) ? part : y;
@@ -359,7 +367,6 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     a.S = p.S;
     a.Gs = p.Gs;
     a.red_floats = p.red_floats;
-    a.mats = W2 ? 2 : 1;
     a.act = act;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
@@ -371,7 +378,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void *args[] = {&a, &map, &map2};
+    void *args[] = {&a, &maps};  // the kernel reads sizeof(WeightMaps<MATS>) bytes of it
     if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return QG_ERR_CUDA;
     return QG_OK;
 }

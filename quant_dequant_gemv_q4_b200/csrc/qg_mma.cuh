@@ -211,10 +211,9 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 // Shared memory of the tensor-core kernel, in order: ring [NW][2][32 x 144 B], x fragments
 // [US][16][BP][4] uint2, x sums [US][8][BP], per-warp tables [NW][256] floats, partial rows
 // [red_floats], mbarriers [NW][2].
-template <int BP>
+template <int BP, int MATS>
 __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
-    mma_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap,
-                    const __grid_constant__ CUtensorMap tmap2)
+    mma_gemv_kernel(const RowsArgs a, const __grid_constant__ WeightMaps<MATS> maps)
 {
     constexpr int NW = MmaWarps<BP>::value;
     constexpr int UB = 144;
@@ -235,7 +234,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     const int US_s = min(a.US, a.UPR - s * a.US);
     const int64_t R0 = ((int64_t)cta * a.N) / a.Gs, R1 = ((int64_t)(cta + 1) * a.N) / a.Gs;
     const int rows = (int)(R1 - R0);
-    const BandShape bs = band_shape(rows, US_s, NW, a.mats);
+    const BandShape bs = band_shape<MATS>(rows, US_s, NW);
     const int npairs = bs.G * bs.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;
@@ -255,24 +254,31 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     uint8_t *myring = ring + warp * kRowsStages * BOX;
     const uint32_t bar0 = smem_u32(bars + warp * kRowsStages);
     int iq = warp, iu = 0, iub = 0;
-    if (iq < npairs) pair_units(iq, iu, iub);
+    int ig_row = 0, ig_map = 0;  // the pair's first row in its matrix, and its matrix
+    auto cursor_pair = [&]() {
+        pair_units(iq, iu, iub);
+        const int g = iq / bs.P;  // group g of matrix 0, or group g - Gm of matrix 1
+        const bool second = (MATS > 1) && g >= bs.Gm;
+        ig_row = (int)R0 + 32 * (second ? g - bs.Gm : g);
+        ig_map = second ? MATS - 1 : 0;
+    };
+    if (iq < npairs) cursor_pair();
     auto issue = [&](int i) {
         const uint32_t bar = bar0 + 8 * (i % kRowsStages);
         mbar_arrive_expect_tx(bar, BOX);
-        const int g = iq / bs.P;  // matrix g / Gm, row group g % Gm
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), g < bs.Gm ? &tmap : &tmap2,
-                    (ucol0 + iu) * INNER, (int)(R0 + 32 * (g % bs.Gm)), bar);
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
+                    ig_row, bar);
         if (++iu == iub) {
             iq += NW;
-            if (iq < npairs) pair_units(iq, iu, iub);
+            if (iq < npairs) cursor_pair();
         }
     };
 
     // 1. weight prefetch (independent of the previous kernel on the stream)
     if (nsteps > 0 && lane == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
-        if (a.mats > 1)
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap2)) : "memory");
+#pragma unroll
+        for (int m = 0; m < MATS; ++m)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
 #pragma unroll
         for (int b = 0; b < BP; ++b) v[b] = dtab[lane * BP + b] + accM[b];
         __syncwarp();
-        if (bs.P == 1 && a.mats == 1) {
+        if (bs.P == 1 && MATS == 1) {
             const int rr = (q / bs.P) * 32 + lane;
             if (rr < rows) {
                 float *dst = a.out + ((int64_t)s * a.N + R0 + rr) * a.B;
@@ -345,9 +351,9 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     }
     const bool any_failed = __syncthreads_or(failed ? 1 : 0);
     // 4. rows of the band: sum the K parts (and combine the pair) in part order, write once
-    if (!any_failed && (bs.P > 1 || a.mats > 1)) band_finish<BP>(a, bs, red, s, R0, rows);
+    if (!any_failed && (bs.P > 1 || MATS > 1)) band_finish<BP, MATS>(a, bs, red, s, R0, rows);
     // 5. K slices: the last CTA of the band adds them up
-    if (a.S > 1) splitk_fixup(a, cta, R0, rows);
+    if (a.S > 1) splitk_fixup<MATS>(a, cta, R0, rows);
 }
 
 }  // namespace qg

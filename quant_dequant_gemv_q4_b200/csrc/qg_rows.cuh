@@ -59,8 +59,7 @@ struct RowsArgs {
     int S;           // slices
     int Gs;          // CTAs per slice (row bands)
     int red_floats;  // floats of the per-CTA partial-row buffer
-    int mats;        // 1: y = W x; 2: the gate/up pair, two matrices (the second tensor map) on x
-    int act;         // mats == 2: 1 writes h = silu(gate) * up
+    int act;  // gate/up pair (MATS == 2): 1 writes h = silu(gate) * up
 };
 
 // silu(v) * u, the FFN activation of the gate/up pair (silu(v) = v / (1 + e^-v))
@@ -305,19 +304,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 struct BandShape {
     int Gm, G, P;
 };
-__device__ __forceinline__ BandShape band_shape(int rows, int US_s, int NW, int mats)
+template <int MATS>
+__device__ __forceinline__ BandShape band_shape(int rows, int US_s, int NW)
 {
     BandShape b;
     b.Gm = (rows + 31) / 32;
-    b.G = mats * b.Gm;
+    b.G = MATS * b.Gm;
     b.P = max(1, min(NW / max(b.G, 1), US_s));
     return b;
 }
 
 // The band's finished rows: sum the K parts of every matrix in part order from the partial rows
 // red[pair][32][BP] and write y (one slice: y itself, through the pair's activation) or this
-// slice's partial rows part[s][mats][N][B].
-template <int BP>
+// slice's partial rows part[s][MATS][N][B].
+template <int BP, int MATS>
 __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &bs, const float *red,
                                             int s, int64_t R0, int rows)
 {
@@ -325,8 +325,9 @@ __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &
     for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
         const int rr = t / a.B, b = t - rr * a.B;
         const int g = rr >> 5, l = rr & 31;
-        float v[2] = {0.0f, 0.0f};
-        for (int m = 0; m < a.mats; ++m) {
+        float v[MATS];
+#pragma unroll
+        for (int m = 0; m < MATS; ++m) {
             float sum = 0.0f;
             for (int p = 0; p < bs.P; ++p)
                 sum += red[((size_t)((m * bs.Gm + g) * bs.P + p) * 32 + l) * BP + b];
@@ -334,9 +335,11 @@ __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &
         }
         const int64_t idx = R0 * a.B + t;
         if (a.S == 1) {
-            a.out[idx] = (a.mats == 2 && a.act) ? silu_mul(v[0], v[1]) : v[0];
+            if (MATS == 2) a.out[idx] = a.act ? silu_mul(v[0], v[MATS - 1]) : v[0];
+            else a.out[idx] = v[0];
         } else {
-            for (int m = 0; m < a.mats; ++m) a.out[((int64_t)s * a.mats + m) * NB + idx] = v[m];
+#pragma unroll
+            for (int m = 0; m < MATS; ++m) a.out[((int64_t)s * MATS + m) * NB + idx] = v[m];
         }
     }
 }
@@ -346,6 +349,7 @@ __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &
 // counter, and the last of the S CTAs to arrive adds the S slices in slice order (so y does not
 // depend on arrival order), writes y and resets the counter for the next call.  Every CTA
 // arrives, also after a copy timeout, so the counters always return to zero.
+template <int MATS>
 __device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_t R0, int rows)
 {
     __shared__ int s_last;
@@ -362,20 +366,29 @@ __device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_
     const int64_t NB = a.N * a.B;
     for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
         const int64_t idx = R0 * a.B + t;
-        float v[2] = {0.0f, 0.0f};
-        for (int m = 0; m < a.mats; ++m) {
+        float v[MATS];
+#pragma unroll
+        for (int m = 0; m < MATS; ++m) {
             float sum = 0.0f;
-            for (int s2 = 0; s2 < a.S; ++s2) sum += __ldcg(a.out + ((int64_t)s2 * a.mats + m) * NB + idx);
+            for (int s2 = 0; s2 < a.S; ++s2) sum += __ldcg(a.out + ((int64_t)s2 * MATS + m) * NB + idx);
             v[m] = sum;
         }
-        a.y[idx] = (a.mats == 2 && a.act) ? silu_mul(v[0], v[1]) : v[0];
+        if (MATS == 2) a.y[idx] = a.act ? silu_mul(v[0], v[MATS - 1]) : v[0];
+        else a.y[idx] = v[0];
     }
 }
 
-template <int FMT, int BP>
+// The weight tensor maps of a launch: one per matrix (a kernel parameter, in the parameter space
+// the TMA reads descriptors from).
+template <int MATS> struct WeightMaps {
+    CUtensorMap m[MATS];
+};
+
+// MATS = 1: y = W x.  MATS = 2: the gate/up pair, the second matrix through maps.m[1] (the band's
+// row groups of both matrices, matrix-major), combined by band_finish / splitk_fixup.
+template <int FMT, int BP, int MATS>
 __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
-    rows_gemv_kernel(const RowsArgs a, const __grid_constant__ CUtensorMap tmap,
-                     const __grid_constant__ CUtensorMap tmap2)
+    rows_gemv_kernel(const RowsArgs a, const __grid_constant__ WeightMaps<MATS> maps)
 {
     constexpr int NW = RowsWarps<FMT, BP>::value;
     constexpr int UB = RowsFmt<FMT>::kUnitBytes;
@@ -395,7 +408,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     const int US_s = min(a.US, a.UPR - s * a.US);
     const int64_t R0 = ((int64_t)cta * a.N) / a.Gs, R1 = ((int64_t)(cta + 1) * a.N) / a.Gs;
     const int rows = (int)(R1 - R0);
-    const BandShape bs = band_shape(rows, US_s, NW, a.mats);
+    const BandShape bs = band_shape<MATS>(rows, US_s, NW);
     const int npairs = bs.G * bs.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;  // first unit column of this slice
@@ -416,25 +429,32 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     const uint32_t bar0 = smem_u32(bars + warp * kRowsStages);
     // issue cursor (lane 0): pair iq, unit iu
     int iq = warp, iu = 0, iub = 0;
-    if (iq < npairs) pair_units(iq, iu, iub);
+    int ig_row = 0, ig_map = 0;  // the pair's first row in its matrix, and its matrix
+    auto cursor_pair = [&]() {
+        pair_units(iq, iu, iub);
+        const int g = iq / bs.P;  // group g of matrix 0, or group g - Gm of matrix 1
+        const bool second = (MATS > 1) && g >= bs.Gm;
+        ig_row = (int)R0 + 32 * (second ? g - bs.Gm : g);
+        ig_map = second ? MATS - 1 : 0;
+    };
+    if (iq < npairs) cursor_pair();
     auto issue = [&](int i) {
         const uint32_t bar = bar0 + 8 * (i % kRowsStages);
         mbar_arrive_expect_tx(bar, BOX);
-        const int g = iq / bs.P;  // matrix g / Gm, row group g % Gm
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), g < bs.Gm ? &tmap : &tmap2,
-                    (ucol0 + iu) * INNER, (int)(R0 + 32 * (g % bs.Gm)), bar);
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
+                    ig_row, bar);
         if (++iu == iub) {
             iq += NW;
-            if (iq < npairs) pair_units(iq, iu, iub);
+            if (iq < npairs) cursor_pair();
         }
     };
 
     // 1. weight prefetch (independent of the previous kernel on the stream): the first steps
     //    into the ring
     if (nsteps > 0 && lane == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
-        if (a.mats > 1)
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap2)) : "memory");
+#pragma unroll
+        for (int m = 0; m < MATS; ++m)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
@@ -481,7 +501,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
                 issue(step + kRowsStages);
             }
         }
-        if (bs.P == 1 && a.mats == 1) {
+        if (bs.P == 1 && MATS == 1) {
             // a single K part of a single matrix: the row is complete, write it
             const int rr = (q / bs.P) * 32 + lane;
             if (rr < rows) {
@@ -496,9 +516,9 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     }
     const bool any_failed = __syncthreads_or(failed ? 1 : 0);
     // 4. rows of the band: sum the K parts (and combine the pair) in part order, write once
-    if (!any_failed && (bs.P > 1 || a.mats > 1)) band_finish<BP>(a, bs, red, s, R0, rows);
+    if (!any_failed && (bs.P > 1 || MATS > 1)) band_finish<BP, MATS>(a, bs, red, s, R0, rows);
     // 5. K slices: the last CTA of the band adds them up
-    if (a.S > 1) splitk_fixup(a, cta, R0, rows);
+    if (a.S > 1) splitk_fixup<MATS>(a, cta, R0, rows);
 }
 
 }  // namespace qg
