@@ -124,6 +124,16 @@ int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int
 int qg_gemv_gate_up_silu(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K,
                          const uint16_t *x, int B, float *h, void *stream);
 
+/* The output projection with the residual add fused into its epilogue:
+ *     y[n,b] = (dequant(W) . x)[n,b] + r[n,b]
+ * ("Qwen3.6 27B Single-B70 Maximum-Speed Requirements And Execution Plan", "Phase 3: Maximum
+ * Useful Fusion": the output projection plus residual).  r is device fp32 [N][B], 4-byte aligned,
+ * read only; it may be y itself (an in-place update of the residual stream: each element is read
+ * once, by the thread that then writes it).  Arguments and errors otherwise as qg_gemv, plus
+ * QG_ERR_SHAPE when K % 256 != 0.  The sum is the GEMV's fp32 result plus r, rounded once. */
+int qg_gemv_residual(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
+                     const float *r, float *y, void *stream);
+
 /* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant,
  * for DIRECT / FACTORED / TENSOR when K % 256 != 0, and for TENSOR with Q8_0.  The other variants
  * take both formats. */

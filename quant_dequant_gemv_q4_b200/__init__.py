@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.qg_gemv_noalloc.restype = I
         L.qg_gemv_gate_up_silu.argtypes = [P, P, I, I64, I64, P, I, P, P]
         L.qg_gemv_gate_up_silu.restype = I
+        L.qg_gemv_residual.argtypes = [P, I, I64, I64, P, I, P, P, P]
+        L.qg_gemv_residual.restype = I
         L.qg_dequant_f32.argtypes = [P, I, I64, I64, P, P]
         L.qg_dequant_f32.restype = I
         L.qg_pack_reference.argtypes = [I, I64, I64, P, P, P, P, P, P]
@@ -144,6 +146,12 @@ def qg_gemv_gate_up_silu(Wg, Wu, fmt: int, N: int, K: int, x, B: int, h, stream=
     """h = silu(dequant(Wg) . x) * (dequant(Wu) . x) in one launch (fp32 h [N][B])."""
     _ok(lib().qg_gemv_gate_up_silu(_ptr(Wg), _ptr(Wu), int(fmt), int(N), int(K), _ptr(x), int(B),
                                    _ptr(h), _stream(stream)), "qg_gemv_gate_up_silu")
+
+
+def qg_gemv_residual(W, fmt: int, N: int, K: int, x, B: int, r, y, stream=None) -> None:
+    """y = dequant(W) . x + r (r may be y itself: in-place residual update)."""
+    _ok(lib().qg_gemv_residual(_ptr(W), int(fmt), int(N), int(K), _ptr(x), int(B), _ptr(r), _ptr(y),
+                               _stream(stream)), "qg_gemv_residual")
 
 
 def qg_gemv_noalloc(W, fmt: int, N: int, K: int, x, B: int, y, stream=None) -> None:

@@ -344,7 +344,8 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
 // word; `part` holds S*N*B floats when S > 1.
 int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
                 cudaStream_t st, const DeviceInfo &di, int dev, const RowsPlan &p, int *err,
-                unsigned *cnt, float *part, bool pdl, const void *W2 = nullptr, int act = 0)
+                unsigned *cnt, float *part, bool pdl, const void *W2 = nullptr, int act = 0,
+                const float *res = nullptr)
 {
     const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor, W2 ? 2 : 1);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
@@ -368,6 +369,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     a.Gs = p.Gs;
     a.red_floats = p.red_floats;
     a.act = act;
+    a.res = res;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
     cfg.blockDim = dim3(p.NW * 32);
@@ -548,9 +550,46 @@ int gate_up_impl(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K, 
     return QG_OK;
 }
 
+// y = W x + r with the residual add in the streaming kernels' epilogue.
+int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
+                  const float *r, float *y, void *stream)
+{
+    int rc = check_common(W, fmt, N, K);
+    if (rc != QG_OK) return rc;
+    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (N == 0) return QG_OK;
+    if (!x || !y || !r) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0 ||
+        reinterpret_cast<uintptr_t>(r) % 4 != 0)
+        return QG_ERR_ALIGN;
+    if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
+    DeviceInfo di;
+    int dev = 0;
+    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    const int var = auto_variant(fmt, K, B);
+    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
+    if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+    WsView ws;
+    const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
+    const size_t ncnt = (p.S > 1) ? (size_t)p.Gs : 0;
+    if ((rc = get_workspace(dev, stream, ncnt, 0, part_f, &ws)) != QG_OK) return rc;
+    if ((rc = launch_rows(W, fmt, N, K, x, B, y, static_cast<cudaStream_t>(stream), di, dev, p, ws.err,
+                          ws.cnt, ws.part, true, nullptr, 0, r)) != QG_OK)
+        return rc;
+    t_last_variant = var;
+    t_last_splits = p.S;
+    return QG_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int qg_gemv_residual(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
+                     const float *r, float *y, void *stream)
+{
+    return residual_impl(W, fmt, N, K, x, B, r, y, stream);
+}
 
 int qg_gemv_gate_up_silu(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K,
                          const uint16_t *x, int B, float *h, void *stream)

@@ -340,8 +340,13 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
         if (bs.P == 1 && MATS == 1) {
             const int rr = (q / bs.P) * 32 + lane;
             if (rr < rows) {
-                float *dst = a.out + ((int64_t)s * a.N + R0 + rr) * a.B;
-                for (int b = 0; b < a.B; ++b) dst[b] = v[b];
+                const int64_t row0 = (R0 + rr) * a.B;
+                float *dst = a.out + (int64_t)s * a.N * a.B + row0;
+                if (a.S == 1 && a.res) {
+                    for (int b = 0; b < a.B; ++b) dst[b] = v[b] + a.res[row0 + b];
+                } else {
+                    for (int b = 0; b < a.B; ++b) dst[b] = v[b];
+                }
             }
         } else {
             float *r = red + ((size_t)q * 32 + lane) * BP;

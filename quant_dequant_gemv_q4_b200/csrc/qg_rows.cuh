@@ -60,6 +60,7 @@ struct RowsArgs {
     int Gs;          // CTAs per slice (row bands)
     int red_floats;  // floats of the per-CTA partial-row buffer
     int act;  // gate/up pair (MATS == 2): 1 writes h = silu(gate) * up
+    const float *res;  // MATS == 1: y = W x + res (fp32 [N][B], may alias y), or nullptr
 };
 
 // silu(v) * u, the FFN activation of the gate/up pair (silu(v) = v / (1 + e^-v))
@@ -336,7 +337,7 @@ __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &
         const int64_t idx = R0 * a.B + t;
         if (a.S == 1) {
             if (MATS == 2) a.out[idx] = a.act ? silu_mul(v[0], v[MATS - 1]) : v[0];
-            else a.out[idx] = v[0];
+            else a.out[idx] = a.res ? v[0] + a.res[idx] : v[0];
         } else {
 #pragma unroll
             for (int m = 0; m < MATS; ++m) a.out[((int64_t)s * MATS + m) * NB + idx] = v[m];
@@ -374,7 +375,7 @@ __device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_
             v[m] = sum;
         }
         if (MATS == 2) a.y[idx] = a.act ? silu_mul(v[0], v[MATS - 1]) : v[0];
-        else a.y[idx] = v[0];
+        else a.y[idx] = a.res ? v[0] + a.res[idx] : v[0];
     }
 }
 
@@ -505,8 +506,13 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
             // a single K part of a single matrix: the row is complete, write it
             const int rr = (q / bs.P) * 32 + lane;
             if (rr < rows) {
-                float *dst = a.out + ((int64_t)s * a.N + R0 + rr) * a.B;
-                for (int b = 0; b < a.B; ++b) dst[b] = acc[b];
+                const int64_t row0 = (R0 + rr) * a.B;
+                float *dst = a.out + (int64_t)s * a.N * a.B + row0;
+                if (a.S == 1 && a.res) {
+                    for (int b = 0; b < a.B; ++b) dst[b] = acc[b] + a.res[row0 + b];
+                } else {
+                    for (int b = 0; b < a.B; ++b) dst[b] = acc[b];
+                }
             }
         } else {
             float *r = red + ((size_t)q * 32 + lane) * BP;

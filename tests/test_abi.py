@@ -171,3 +171,13 @@ def test_gate_up_rejects_bad_arguments(L):
     # the fused path needs whole 256-weight units per row (Q8_0 K = 96 is a valid tensor)
     assert f(FAKE, FAKE, 8, 4, 96, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
     assert f(None, None, 12, 0, 256, None, 1, None, None) == qg.QG_OK
+
+
+def test_residual_rejects_bad_arguments(L):
+    f = L.qg_gemv_residual
+    assert f(FAKE, 5, 4, 256, FAKE, 1, FAKE, FAKE, None) == qg.QG_ERR_FMT
+    assert f(FAKE, 12, 4, 256, FAKE, 1, None, FAKE, None) == qg.QG_ERR_NULL
+    assert f(FAKE, 12, 4, 256, FAKE, 1, FAKE + 2, FAKE, None) == qg.QG_ERR_ALIGN
+    assert f(FAKE, 12, 4, 256, FAKE, 9, FAKE, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, 8, 4, 96, FAKE, 1, FAKE, FAKE, None) == qg.QG_ERR_SHAPE
+    assert f(None, 12, 0, 256, None, 1, None, None, None) == qg.QG_OK
