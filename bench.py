@@ -39,6 +39,7 @@ METRIC = "Q4_K GEMV effective HBM GB/s and % of B200 HBM roofline (\u00b5s/call)
 UNIT = "GB/s"
 HEADLINE = synth.Gemv("ffn_gate", synth.Q4_K, 17408, 5120, 1, 0)
 HEADLINE_B8 = synth.Gemv("ffn_gate_b8", synth.Q4_K, 17408, 5120, 8, 0)
+HEADLINE_B16 = synth.Gemv("ffn_gate_b16", synth.Q4_K, 17408, 5120, 16, 0)
 HEADLINE_SEED = 4  # the batched-verify workload's seed
 FALLBACK_HBM_GBS = 6650.0
 
@@ -568,6 +569,16 @@ def main(argv=None):
           "steps": steps8}
     del cs8
 
+    # B = 16 (verify width beyond 8: the tensor-core kernel's two 8-column tiles)
+    cs16 = CallSet([HEADLINE_B16], HEADLINE_SEED, device, l2)
+    secs16, _ = time_callset(cs16, steps8, args.warmup, args.variant, None)
+    secs16 = dist_max(secs16, device)
+    b16 = {"us_per_call": round(secs16 * 1e6 / steps8, 3),
+           "gbs": round(cs16.bytes_per_step * steps8 / secs16 / 1e9, 1),
+           "frac_of_hbm": round(cs16.bytes_per_step * steps8 / secs16 / 1e9 / hbm, 4),
+           "splits": qg.qg_last_splits(), "steps": steps8}
+    del cs16
+
     # the fused FFN gate/up pair (one launch, two weight streams, h = silu(g) * u)
     gate_up = []
     for Bg in (1, 8):
@@ -645,6 +656,7 @@ def main(argv=None):
         "variant": variant_used,
         "roofline": roofline,
         "b8": b8,
+        "b16": b16,
         "gate_up_silu": gate_up,
         "clocks": clocks,
         "e2e": e2e,

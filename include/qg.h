@@ -1,7 +1,7 @@
 /*
  * qg.h -- C ABI of libqg, a B200 (sm_100a) dequant GEMV over GGML block-quantized weights:
  *
- *     y[N,B] = dequant(W[N,K]) . x[K,B]      x fp16, accumulation fp32, y fp32, 1 <= B <= 8
+ *     y[N,B] = dequant(W[N,K]) . x[K,B]      x fp16, accumulation fp32, y fp32, 1 <= B <= 16
  *
  * The operation is the mixed-quant GEMV of "HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle)"
  * (second prompt, section "SPEC": y = dequant(W[N,K]) @ x[K], the format chosen by a tensor-type
@@ -59,7 +59,7 @@ enum {
     QG_ERR_NULL = 1,    /* a required pointer is NULL */
     QG_ERR_FMT = 2,     /* unknown format flag */
     QG_ERR_SHAPE = 3,   /* N < 0, K < 1, or K not a multiple of the block size */
-    QG_ERR_BATCH = 4,   /* B outside 1..8 */
+    QG_ERR_BATCH = 4,   /* B outside 1..8, or outside 1..16 for Q4_K with K % 256 == 0 */
     QG_ERR_ALIGN = 5,   /* W not 16-byte aligned, x not 2-byte aligned or y not 4-byte aligned */
     QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
     QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
@@ -101,7 +101,8 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
  *   fmt    QG_FMT_Q4_K or QG_FMT_Q8_0
  *   N, K   rows and reduction length; N >= 0 (N == 0 does nothing); K >= 1, K % block == 0
  *   x      device, fp16 bits [K][B], 2-byte aligned, read only
- *   B      number of columns, 1..8
+ *   B      number of columns: 1..8; 1..16 for Q4_K with K % 256 == 0 (9..16 columns run on the
+ *          tensor-core kernel, every weight still read once)
  *   y      device, fp32 [N][B], 4-byte aligned, fully overwritten (not accumulated)
  *   stream a cudaStream_t (NULL = the legacy default stream); the call is asynchronous
  * Returns QG_OK once the work is enqueued. */

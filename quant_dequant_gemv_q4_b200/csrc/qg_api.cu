@@ -157,7 +157,10 @@ int get_workspace(int dev, void *stream, size_t nw, size_t slot_f, size_t part_f
 // ---------------------------------------------------------------------------------------------
 // Planning.
 // ---------------------------------------------------------------------------------------------
-int padded_cols(int B) { return B == 1 ? 1 : B == 2 ? 2 : B <= 4 ? 4 : 8; }
+// columns of x: 1..8 on every kernel, up to 16 on the tensor-core kernel (Q4_K, K % 256 == 0)
+constexpr int kMaxB = 16;
+
+int padded_cols(int B) { return B == 1 ? 1 : B == 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16; }
 
 struct Plan {
     int BP, S, US, Gs, G, xs_floats;
@@ -229,13 +232,13 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
     int NW;
     if (tensor)
-        NW = BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
+        NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
     else if (fmt == kFmtQ4_K)
         NW = BP >= 8 ? RowsWarps<kFmtQ4_K, 8>::value : RowsWarps<kFmtQ4_K, 1>::value;
     else
         NW = BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
     const size_t ring = (size_t)NW * kRowsStages * 32 * UB;
-    const size_t tabs = tensor ? (size_t)NW * 256 * sizeof(float) : 0;  // per-warp scale tables
+    const size_t tabs = tensor ? (size_t)NW * std::max(256, 32 * BP) * sizeof(float) : 0;  // per-warp tables
     const size_t bars = (size_t)NW * kRowsStages * 8;
     const int64_t UPR = K / 256;
     // K slices: the fewest for which x fits in shared memory and the row bands keep at least 85%
@@ -283,6 +286,14 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
     case 4: return reinterpret_cast<const void *>(&KERNEL(4));                 \
     default: return reinterpret_cast<const void *>(&KERNEL(8));                \
     }
+#define QG_BP_SWITCH16(KERNEL)                                                 \
+    switch (BP) {                                                              \
+    case 1: return reinterpret_cast<const void *>(&KERNEL(1));                 \
+    case 2: return reinterpret_cast<const void *>(&KERNEL(2));                 \
+    case 4: return reinterpret_cast<const void *>(&KERNEL(4));                 \
+    case 8: return reinterpret_cast<const void *>(&KERNEL(8));                 \
+    default: return reinterpret_cast<const void *>(&KERNEL(16));               \
+    }
 #define QG_MMA1(bp) mma_gemv_kernel<bp, 1>
 #define QG_MMA2(bp) mma_gemv_kernel<bp, 2>
 #define QG_ROWS_Q4K1(bp) rows_gemv_kernel<kFmtQ4_K, bp, 1>
@@ -290,8 +301,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
 #define QG_ROWS_Q802(bp) rows_gemv_kernel<kFmtQ8_0, bp, 2>
     if (tensor) {
-        if (mats == 2) { QG_BP_SWITCH(QG_MMA2) }
-        QG_BP_SWITCH(QG_MMA1)
+        if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
+        QG_BP_SWITCH16(QG_MMA1)
     }
     if (fmt == kFmtQ8_0) {
         if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q802) }
@@ -305,6 +316,7 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #undef QG_ROWS_Q4K1
 #undef QG_MMA2
 #undef QG_MMA1
+#undef QG_BP_SWITCH16
 #undef QG_BP_SWITCH
 }
 
@@ -425,7 +437,7 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
 {
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
-    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
     if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TENSOR) return QG_ERR_VARIANT;
     if (N == 0) return QG_OK;
     if (!x || !y) return QG_ERR_NULL;
@@ -438,6 +450,7 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
     if (var == QG_VARIANT_TENSOR && fmt != QG_FMT_Q4_K) return QG_ERR_VARIANT;
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -526,16 +539,17 @@ int gate_up_impl(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K, 
     int rc = check_common(Wg, fmt, N, K);
     if (rc != QG_OK) return rc;
     if ((rc = check_common(Wu, fmt, N, K)) != QG_OK) return rc;
-    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
     if (N == 0) return QG_OK;
     if (!x || !h) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(h) % 4 != 0)
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
+    const int var = auto_variant(fmt, K, B);
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
-    const int var = auto_variant(fmt, K, B);
     const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR, 2);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     WsView ws;
@@ -556,17 +570,18 @@ int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *
 {
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
-    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
     if (N == 0) return QG_OK;
     if (!x || !y || !r) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0 ||
         reinterpret_cast<uintptr_t>(r) % 4 != 0)
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
+    const int var = auto_variant(fmt, K, B);
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
-    const int var = auto_variant(fmt, K, B);
     const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     WsView ws;
@@ -694,7 +709,7 @@ const char *qg_status_string(int status)
     case QG_ERR_NULL: return "a required pointer is NULL";
     case QG_ERR_FMT: return "unknown format flag";
     case QG_ERR_SHAPE: return "invalid shape (N < 0, K < 1 or K not a multiple of the block size)";
-    case QG_ERR_BATCH: return "B must be in 1..8";
+    case QG_ERR_BATCH: return "B must be in 1..8 (1..16 for Q4_K with K % 256 == 0)";
     case QG_ERR_ALIGN: return "misaligned pointer (W 16 B, x 2 B, y 4 B)";
     case QG_ERR_CUDA: return "CUDA runtime error";
     case QG_ERR_NOMEM: return "workspace allocation failed";
@@ -751,16 +766,17 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
 {
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
-    if (B < 1 || B > 8) return QG_ERR_BATCH;
+    if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
     if (N == 0) return QG_OK;
     if (!x || !y) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
         return QG_ERR_ALIGN;
+    const int var = auto_variant(fmt, K, B);
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int var = auto_variant(fmt, K, B);
     if (var == QG_VARIANT_GENERIC) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // no scratch
 
     const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);

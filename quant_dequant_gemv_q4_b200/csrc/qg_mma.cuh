@@ -32,9 +32,18 @@
 
 namespace qg {
 
-// warps per CTA of the tensor-core kernel (shared memory: ring + x fragments + tables)
+// warps per CTA of the tensor-core kernel (shared memory: ring + x fragments + tables; at 16
+// columns, registers)
 template <int BP> struct MmaWarps {
-    static constexpr int value = BP >= 8 ? 12 : 16;
+    static constexpr int value = BP >= 16 ? 8 : BP >= 8 ? 12 : 16;
+};
+// n-tiles of 8 columns per mma (16 columns: two, sharing the unpacked A fragment)
+template <int BP> struct MmaNT {
+    static constexpr int value = BP > 8 ? 2 : 1;
+};
+// floats of a warp's table: D_j [8][32], reused for the epilogue's [32][BP] rows
+template <int BP> struct MmaTab {
+    static constexpr int value = 32 * BP > 256 ? 32 * BP : 256;
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -130,8 +139,9 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
 // float4.
 template <int BP>
 __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
-                                             int US, int j, float *dtab, float (&acc)[2][4],
-                                             float (&accM)[BP], int lane)
+                                             int US, int j, float *dtab,
+                                             float (&acc)[2][MmaNT<BP>::value][4], float (&accM)[BP],
+                                             int lane)
 {
     const int g = lane >> 2, t = lane & 3;
     {
@@ -171,14 +181,19 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
         }
     }
     __syncwarp();
-    const int col = g % BP;
+    // n-tile nt covers columns 8nt .. 8nt+7 (one tile for BP <= 8); lane g supplies column 8nt + g
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        uint2 xb[2][2];
+        uint2 xb[MmaNT<BP>::value][2][2];
 #pragma unroll
-        for (int lh = 0; lh < 2; ++lh)
+        for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) xb[lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = (BP > 8) ? 8 * nt + g : g % BP;
+                    xb[nt][lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
+                }
         const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * g);
         const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * g);
 #pragma unroll
@@ -186,23 +201,35 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
             const uint8_t *rowA = u0 + (tile * 16 + g) * 144 + 16 + 32 * c + 8 * t;
             const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);            // row tile*16 + g
             const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * 144);  // row tile*16 + g + 8
-            float cl[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ch[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float cl[MmaNT<BP>::value][4], ch[MmaNT<BP>::value][4];
+#pragma unroll
+            for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) cl[nt][k] = ch[nt][k] = 0.0f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t wa = h ? wA.y : wA.x, wb = h ? wB.y : wB.x;
                 const uint32_t sa = __umulhi(wa, 1u << 24), sb = __umulhi(wb, 1u << 24);  // >> 8
-                mma_16816(cl, wa & 0x000F000Fu, wb & 0x000F000Fu, sa & 0x000F000Fu,
-                          sb & 0x000F000Fu, xb[0][h].x, xb[0][h].y);
-                mma_16816(ch, wa & 0x00F000F0u, wb & 0x00F000F0u, sa & 0x00F000F0u,
-                          sb & 0x00F000F0u, xb[1][h].x, xb[1][h].y);
+                const uint32_t l0 = wa & 0x000F000Fu, l1 = wb & 0x000F000Fu, l2 = sa & 0x000F000Fu,
+                               l3 = sb & 0x000F000Fu;
+                const uint32_t h0 = wa & 0x00F000F0u, h1 = wb & 0x00F000F0u, h2 = sa & 0x00F000F0u,
+                               h3 = sb & 0x00F000F0u;
+#pragma unroll
+                for (int nt = 0; nt < MmaNT<BP>::value; ++nt) {
+                    mma_16816(cl[nt], l0, l1, l2, l3, xb[nt][0][h].x, xb[nt][0][h].y);
+                    mma_16816(ch[nt], h0, h1, h2, h3, xb[nt][1][h].x, xb[nt][1][h].y);
+                }
             }
             const float la = tile ? Dlo.z : Dlo.x, lb = tile ? Dlo.w : Dlo.y;
             const float ha = tile ? Dhi.z : Dhi.x, hb = tile ? Dhi.w : Dhi.y;
-            acc[tile][0] = fmaf(ha, ch[0], fmaf(la, cl[0], acc[tile][0]));
-            acc[tile][2] = fmaf(hb, ch[2], fmaf(lb, cl[2], acc[tile][2]));
-            if (BP > 1) {
-                acc[tile][1] = fmaf(ha, ch[1], fmaf(la, cl[1], acc[tile][1]));
-                acc[tile][3] = fmaf(hb, ch[3], fmaf(lb, cl[3], acc[tile][3]));
+#pragma unroll
+            for (int nt = 0; nt < MmaNT<BP>::value; ++nt) {
+                acc[tile][nt][0] = fmaf(ha, ch[nt][0], fmaf(la, cl[nt][0], acc[tile][nt][0]));
+                acc[tile][nt][2] = fmaf(hb, ch[nt][2], fmaf(lb, cl[nt][2], acc[tile][nt][2]));
+                if (BP > 1) {
+                    acc[tile][nt][1] = fmaf(ha, ch[nt][1], fmaf(la, cl[nt][1], acc[tile][nt][1]));
+                    acc[tile][nt][3] = fmaf(hb, ch[nt][3], fmaf(lb, cl[nt][3], acc[tile][nt][3]));
+                }
             }
         }
     }
@@ -226,7 +253,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     uint2 *xf = reinterpret_cast<uint2 *>(smem + NW * kRowsStages * BOX);
     float *xsum = reinterpret_cast<float *>(xf + (size_t)a.US * 16 * BP * 4);
     float *tabs = xsum + a.US * 8 * BP;
-    float *red = tabs + NW * 256;
+    float *red = tabs + NW * MmaTab<BP>::value;
     uint64_t *bars = reinterpret_cast<uint64_t *>(red + a.red_floats);
 
     const int s = blockIdx.x / a.Gs;
@@ -238,7 +265,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     const int npairs = bs.G * bs.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;
-    float *dtab = tabs + warp * 256;
+    float *dtab = tabs + warp * MmaTab<BP>::value;
 
     auto pair_units = [&](int q, int &ua, int &ub) {
         const int p = q % bs.P;
@@ -296,7 +323,13 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     for (int q = warp; q < npairs && !failed; q += NW) {
         int ua, ub;
         pair_units(q, ua, ub);
-        float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+        float acc[2][MmaNT<BP>::value][4];
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+            for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[tile][nt][k] = 0.0f;
         float accM[BP];
 #pragma unroll
         for (int b = 0; b < BP; ++b) accM[b] = 0.0f;
@@ -327,10 +360,12 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int col = 2 * t + (i & 1);
-                    if (col < BP) dtab[(tile * 16 + g + 8 * (i >> 1)) * BP + col] = acc[tile][i];
-                }
+                for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int col = 8 * nt + 2 * t + (i & 1);
+                        if (col < BP) dtab[(tile * 16 + g + 8 * (i >> 1)) * BP + col] = acc[tile][nt][i];
+                    }
         }
         __syncwarp();
         float v[BP];

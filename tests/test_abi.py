@@ -112,7 +112,7 @@ FAKE = 0x10000  # a 16-byte-aligned non-null pointer value that is never derefer
     ((FAKE, 12, -1, 256, FAKE, 1, FAKE), qg.QG_ERR_SHAPE),
     ((FAKE, 8, 4, 48, FAKE, 1, FAKE), qg.QG_ERR_SHAPE),
     ((FAKE, 12, 4, 256, FAKE, 0, FAKE), qg.QG_ERR_BATCH),
-    ((FAKE, 12, 4, 256, FAKE, 9, FAKE), qg.QG_ERR_BATCH),
+    ((FAKE, 12, 4, 256, FAKE, 17, FAKE), qg.QG_ERR_BATCH),
     ((0, 12, 4, 256, FAKE, 1, FAKE), qg.QG_ERR_NULL),
     ((FAKE, 12, 4, 256, 0, 1, FAKE), qg.QG_ERR_NULL),
     ((FAKE, 12, 4, 256, FAKE, 1, 0), qg.QG_ERR_NULL),
@@ -165,7 +165,7 @@ def test_gate_up_rejects_bad_arguments(L):
     assert f(None, FAKE, 12, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_NULL
     assert f(FAKE, FAKE + 8, 12, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_ALIGN
     assert f(FAKE, FAKE, 12, 4, 256, FAKE, 0, FAKE, None) == qg.QG_ERR_BATCH
-    assert f(FAKE, FAKE, 12, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, FAKE, 12, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
     assert f(FAKE, FAKE, 12, 4, 256, None, 1, FAKE, None) == qg.QG_ERR_NULL
     assert f(FAKE, FAKE, 12, 4, 256, FAKE, 1, FAKE + 2, None) == qg.QG_ERR_ALIGN
     # the fused path needs whole 256-weight units per row (Q8_0 K = 96 is a valid tensor)
@@ -178,6 +178,17 @@ def test_residual_rejects_bad_arguments(L):
     assert f(FAKE, 5, 4, 256, FAKE, 1, FAKE, FAKE, None) == qg.QG_ERR_FMT
     assert f(FAKE, 12, 4, 256, FAKE, 1, None, FAKE, None) == qg.QG_ERR_NULL
     assert f(FAKE, 12, 4, 256, FAKE, 1, FAKE + 2, FAKE, None) == qg.QG_ERR_ALIGN
-    assert f(FAKE, 12, 4, 256, FAKE, 9, FAKE, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, 12, 4, 256, FAKE, 17, FAKE, FAKE, None) == qg.QG_ERR_BATCH
     assert f(FAKE, 8, 4, 96, FAKE, 1, FAKE, FAKE, None) == qg.QG_ERR_SHAPE
     assert f(None, 12, 0, 256, None, 1, None, None, None) == qg.QG_OK
+
+
+def test_batch_width_limits(L):
+    # 1..8 everywhere; 9..16 only on the tensor-core kernel (Q4_K, K % 256 == 0)
+    assert L.qg_gemv(FAKE, 12, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv(FAKE, 8, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # Q8_0
+    for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC):
+        assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_noalloc(FAKE, 8, 4, 256, FAKE, 16, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 8, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_residual(FAKE, 8, 4, 256, FAKE, 12, FAKE, FAKE, None) == qg.QG_ERR_BATCH

@@ -55,7 +55,7 @@ def assert_h_within(h, ref, what=""):
 
 
 @pytest.mark.parametrize("N,K", [(1, 256), (33, 5120), (300, 768), (129, 2560)])
-@pytest.mark.parametrize("B", [1, 2, 3, 8])
+@pytest.mark.parametrize("B", [1, 2, 3, 8, 16])
 def test_gate_up_q4k_small(dev, orc, N, K, B):
     Wg = synth.q4k_weights(N, K, seed=N + K)
     Wu = synth.q4k_weights(N, K, seed=N + K + 1)

@@ -332,3 +332,45 @@ def test_x_not_16_byte_aligned(dev, orc, B):
         qg.qg_gemv_variant(_t(W, dev), Q4_K, N, K, xd, B, y, None, v)
         torch.cuda.synchronize()
         assert_within(y.cpu().numpy(), yref, A, f"unaligned x v{v}")
+
+
+# ------------------------------------------------------------------------------------------------
+# Verify widths 9..16 (tensor-core kernel only; each weight still read once per call)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("variant", [0, 4])
+@pytest.mark.parametrize("N,K", [(1, 256), (33, 5120), (300, 768), (129, 2560)])
+@pytest.mark.parametrize("B", [9, 12, 16])
+def test_q4k_gemv_wide(dev, orc, variant, N, K, B):
+    W = synth.q4k_weights(N, K, seed=N * 3 + K)
+    x = synth.activations(K, B, seed=B + 90, massive_frac=1e-3)
+    y = gpu_gemv(dev, W, Q4_K, N, K, x, variant)
+    yref, A = orc.gemv(W, Q4_K, N, K, x, B)
+    assert_within(y, yref, A, f"q4k v{variant} N={N} K={K} B={B}")
+
+
+def test_wide_b_rejected_off_the_tensor_kernel(dev):
+    import quant_dequant_gemv_q4_b200 as qg
+    W = synth.q4k_weights(8, 256, seed=1)
+    x = synth.activations(256, 9, seed=1)
+    for v in (1, 2, 3):
+        with pytest.raises(qg.QgError) as e:
+            gpu_gemv(dev, W, Q4_K, 8, 256, x, v)
+        assert e.value.status == qg.QG_ERR_BATCH
+    Wq = synth.q8_0_weights(8, 256, seed=1)
+    with pytest.raises(qg.QgError) as e:
+        gpu_gemv(dev, Wq, Q8_0, 8, 256, x, 0)
+    assert e.value.status == qg.QG_ERR_BATCH
+
+
+def test_verify_width_16_full_size_sampled(dev, orc):
+    """The FFN gate tensor (17408 x 5120) at B = 16: sampled rows, and bitwise repeatable."""
+    N, K, B = 17408, 5120, 16
+    W = synth.q4k_weights(N, K, seed=301)
+    x = synth.activations(K, B, seed=302)
+    y = gpu_gemv(dev, W, Q4_K, N, K, x, 0)
+    rows = _sample_rows(N, np.random.default_rng(4), k=96)
+    yref, A = orc.gemv(W, Q4_K, N, K, x, B, rows=rows)
+    assert_within(y[rows], yref, A, "17408x5120 B=16")
+    y2 = gpu_gemv(dev, W, Q4_K, N, K, x, 0)
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))

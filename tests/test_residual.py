@@ -53,7 +53,7 @@ def run(dev, W, fmt, N, K, x, r, inplace=False):
     return y.cpu().numpy()
 
 
-@pytest.mark.parametrize("fmt,N,K,B", [(Q4_K, 33, 5120, 1), (Q4_K, 300, 768, 3), (Q4_K, 129, 2560, 8),
+@pytest.mark.parametrize("fmt,N,K,B", [(Q4_K, 33, 5120, 1), (Q4_K, 300, 768, 3), (Q4_K, 129, 2560, 8), (Q4_K, 70, 1280, 12),
                                        (Q8_0, 77, 1024, 1), (Q8_0, 200, 2048, 4)])
 @pytest.mark.parametrize("inplace", [False, True])
 def test_residual_small(dev, orc, fmt, N, K, B, inplace):
