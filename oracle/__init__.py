@@ -21,6 +21,8 @@ import numpy as np
 
 Q8_0 = 8  # GGML type id of the Q8_0 block format
 Q4_K = 12  # GGML type id of the Q4_K superblock format
+Q5_K = 13  # GGML type id of the Q5_K superblock format
+Q6_K = 14  # GGML type id of the Q6_K superblock format
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qg_oracle.c")
@@ -61,6 +63,10 @@ def lib():
         L.orc_unpack_q4k.restype = I
         L.orc_unpack_q8_0.argtypes = [P, I64, P, P]
         L.orc_unpack_q8_0.restype = I
+        L.orc_unpack_q5k.argtypes = [P, I64, P, P, P, P, P]
+        L.orc_unpack_q5k.restype = I
+        L.orc_unpack_q6k.argtypes = [P, I64, P, P, P]
+        L.orc_unpack_q6k.restype = I
         _lib = L
     return _lib
 
@@ -159,3 +165,29 @@ def unpack_q8_0(W: np.ndarray, nblk: int) -> dict:
     q = np.empty((nblk, 32), np.int8)
     _check(lib().orc_unpack_q8_0(_ptr(W), nblk, _ptr(d), _ptr(q)), "unpack_q8_0")
     return {"d": d, "q": q}
+
+
+def unpack_q5k(W: np.ndarray, nsb: int) -> dict:
+    """Field view of nsb Q5_K superblocks: d, dmin (fp16 bits), sc, m [nsb, 8], q [nsb, 256] in 0..31."""
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    assert W.size >= nsb * 176
+    d = np.empty(nsb, np.uint16)
+    dmin = np.empty(nsb, np.uint16)
+    sc = np.empty((nsb, 8), np.uint8)
+    m = np.empty((nsb, 8), np.uint8)
+    q = np.empty((nsb, 256), np.uint8)
+    _check(lib().orc_unpack_q5k(_ptr(W), nsb, _ptr(d), _ptr(dmin), _ptr(sc), _ptr(m), _ptr(q)),
+           "unpack_q5k")
+    return {"d": d, "dmin": dmin, "sc": sc, "m": m, "q": q}
+
+
+def unpack_q6k(W: np.ndarray, nsb: int) -> dict:
+    """Field view of nsb Q6_K superblocks: d (fp16 bits), scales [nsb, 16] int8, q [nsb, 256] in
+    -32..31."""
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    assert W.size >= nsb * 210
+    d = np.empty(nsb, np.uint16)
+    scales = np.empty((nsb, 16), np.int8)
+    q = np.empty((nsb, 256), np.int8)
+    _check(lib().orc_unpack_q6k(_ptr(W), nsb, _ptr(d), _ptr(scales), _ptr(q)), "unpack_q6k")
+    return {"d": d, "scales": scales, "q": q}

@@ -40,9 +40,11 @@
 #include <stdlib.h>
 #include <string.h>
 
-/* Format flags: GGML's type ids for the two block formats. */
+/* Format flags: GGML's type ids for the block formats. */
 #define ORC_Q8_0 8
 #define ORC_Q4_K 12
+#define ORC_Q5_K 13
+#define ORC_Q6_K 14
 
 #define ORC_OK 0
 #define ORC_EINVAL 1
@@ -117,6 +119,67 @@ static void orc_dequant_q4k_block(const uint8_t *blk, float *w)
     }
 }
 
+/* Q5_K: the Q4_K superblock with a fifth bit per weight.  176 bytes: fp16 d (0-1), fp16 dmin
+ * (2-3), the Q4_K scale table (4-15), qh[32] (16-47), qs[128] (48-175).  The low four bits of
+ * weight i are its Q4_K nibble in qs; with c = i / 64 and r = i % 64, its fifth bit is bit 2c
+ * (r < 32) or bit 2c + 1 (r >= 32) of qh[r % 32].  w = d * sc_j * q - dmin * m_j, q in 0..31
+ * (d*sc*q has at most 22 significant bits: exact in fp64, rounded once to fp32). */
+static int orc_q5k_quant(const uint8_t *qh, const uint8_t *qs, int i)
+{
+    int c = i / 64;
+    int r = i % 64;
+    int bit = (qh[r % 32] >> (2 * c + (r >= 32 ? 1 : 0))) & 1;
+    return orc_q4k_quant(qs, i) + 16 * bit;
+}
+
+static void orc_dequant_q5k_block(const uint8_t *blk, float *w)
+{
+    double d = orc_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+    double dmin = orc_half_to_double((uint16_t)(blk[2] | (blk[3] << 8)));
+    const uint8_t *scales = blk + 4;
+    const uint8_t *qh = blk + 16;
+    const uint8_t *qs = blk + 48;
+    for (int i = 0; i < 256; ++i) {
+        int sc, m;
+        orc_q4k_scale_min(scales, i / 32, &sc, &m);
+        int q = orc_q5k_quant(qh, qs, i);
+        double exact = d * (double)sc * (double)q - dmin * (double)m;
+        w[i] = (float)exact;
+    }
+}
+
+/* Q6_K: 256 weights in 210 bytes: ql[128] (0-127), qh[64] (128-191), int8 scales[16]
+ * (192-207), fp16 d (208-209).  The superblock is two halves of 128 weights; in half n, with
+ * r = i % 128, k = r / 32 and l = r % 32, weight i takes
+ *   its low four bits from ql[64n + l + 32 (k % 2)]: the low nibble for k < 2, the high for k >= 2,
+ *   its high two bits from bits 2k, 2k+1 of qh[32n + l],
+ * and w = d * scales[i / 16] * (q - 32), q in 0..63 (a signed 6-bit value; the product has up to
+ * 25 significant bits: exact in fp64, rounded once to fp32). */
+static int orc_q6k_quant(const uint8_t *ql, const uint8_t *qh, int i)
+{
+    int n = i / 128;
+    int r = i % 128;
+    int k = r / 32;
+    int l = r % 32;
+    uint8_t lb = ql[64 * n + l + 32 * (k % 2)];
+    int low = (k < 2) ? (lb & 15) : (lb >> 4);
+    int high = (qh[32 * n + l] >> (2 * k)) & 3;
+    return low + 16 * high - 32;
+}
+
+static void orc_dequant_q6k_block(const uint8_t *blk, float *w)
+{
+    const uint8_t *ql = blk;
+    const uint8_t *qh = blk + 128;
+    const int8_t *scales = (const int8_t *)(blk + 192);
+    double d = orc_half_to_double((uint16_t)(blk[208] | (blk[209] << 8)));
+    for (int i = 0; i < 256; ++i) {
+        int q = orc_q6k_quant(ql, qh, i);
+        double exact = d * (double)scales[i / 16] * (double)q;
+        w[i] = (float)exact;
+    }
+}
+
 /* One Q8_0 block (34 bytes) -> 32 fp32 weights, w = d * q. */
 static void orc_dequant_q8_0_block(const uint8_t *blk, float *w)
 {
@@ -135,6 +198,12 @@ static int orc_block_geometry(int fmt, int64_t K, int64_t *block_w, int64_t *blo
     } else if (fmt == ORC_Q8_0) {
         *block_w = 32;
         *block_b = 34;
+    } else if (fmt == ORC_Q5_K) {
+        *block_w = 256;
+        *block_b = 176;
+    } else if (fmt == ORC_Q6_K) {
+        *block_w = 256;
+        *block_b = 210;
     } else {
         return ORC_EINVAL;
     }
@@ -160,6 +229,10 @@ static void orc_dequant_row(int fmt, const uint8_t *W, int64_t n, int64_t K, flo
     for (int64_t t = 0; t < nblk; ++t) {
         if (fmt == ORC_Q4_K)
             orc_dequant_q4k_block(row + t * bb, w + t * bw);
+        else if (fmt == ORC_Q5_K)
+            orc_dequant_q5k_block(row + t * bb, w + t * bw);
+        else if (fmt == ORC_Q6_K)
+            orc_dequant_q6k_block(row + t * bb, w + t * bw);
         else
             orc_dequant_q8_0_block(row + t * bb, w + t * bw);
     }
@@ -255,6 +328,40 @@ int orc_unpack_q8_0(const uint8_t *W, int64_t nblk, uint16_t *d, int8_t *q)
         const uint8_t *blk = W + t * 34;
         d[t] = (uint16_t)(blk[0] | (blk[1] << 8));
         for (int i = 0; i < 32; ++i) q[32 * t + i] = (int8_t)blk[2 + i];
+    }
+    return ORC_OK;
+}
+
+/* Field view of Q5_K superblocks: as orc_unpack_q4k, with q[256s + i] in 0..31. */
+int orc_unpack_q5k(const uint8_t *W, int64_t nsb, uint16_t *d, uint16_t *dmin, uint8_t *sc,
+                   uint8_t *m, uint8_t *q)
+{
+    if (!W || !d || !dmin || !sc || !m || !q || nsb < 0) return ORC_EINVAL;
+    for (int64_t s = 0; s < nsb; ++s) {
+        const uint8_t *blk = W + s * 176;
+        d[s] = (uint16_t)(blk[0] | (blk[1] << 8));
+        dmin[s] = (uint16_t)(blk[2] | (blk[3] << 8));
+        for (int j = 0; j < 8; ++j) {
+            int a, b;
+            orc_q4k_scale_min(blk + 4, j, &a, &b);
+            sc[8 * s + j] = (uint8_t)a;
+            m[8 * s + j] = (uint8_t)b;
+        }
+        for (int i = 0; i < 256; ++i) q[256 * s + i] = (uint8_t)orc_q5k_quant(blk + 16, blk + 48, i);
+    }
+    return ORC_OK;
+}
+
+/* Field view of Q6_K superblocks: d[s] (fp16 bits), scales[16s + t] (int8), q[256s + i] in
+ * -32..31 (the stored 6-bit value minus 32). */
+int orc_unpack_q6k(const uint8_t *W, int64_t nsb, uint16_t *d, int8_t *scales, int8_t *q)
+{
+    if (!W || !d || !scales || !q || nsb < 0) return ORC_EINVAL;
+    for (int64_t s = 0; s < nsb; ++s) {
+        const uint8_t *blk = W + s * 210;
+        d[s] = (uint16_t)(blk[208] | (blk[209] << 8));
+        for (int t = 0; t < 16; ++t) scales[16 * s + t] = (int8_t)blk[192 + t];
+        for (int i = 0; i < 256; ++i) q[256 * s + i] = (int8_t)orc_q6k_quant(blk, blk + 128, i);
     }
     return ORC_OK;
 }

@@ -13,6 +13,13 @@ oracle tests.)
 Q8_0 block bytes (34 per 32 weights): bytes 0-1 = fp16 d ~ U(1e-3, 1e-2), bytes 2-33 = int8 q
 uniform on -127..127 (-128 is never drawn).
 
+Q5_K superblock bytes (176 per 256 weights): d and dmin as for Q4_K (bytes 0-3), bytes 4-175
+uniform random: uniform (sc, m) as for Q4_K, and uniform 5-bit q (qh and qs together hold each
+weight's five bits once).
+
+Q6_K superblock bytes (210 per 256 weights): bytes 0-207 uniform random (uniform 6-bit q, stored
+q - 32 in -32..31, and uniform int8 scales per 16 weights), bytes 208-209 = fp16 d ~ U(1e-5, 2e-4).
+
 Activations: x fp16 [K, B] with entries N(0, 1) drawn in fp64 and rounded once to fp16; for the
 "massive activation" FFN inputs each entry is independently, with probability 1e-3, multiplied by
 100 before that rounding.
@@ -28,9 +35,11 @@ import numpy as np
 
 Q8_0 = 8
 Q4_K = 12
+Q5_K = 13
+Q6_K = 14
 
-BLOCK_WEIGHTS = {Q4_K: 256, Q8_0: 32}
-BLOCK_BYTES = {Q4_K: 144, Q8_0: 34}
+BLOCK_WEIGHTS = {Q4_K: 256, Q8_0: 32, Q5_K: 256, Q6_K: 256}
+BLOCK_BYTES = {Q4_K: 144, Q8_0: 34, Q5_K: 176, Q6_K: 210}
 
 
 def _rng(seed: int, tensor_id: int, purpose: int) -> np.random.Generator:
@@ -69,11 +78,40 @@ def q8_0_weights(N: int, K: int, seed: int, tensor_id: int = 0,
     return blk.reshape(-1)
 
 
+def q5k_weights(N: int, K: int, seed: int, tensor_id: int = 0,
+                d_range=(1e-4, 2e-3), dmin_range=(0.0, 1e-3)) -> np.ndarray:
+    """Random Q5_K tensor [N, K] as raw bytes (uint8, N*K/256*176)."""
+    assert K % 256 == 0
+    g = _rng(seed, tensor_id, 0)
+    nsb = N * (K // 256)
+    blk = g.integers(0, 256, size=(nsb, 176), dtype=np.uint8)
+    d = g.uniform(d_range[0], d_range[1], size=nsb).astype(np.float16)
+    dmin = g.uniform(dmin_range[0], dmin_range[1], size=nsb).astype(np.float16)
+    blk[:, 0:2] = d.view(np.uint8).reshape(nsb, 2)
+    blk[:, 2:4] = dmin.view(np.uint8).reshape(nsb, 2)
+    return blk.reshape(-1)
+
+
+def q6k_weights(N: int, K: int, seed: int, tensor_id: int = 0, d_range=(1e-5, 2e-4)) -> np.ndarray:
+    """Random Q6_K tensor [N, K] as raw bytes (uint8, N*K/256*210)."""
+    assert K % 256 == 0
+    g = _rng(seed, tensor_id, 0)
+    nsb = N * (K // 256)
+    blk = g.integers(0, 256, size=(nsb, 210), dtype=np.uint8)
+    d = g.uniform(d_range[0], d_range[1], size=nsb).astype(np.float16)
+    blk[:, 208:210] = d.view(np.uint8).reshape(nsb, 2)
+    return blk.reshape(-1)
+
+
 def weights(fmt: int, N: int, K: int, seed: int, tensor_id: int = 0) -> np.ndarray:
     if fmt == Q4_K:
         return q4k_weights(N, K, seed, tensor_id)
     if fmt == Q8_0:
         return q8_0_weights(N, K, seed, tensor_id)
+    if fmt == Q5_K:
+        return q5k_weights(N, K, seed, tensor_id)
+    if fmt == Q6_K:
+        return q6k_weights(N, K, seed, tensor_id)
     raise ValueError(f"unknown format {fmt}")
 
 

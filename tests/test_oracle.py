@@ -232,7 +232,7 @@ def test_q8_0_exact_integer_case(orc):
 
 # --- the GEMV as a whole ------------------------------------------------------------------------
 
-@pytest.mark.parametrize("fmt", [Q4_K, Q8_0])
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14])
 @pytest.mark.parametrize("N,K", [(1, 256), (2, 512), (3, 256), (3, 512)])
 def test_brute_force_tiny(orc, fmt, N, K):
     """Oracle y and A equal a numpy fp64 matmul of the dequantized matrix, for B = 1..8."""
@@ -256,7 +256,7 @@ def test_rows_subset_matches_full(orc):
     assert np.array_equal(ys, y[rows]) and np.array_equal(As, A[rows])
 
 
-@pytest.mark.parametrize("fmt", [Q4_K, Q8_0])
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14])
 def test_linearity(orc, fmt):
     """y(2x) = 2 y(x) and y(x/8) = y(x)/8 exactly (power-of-two scalings are exact in fp16 for
     these magnitudes); y(x1) + y(x2) = y(x1 + x2) for x1, x2 with disjoint supports."""
@@ -332,3 +332,107 @@ def test_gate_up_silu_composition(orc):
     # with W_u = W_g, h = silu(g) * g >= 0 wherever g >= 0
     hs, gs, *_ = orc.gate_up_silu(Wg, Wg, Q4_K, N, K, x, B)
     assert np.all(hs[gs >= 0] >= 0)
+
+
+# --- Q5_K and Q6_K (GGML layouts; the T4 dossier's quant mix names them) ------------------------
+
+Q5_K, Q6_K = 13, 14
+
+
+def _q5k_golden_block():
+    g = read_golden("q5k_superblock.txt")
+    blk = np.zeros(176, np.uint8)
+    d, dmin = int(g["d"][0][0], 16), int(g["dmin"][0][0], 16)
+    blk[0:2] = [d & 0xFF, d >> 8]
+    blk[2:4] = [dmin & 0xFF, dmin >> 8]
+    blk[4:16] = _hexbytes(g["scales"][0])
+    blk[16:48] = np.arange(32, dtype=np.uint8)
+    for c in range(4):
+        for l in range(32):
+            blk[48 + 32 * c + l] = (l & 15) | (((l + c) & 15) << 4)
+    return blk, g
+
+
+def _q6k_golden_block():
+    g = read_golden("q6k_superblock.txt")
+    blk = np.zeros(210, np.uint8)
+    blk[0:128] = np.arange(128, dtype=np.uint8)
+    blk[128:192] = 0xE4
+    blk[192:208] = (np.arange(16) - 8).astype(np.int8).view(np.uint8)
+    d = int(g["d"][0][0], 16)
+    blk[208:210] = [d & 0xFF, d >> 8]
+    return blk, g
+
+
+def test_q5k_superblock_golden(orc):
+    blk, g = _q5k_golden_block()
+    w = orc.dequant(blk, Q5_K, 1, 256)[0]
+    for i, v in g["w"]:
+        assert w[int(i)] == np.float32(float(v)), i
+
+
+def test_q6k_superblock_golden(orc):
+    blk, g = _q6k_golden_block()
+    w = orc.dequant(blk, Q6_K, 1, 256)[0]
+    for i, v in g["w"]:
+        assert w[int(i)] == np.float32(float(v)), i
+
+
+def test_q5k_each_fifth_bit_moves_one_weight_by_16_d_sc(orc):
+    """Setting one qh bit raises exactly one weight by 16 * d * sc_j: bit b of qh[l] belongs to
+    weight 64 (b // 2) + 32 (b % 2) + l."""
+    blk, _ = _q5k_golden_block()
+    blk[16:48] = 0
+    base = orc.dequant(blk, Q5_K, 1, 256)[0].astype(np.float64)
+    sc = [1, 2, 3, 4, 26, 43, 60, 13]
+    for l in (0, 7, 31):
+        for b in range(8):
+            blk2 = blk.copy()
+            blk2[16 + l] = 1 << b
+            w = orc.dequant(blk2, Q5_K, 1, 256)[0].astype(np.float64)
+            i = 64 * (b // 2) + 32 * (b % 2) + l
+            diff = w - base
+            assert np.count_nonzero(diff) == 1 and diff[i] == 16 * 1.0 * sc[i // 32], (l, b)
+
+
+def test_q6k_zero_point_and_extremes(orc):
+    """q - 32 spans -32..31: ql = 0 with every high pair = 2 gives q - 32 = 0 (all weights 0);
+    ql = 0xFF, qh = 0xFF gives 31 * d * scale; ql = 0, qh = 0 gives -32 * d * scale."""
+    blk, _ = _q6k_golden_block()
+    blk[0:128] = 0
+    blk[128:192] = 0xAA
+    assert np.all(orc.dequant(blk, Q6_K, 1, 256)[0] == 0.0)
+    scale = (np.arange(16) - 8).repeat(16).astype(np.float64)
+    blk[0:192] = 0xFF
+    assert np.array_equal(orc.dequant(blk, Q6_K, 1, 256)[0], (0.5 * scale * 31).astype(np.float32))
+    blk[0:192] = 0
+    assert np.array_equal(orc.dequant(blk, Q6_K, 1, 256)[0], (0.5 * scale * -32).astype(np.float32))
+
+
+def test_q5k_min_term_closed_form(orc):
+    """All q = 0 (qs and qh zero): y = -dmin * sum_j m_j * X_j."""
+    N, K, B = 3, 512, 2
+    W = synth.q5k_weights(N, K, seed=5).reshape(-1, 176).copy()
+    W[:, 16:176] = 0
+    x = synth.activations(K, B, seed=5)
+    y, _ = orc.gemv(W.reshape(-1), Q5_K, N, K, x, B)
+    f = orc.unpack_q5k(W.reshape(-1), W.shape[0])
+    xd = x.astype(np.float64).reshape(K // 32, 32, B).sum(axis=1)  # X_j per sub-block
+    dmin = np.array([orc.half_to_double(int(v)) for v in f["dmin"]]).repeat(8)
+    m = f["m"].astype(np.float64).reshape(-1)
+    want = np.stack([-(dmin[n * 16:(n + 1) * 16] * m[n * 16:(n + 1) * 16])[:, None] * xd
+                     for n in range(N)]).sum(axis=1)
+    np.testing.assert_allclose(y, want, rtol=1e-14, atol=1e-14)
+
+
+def test_q6k_exact_integer_case(orc):
+    """d = 1, every scale 1: w = q - 32 is an integer in -32..31; with integer x, y is exact."""
+    rng = np.random.default_rng(6)
+    N, K, B = 4, 1024, 3
+    W = synth.q6k_weights(N, K, seed=6).reshape(-1, 210).copy()
+    W[:, 192:208] = 1
+    W[:, 208:210] = np.array([0x00, 0x3C], np.uint8)
+    x = rng.integers(-16, 17, size=(K, B)).astype(np.float16)
+    y, _ = orc.gemv(W.reshape(-1), Q6_K, N, K, x, B)
+    q = orc.unpack_q6k(W.reshape(-1), W.shape[0])["q"].astype(np.int64).reshape(N, K)
+    assert np.array_equal(y, (q @ x.astype(np.int64)).astype(np.float64))
