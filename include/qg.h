@@ -17,11 +17,20 @@
  *                w = d*sc_j*q - dmin*m_j with 6-bit (sc_j, m_j) of sub-block j = i/32 packed in
  *                scales[12] (get_scale_min_k4 layout) and q the 4-bit nibble of weight i:
  *                byte qs[32*(i/64) + i%32], low nibble if i%64 < 32 else high nibble.
+ *   QG_FMT_Q5_K: 256 weights in 176 bytes {fp16 d; fp16 dmin; u8 scales[12]; u8 qh[32];
+ *                u8 qs[128]}: the Q4_K superblock with a fifth bit per weight.  q in 0..31 is the
+ *                Q4_K nibble plus 16 * (bit 2*(i/64) + (i%64 >= 32) of qh[i%32]);
+ *                w = d*sc_j*q - dmin*m_j as Q4_K.
+ *   QG_FMT_Q6_K: 256 weights in 210 bytes {u8 ql[128]; u8 qh[64]; i8 scales[16]; fp16 d}.  In half
+ *                h = i/128, with r = i%128, t = r/32 and l = r%32, the low four bits of q are
+ *                ql[64h + l + 32*(t%2)] (low nibble for t < 2, high nibble for t >= 2), the high two
+ *                bits are bits 2t, 2t+1 of qh[32h + l]; w = d*scales[i/16]*(q - 32), q in 0..63.
+ *                (The T4 dossier's "QUANTIZATION MIX" lists Q5_K and Q6_K next to Q4_K.)
  *   QG_FMT_Q8_0: 32 weights in 34 bytes {fp16 d; i8 qs[32]}, w = d*q.
  *   The flag values are GGML's type ids.
  *
- * Layouts: W row-major, row n = K/256 consecutive superblocks (Q4_K) or K/32 consecutive blocks
- * (Q8_0); x[k*B + b] (fp16 bits); y[n*B + b] (fp32).  A caller holding activations [B][K] passes
+ * Layouts: W row-major, row n = K/256 consecutive superblocks (K-quants) or K/32 consecutive
+ * blocks (Q8_0); x[k*B + b] (fp16 bits); y[n*B + b] (fp32).  A caller holding activations [B][K] passes
  * their transpose.
  *
  * Ownership: every pointer is the caller's; the library never frees caller memory.  The library
@@ -51,7 +60,7 @@ extern "C" {
 #endif
 
 /* Block formats (GGML type ids). */
-enum { QG_FMT_Q8_0 = 8, QG_FMT_Q4_K = 12 };
+enum { QG_FMT_Q8_0 = 8, QG_FMT_Q4_K = 12, QG_FMT_Q5_K = 13, QG_FMT_Q6_K = 14 };
 
 /* Status codes. */
 enum {
@@ -59,11 +68,12 @@ enum {
     QG_ERR_NULL = 1,    /* a required pointer is NULL */
     QG_ERR_FMT = 2,     /* unknown format flag */
     QG_ERR_SHAPE = 3,   /* N < 0, K < 1, or K not a multiple of the block size */
-    QG_ERR_BATCH = 4,   /* B outside 1..8, or outside 1..16 for Q4_K with K % 256 == 0 */
+    QG_ERR_BATCH = 4,   /* B outside 1..8 (1..16 for Q4_K with K % 256 == 0) */
     QG_ERR_ALIGN = 5,   /* W not 16-byte aligned, x not 2-byte aligned or y not 4-byte aligned */
     QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
     QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
-    QG_ERR_RANGE = 8,   /* a packer field is out of range (sc, m > 63; Q4_K q > 15; Q8_0 q = -128) */
+    QG_ERR_RANGE = 8,   /* a packer field is out of range (sc, m > 63; q above 15 / 31 / 63 for
+                           Q4_K / Q5_K / Q6_K; Q8_0 q = -128) */
     QG_ERR_VARIANT = 9, /* unknown kernel variant, or a variant that does not take this format */
     QG_ERR_SCRATCH = 10 /* qg_gemv_noalloc: the call needs more scratch than its fixed array holds */
 };
@@ -74,13 +84,15 @@ enum {
     QG_VARIANT_AUTO = 0,
     /* Each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m) (Q4_K; the
      * dump's value) or w = d*q (Q8_0) and multiplied by x: the error is bounded relative to
-     * sum|w*x| for any input.  Four lanes per 256-weight unit; slower. */
+     * sum|w*x| for any input.  Four lanes per 256-weight unit; slower.  Q4_K and Q8_0 only. */
     QG_VARIANT_DIRECT = 1,
-    /* One lane per row.  Q4_K: the scale and min are applied per 32-weight sub-block,
+    /* One lane per row.  Q4_K and Q5_K: the scale and min are applied per 32-weight sub-block,
      * y = sum_j (d*sc_j)*sum(q*x) - (dmin*m_j)*sum(x), with every q*x product exact; the error is
      * bounded relative to sum(|d*sc*q*x| + |dmin*m*x|), which exceeds sum|w*x| only when
-     * d*sc*q and dmin*m nearly cancel.  Q8_0: the block scale d is applied per 32 weights (error
-     * relative to sum|w*x|).  Requires K % 256 == 0. */
+     * d*sc*q and dmin*m nearly cancel.  Q6_K: per 16-weight group,
+     * y = sum_t (d*sc_t)*(sum(q*x) - 32*sum(x)), the same kind of bound with 32*|d*sc*x| in place
+     * of |dmin*m*x|.  Q8_0: the block scale d is applied per 32 weights (error relative to
+     * sum|w*x|).  Requires K % 256 == 0. */
     QG_VARIANT_FACTORED = 2,
     /* Any format and shape: one warp per row, plain loads, no shared-memory staging.  Used by
      * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0). */
@@ -93,12 +105,12 @@ enum {
 };
 
 /* Bytes of an N x K tensor in format fmt; 0 if fmt is unknown, N < 0, K < 1 or K is not a
- * multiple of the block size (256 for Q4_K, 32 for Q8_0). */
+ * multiple of the block size (256 for the K-quants, 32 for Q8_0). */
 size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
 
 /* y = dequant(W) . x on the device.
  *   W      device, qg_weight_bytes(fmt, N, K) bytes, 16-byte aligned, read only
- *   fmt    QG_FMT_Q4_K or QG_FMT_Q8_0
+ *   fmt    QG_FMT_Q4_K, QG_FMT_Q5_K, QG_FMT_Q6_K or QG_FMT_Q8_0
  *   N, K   rows and reduction length; N >= 0 (N == 0 does nothing); K >= 1, K % block == 0
  *   x      device, fp16 bits [K][B], 2-byte aligned, read only
  *   B      number of columns: 1..8; 1..16 for Q4_K with K % 256 == 0 (9..16 columns run on the
@@ -136,8 +148,8 @@ int qg_gemv_residual(const void *W, int fmt, int64_t N, int64_t K, const uint16_
                      const float *r, float *y, void *stream);
 
 /* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant,
- * for DIRECT / FACTORED / TENSOR when K % 256 != 0, and for TENSOR with Q8_0.  The other variants
- * take both formats. */
+ * for DIRECT / FACTORED / TENSOR when K % 256 != 0, for TENSOR with any format but Q4_K, and for
+ * DIRECT with Q5_K or Q6_K.  FACTORED and GENERIC take every format. */
 int qg_gemv_variant(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
                     float *y, void *stream, int variant);
 
@@ -149,6 +161,9 @@ int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, voi
 /* Host-side bit packer (fields -> GGML bytes); it does not choose scales, it only places bits.
  *   Q4_K: d[N*K/256], dmin[N*K/256] fp16 bits; sc[N*K/32], m[N*K/32] 6-bit values (<= 63);
  *         q = uint8 [N*K] values 0..15, weight order.
+ *   Q5_K: as Q4_K with q = uint8 [N*K] values 0..31.
+ *   Q6_K: d[N*K/256] fp16 bits; sc = the int8 group scales [N*K/16] (two's-complement bytes);
+ *         dmin and m are ignored; q = uint8 [N*K] stored values 0..63 (w = d*sc*(q - 32)).
  *   Q8_0: d[N*K/32] fp16 bits; dmin, sc, m are ignored; q = int8 [N*K] in -127..127.
  *   out   host, qg_weight_bytes(fmt, N, K) bytes.
  * All pointers are host pointers.  QG_ERR_RANGE if a field is out of range (out is then

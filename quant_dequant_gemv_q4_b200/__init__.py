@@ -17,6 +17,8 @@ import numpy as np
 
 QG_FMT_Q8_0 = 8
 QG_FMT_Q4_K = 12
+QG_FMT_Q5_K = 13
+QG_FMT_Q6_K = 14
 
 QG_VARIANT_AUTO = 0
 QG_VARIANT_DIRECT = 1
@@ -167,14 +169,19 @@ def qg_dequant_f32(W, fmt: int, N: int, K: int, out, stream=None) -> None:
 
 
 def qg_pack_reference(fmt: int, N: int, K: int, d, dmin, sc, m, q) -> np.ndarray:
-    """Host bit packer: fields (numpy) -> uint8 tensor bytes."""
+    """Host bit packer: fields (numpy) -> uint8 tensor bytes (Q6_K: sc are the int8 group scales,
+    q the stored values 0..63; dmin, m unused)."""
     out = np.empty(qg_weight_bytes(fmt, N, K), dtype=np.uint8)
     d = np.ascontiguousarray(d, dtype=np.uint16)
     args = [d]
-    if fmt == QG_FMT_Q4_K:
+    if fmt in (QG_FMT_Q4_K, QG_FMT_Q5_K):
         dmin = np.ascontiguousarray(dmin, dtype=np.uint16)
         sc = np.ascontiguousarray(sc, dtype=np.uint8)
         m = np.ascontiguousarray(m, dtype=np.uint8)
+        q = np.ascontiguousarray(q, dtype=np.uint8)
+    elif fmt == QG_FMT_Q6_K:
+        dmin = m = None
+        sc = np.ascontiguousarray(np.asarray(sc).astype(np.int8).view(np.uint8))
         q = np.ascontiguousarray(q, dtype=np.uint8)
     else:
         dmin = sc = m = None

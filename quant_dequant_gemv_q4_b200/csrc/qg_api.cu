@@ -229,15 +229,31 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     RowsPlan best{};
     double best_util = -1.0;
     const int BP = padded_cols(B);
-    const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
-    int NW;
-    if (tensor)
-        NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
-    else if (fmt == kFmtQ4_K)
+    int LB = 0, groups_per_unit = 8, NW = 0;
+    switch (fmt) {
+    case kFmtQ4_K:
+        LB = RowsFmt<kFmtQ4_K>::kLaneBytes;
         NW = BP >= 8 ? RowsWarps<kFmtQ4_K, 8>::value : RowsWarps<kFmtQ4_K, 1>::value;
-    else
+        break;
+    case kFmtQ5_K:
+        LB = RowsFmt<kFmtQ5_K>::kLaneBytes;
+        NW = BP >= 8 ? RowsWarps<kFmtQ5_K, 8>::value : RowsWarps<kFmtQ5_K, 1>::value;
+        break;
+    case kFmtQ6_K:
+        LB = RowsFmt<kFmtQ6_K>::kLaneBytes;
+        groups_per_unit = RowsFmt<kFmtQ6_K>::kGroups;
+        NW = BP >= 4 ? RowsWarps<kFmtQ6_K, 4>::value : RowsWarps<kFmtQ6_K, 1>::value;
+        break;
+    default:
+        LB = RowsFmt<kFmtQ8_0>::kLaneBytes;
         NW = BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
-    const size_t ring = (size_t)NW * kRowsStages * 32 * UB;
+        break;
+    }
+    if (tensor) {
+        LB = RowsFmt<kFmtQ4_K>::kLaneBytes;
+        NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
+    }
+    const size_t ring = (size_t)NW * kRowsStages * 32 * LB;
     const size_t tabs = tensor ? (size_t)NW * std::max(256, 32 * BP) * sizeof(float) : 0;  // per-warp tables
     const size_t bars = (size_t)NW * kRowsStages * 8;
     const int64_t UPR = K / 256;
@@ -255,7 +271,8 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         const int64_t band_rows = (N + Gs - 1) / Gs;
         const int64_t groups = (int64_t)mats * ((band_rows + 31) / 32);
         const int red = (int)((mats == 1 ? NW : std::max<int64_t>(NW, groups)) * 32 * BP);
-        const size_t smem = ring + (size_t)US * (512 + 32) * BP + tabs + (size_t)red * sizeof(float) + bars;
+        const size_t smem = ring + (size_t)US * (512 + 4 * groups_per_unit) * BP + tabs +
+                            (size_t)red * sizeof(float) + bars;
         if (smem + 128 > (size_t)di.smem_optin) continue;
         const double util = ((double)N / (double)Gs) / (32.0 * (double)((N / Gs + 31) / 32 > 0 ? (N / Gs + 31) / 32 : 1));
         RowsPlan p;
@@ -300,6 +317,10 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_ROWS_Q4K2(bp) rows_gemv_kernel<kFmtQ4_K, bp, 2>
 #define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
 #define QG_ROWS_Q802(bp) rows_gemv_kernel<kFmtQ8_0, bp, 2>
+#define QG_ROWS_Q5K1(bp) rows_gemv_kernel<kFmtQ5_K, bp, 1>
+#define QG_ROWS_Q5K2(bp) rows_gemv_kernel<kFmtQ5_K, bp, 2>
+#define QG_ROWS_Q6K1(bp) rows_gemv_kernel<kFmtQ6_K, bp, 1>
+#define QG_ROWS_Q6K2(bp) rows_gemv_kernel<kFmtQ6_K, bp, 2>
     if (tensor) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
         QG_BP_SWITCH16(QG_MMA1)
@@ -308,8 +329,20 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
         if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q802) }
         QG_BP_SWITCH(QG_ROWS_Q801)
     }
+    if (fmt == kFmtQ5_K) {
+        if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q5K2) }
+        QG_BP_SWITCH(QG_ROWS_Q5K1)
+    }
+    if (fmt == kFmtQ6_K) {
+        if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q6K2) }
+        QG_BP_SWITCH(QG_ROWS_Q6K1)
+    }
     if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q4K2) }
     QG_BP_SWITCH(QG_ROWS_Q4K1)
+#undef QG_ROWS_Q6K2
+#undef QG_ROWS_Q6K1
+#undef QG_ROWS_Q5K2
+#undef QG_ROWS_Q5K1
 #undef QG_ROWS_Q802
 #undef QG_ROWS_Q801
 #undef QG_ROWS_Q4K2
@@ -341,7 +374,9 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
 {
     auto enc = tensor_map_encoder();
     if (!enc) return QG_ERR_CUDA;
-    const int UB = (fmt == kFmtQ4_K) ? RowsFmt<kFmtQ4_K>::kUnitBytes : RowsFmt<kFmtQ8_0>::kUnitBytes;
+    const int UB = (fmt == kFmtQ4_K)   ? RowsFmt<kFmtQ4_K>::kUnitBytes
+                   : (fmt == kFmtQ5_K) ? RowsFmt<kFmtQ5_K>::kUnitBytes
+                                       : RowsFmt<kFmtQ8_0>::kUnitBytes;
     const cuuint64_t dims[2] = {(cuuint64_t)(K / 256) * (UB / 4), (cuuint64_t)N};
     const cuuint64_t strides[1] = {(cuuint64_t)(K / 256) * UB};
     const cuuint32_t box[2] = {(cuuint32_t)(UB / 4), 32};
@@ -365,9 +400,18 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     WeightMaps<2> maps;  // the first map alone is the WeightMaps<1> of a single matrix
     static_assert(offsetof(WeightMaps<2>, m) == 0 && sizeof(WeightMaps<1>) == sizeof(CUtensorMap),
                   "WeightMaps<1> is a prefix of WeightMaps<2>");
-    if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
-    if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
+    std::memset(&maps, 0, sizeof(maps));
+    const bool per_lane = (fmt == kFmtQ6_K) && !p.tensor;  // rows not 16-byte multiples: no map
+    if (!per_lane) {
+        if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
+        if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
+    }
     RowsArgs a;
+    const int64_t wbytes = (int64_t)qg_weight_bytes(fmt, N, K);
+    a.w[0] = static_cast<const uint8_t *>(W);
+    a.w[1] = static_cast<const uint8_t *>(W2 ? W2 : W);
+    a.wend = wbytes & ~(int64_t)15;
+    a.wtail = (wbytes & 15) ? 1 : 0;
     a.x = x;
     a.out = (p.S > 1) ? part : y;
     a.y = y;
@@ -399,8 +443,9 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
 
 int check_common(const void *W, int fmt, int64_t N, int64_t K)
 {
-    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_FMT;
-    const int64_t bw = (fmt == QG_FMT_Q4_K) ? 256 : 32;
+    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K && fmt != QG_FMT_Q8_0)
+        return QG_ERR_FMT;
+    const int64_t bw = (fmt == QG_FMT_Q8_0) ? 32 : 256;
     if (N < 0 || K < 1 || K % bw != 0) return QG_ERR_SHAPE;
     if (N > 0 && !W) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(W) % 16 != 0) return QG_ERR_ALIGN;
@@ -413,12 +458,13 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
     const int threads = 256;
     const int64_t warps_needed = N;
     const int64_t blocks = std::min<int64_t>((warps_needed + 7) / 8, (int64_t)di.sms * 8);
-    if (fmt == kFmtQ4_K)
-        rowwise_gemv_kernel<kFmtQ4_K><<<(unsigned)blocks, threads, 0, st>>>(
-            static_cast<const uint8_t *>(W), N, K, x, B, y);
-    else
-        rowwise_gemv_kernel<kFmtQ8_0><<<(unsigned)blocks, threads, 0, st>>>(
-            static_cast<const uint8_t *>(W), N, K, x, B, y);
+    const uint8_t *w = static_cast<const uint8_t *>(W);
+    switch (fmt) {
+    case kFmtQ4_K: rowwise_gemv_kernel<kFmtQ4_K><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
+    case kFmtQ5_K: rowwise_gemv_kernel<kFmtQ5_K><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
+    case kFmtQ6_K: rowwise_gemv_kernel<kFmtQ6_K><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
+    default: rowwise_gemv_kernel<kFmtQ8_0><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
+    }
     return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
@@ -450,6 +496,7 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
     if (var == QG_VARIANT_TENSOR && fmt != QG_FMT_Q4_K) return QG_ERR_VARIANT;
+    if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
     DeviceInfo di;
     int dev = 0;
@@ -637,6 +684,14 @@ int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, voi
         const int64_t threads = nsb * 4;
         dequant_q4k_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
             static_cast<const uint8_t *>(W), nsb, out);
+    } else if (fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K) {
+        const int64_t nsb = N * (K / 256);
+        const int64_t threads = nsb * 16;
+        const unsigned grid = (unsigned)((threads + 255) / 256);
+        if (fmt == QG_FMT_Q5_K)
+            dequant_kq_kernel<kFmtQ5_K><<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(W), nsb, out);
+        else
+            dequant_kq_kernel<kFmtQ6_K><<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(W), nsb, out);
     } else {
         const int64_t nblk = N * (K / 32);
         dequant_q8_0_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(

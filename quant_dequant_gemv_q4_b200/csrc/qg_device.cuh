@@ -33,6 +33,8 @@ namespace qg {
 
 constexpr int kFmtQ8_0 = 8;
 constexpr int kFmtQ4_K = 12;
+constexpr int kFmtQ5_K = 13;
+constexpr int kFmtQ6_K = 14;
 
 constexpr int kVarDirect = 1;
 constexpr int kVarFactored = 2;
@@ -143,6 +145,14 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar), "l"(policy)
         : "memory");
+}
+
+// The same without a cache hint.
+__device__ __forceinline__ void bulk_g2s_plain(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint64_t evict_first_policy()
@@ -735,6 +745,71 @@ __global__ void dequant_q8_0_kernel(const uint8_t *W, int64_t nblk, float *out)
 }
 
 // ------------------------------------------------------------------------------------------------
+// Q5_K and Q6_K, one weight at a time (the dump and the plain per-row kernel).  Byte loads only:
+// Q6_K superblocks (210 B) are 2-byte aligned at best.
+//   Q5_K {fp16 d; fp16 dmin; u8 scales[12]; u8 qh[32]; u8 qs[128]}: q = the Q4_K nibble of qs
+//        plus 16 * bit (2c + (r >= 32)) of qh[r % 32] (c = i / 64, r = i % 64);
+//        w = RN(d*sc_j*q - dmin*m_j), both products exact in fp32 (17 + 5 and 11 + 6 bits).
+//   Q6_K {u8 ql[128]; u8 qh[64]; i8 scales[16]; fp16 d}: in half h = i / 128 with r = i % 128,
+//        t = r / 32, l = r % 32: low nibble of ql[64h + 32(t % 2) + l] (t < 2) or its high nibble
+//        (t >= 2), plus 16 * bits 2t..2t+1 of qh[32h + l]; w = RN(d*sc*(q - 32)), d*sc exact.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ float half_bits_to_float(const uint8_t *p)
+{
+    return __half2float(__ushort_as_half((unsigned short)(p[0] | (p[1] << 8))));
+}
+
+// GGML get_scale_min_k4: (sc_j, m_j) of sub-block j from the 12-byte table
+__device__ __forceinline__ void kq_scale_min(const uint8_t *scales, int j, int &sc, int &m)
+{
+    if (j < 4) {
+        sc = scales[j] & 63;
+        m = scales[j + 4] & 63;
+    } else {
+        sc = (scales[j + 4] & 15) | ((scales[j - 4] >> 6) << 4);
+        m = (scales[j + 4] >> 4) | ((scales[j] >> 6) << 4);
+    }
+}
+
+__device__ __forceinline__ float q5k_weight(const uint8_t *blk, int i)
+{
+    int sc, m;
+    kq_scale_min(blk + 4, i >> 5, sc, m);
+    const int c = i >> 6, r = i & 63;
+    const uint8_t qsb = blk[48 + 32 * c + (r & 31)];
+    const int q = ((r < 32) ? (qsb & 15) : (qsb >> 4)) +
+                  16 * ((blk[16 + (r & 31)] >> (2 * c + (r >> 5))) & 1);
+    const float D = __fmul_rn(half_bits_to_float(blk), (float)sc);
+    const float M = __fmul_rn(half_bits_to_float(blk + 2), (float)m);
+    return __fsub_rn(__fmul_rn(D, (float)q), M);
+}
+
+__device__ __forceinline__ float q6k_weight(const uint8_t *blk, int i)
+{
+    const int h = i >> 7, r = i & 127, t = r >> 5, l = r & 31;
+    const uint8_t lb = blk[64 * h + 32 * (t & 1) + l];
+    const int q = ((t < 2) ? (lb & 15) : (lb >> 4)) + 16 * ((blk[128 + 32 * h + l] >> (2 * t)) & 3);
+    const float D = __fmul_rn(half_bits_to_float(blk + 208), (float)(int8_t)blk[192 + (i >> 4)]);
+    return __fmul_rn(D, (float)(q - 32));
+}
+
+// dump: thread t writes the 16 weights of group t % 16 of superblock t / 16
+template <int FMT>
+__global__ void dequant_kq_kernel(const uint8_t *W, int64_t nsb, float *out)
+{
+    constexpr int SB = (FMT == kFmtQ5_K) ? 176 : 210;
+    const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (t >= nsb * 16) return;
+    const int64_t sb = t >> 4;
+    const int g = (int)(t & 15);
+    const uint8_t *blk = W + sb * SB;
+    float *o = out + sb * 256 + 16 * g;
+#pragma unroll 4
+    for (int e = 0; e < 16; ++e)
+        o[e] = (FMT == kFmtQ5_K) ? q5k_weight(blk, 16 * g + e) : q6k_weight(blk, 16 * g + e);
+}
+
+// ------------------------------------------------------------------------------------------------
 // Plain per-row kernel (any K the format allows; no staging): one warp per row, lanes stride
 // over blocks, correctly rounded weights as in the dump, fp32 partial sums, warp reduction.
 // ------------------------------------------------------------------------------------------------
@@ -773,6 +848,22 @@ __global__ void rowwise_gemv_kernel(const uint8_t *W, int64_t N, int64_t K, cons
                             acc[b] = fmaf(wh[e], xh, acc[b]);
                         }
                     }
+                }
+            }
+        } else if (FMT == kFmtQ5_K || FMT == kFmtQ6_K) {
+            constexpr int SB = (FMT == kFmtQ5_K) ? 176 : 210;
+            const int64_t nsb = K / 256;
+            // lane -> (superblock, 16-weight group)
+            for (int64_t it = lane; it < nsb * 16; it += 32) {
+                const int64_t sb = it >> 4;
+                const int g = (int)(it & 15);
+                const uint8_t *blk = W + (n * nsb + sb) * SB;
+                const int64_t k0 = sb * 256 + 16 * g;
+                for (int e = 0; e < 16; ++e) {
+                    const float wv = (FMT == kFmtQ5_K) ? q5k_weight(blk, 16 * g + e)
+                                                       : q6k_weight(blk, 16 * g + e);
+                    for (int b = 0; b < B; ++b)
+                        acc[b] = fmaf(wv, __half2float(__ushort_as_half(x[(k0 + e) * B + b])), acc[b]);
                 }
             }
         } else {

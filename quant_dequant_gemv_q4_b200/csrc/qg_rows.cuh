@@ -31,17 +31,45 @@
 
 namespace qg {
 
+// Per-format geometry of a step (32 rows x one 256-weight unit):
+//   kUnitBytes  bytes of a unit in W
+//   kLaneBytes  ring bytes per lane (row): the unit itself, or for Q6_K a 16-byte aligned window
+//               around it (see rows_issue_lanes)
+//   kGroups     x-sum groups per unit (sub-blocks of 32 weights; Q6_K: scale groups of 16)
+//   kHiOff      the weights of a byte's high nibble sit kHiOff after those of its low nibble
+//   kPerLane    false: one 2-D tensor copy per step; true: one bulk copy per lane
 template <int FMT> struct RowsFmt;
 template <> struct RowsFmt<kFmtQ4_K> {
-    static constexpr int kUnitBytes = 144;
+    static constexpr int kUnitBytes = 144, kLaneBytes = 144, kGroups = 8, kHiOff = 32;
+    static constexpr bool kPerLane = false;
 };
 template <> struct RowsFmt<kFmtQ8_0> {
-    static constexpr int kUnitBytes = 272;
+    static constexpr int kUnitBytes = 272, kLaneBytes = 272, kGroups = 8, kHiOff = 32;
+    static constexpr bool kPerLane = false;
 };
+template <> struct RowsFmt<kFmtQ5_K> {
+    static constexpr int kUnitBytes = 176, kLaneBytes = 176, kGroups = 8, kHiOff = 32;
+    static constexpr bool kPerLane = false;
+};
+template <> struct RowsFmt<kFmtQ6_K> {
+    static constexpr int kUnitBytes = 210, kLaneBytes = 240, kGroups = 16, kHiOff = 64;
+    static constexpr bool kPerLane = true;
+};
+
+// First of the four weights whose x the staging stores at chunk c, word i of a unit: the weights
+// of the low nibbles of qs word i of chunk c (Q4_K, Q5_K, Q8_0: 64c + 4i; Q6_K, whose chunk
+// c = 2h + p is ql[64h + 32p .. 64h + 32p + 31]: 128h + 32p + 4i).
+template <int FMT>
+__device__ __forceinline__ int rows_x_lo(int c, int i)
+{
+    return (FMT == kFmtQ6_K) ? 128 * (c >> 1) + 32 * (c & 1) + 4 * i : 64 * c + 4 * i;
+}
 
 // warps per CTA: as many as the shared-memory budget allows next to x
 template <int FMT, int BP> struct RowsWarps {
-    static constexpr int value = (FMT == kFmtQ4_K) ? (BP >= 8 ? 12 : 16) : (BP >= 4 ? 6 : 8);
+    static constexpr int value = (FMT == kFmtQ4_K || FMT == kFmtQ5_K) ? (BP >= 8 ? 12 : 16)
+                                 : (FMT == kFmtQ6_K)                  ? (BP >= 4 ? 8 : 12)
+                                                                      : (BP >= 4 ? 6 : 8);
 };
 
 constexpr int kRowsStages = 2;  // ring stages per warp (double buffering)
@@ -61,6 +89,9 @@ struct RowsArgs {
     int red_floats;  // floats of the per-CTA partial-row buffer
     int act;  // gate/up pair (MATS == 2): 1 writes h = silu(gate) * up
     const float *res;  // MATS == 1: y = W x + res (fp32 [N][B], may alias y), or nullptr
+    const uint8_t *w[2];  // per-lane copies (Q6_K): the weight tensors (16-byte aligned)
+    int64_t wend;         // per-lane copies: the tensor's byte size rounded down to 16
+    int wtail;            // per-lane copies: 1 if the byte size is not a multiple of 16
 };
 
 // silu(v) * u, the FFN activation of the gate/up pair (silu(v) = v / (1 + e^-v))
@@ -97,18 +128,21 @@ __device__ __forceinline__ int rows_x_off(int US, int j, int c, int i, int b)
     (void)US;
     return (((j * 4 + c) * 8 + i) * BP + b) * 8;
 }
-// x sums per 32-weight sub-block: xsum[(j * 8 + sub) * BP + b]
-template <int BP>
+// x sums per group (G groups per unit: 32-weight sub-blocks, or Q6_K's 16-weight scale groups):
+// xsum[(j * G + g) * BP + b]
+template <int BP, int G = 8>
 __device__ __forceinline__ int rows_xsum_off(int US, int j, int sub, int b)
 {
     (void)US;
-    return (j * 8 + sub) * BP + b;
+    return (j * G + sub) * BP + b;
 }
 
-template <int BP>
+template <int BP, int FMT = kFmtQ4_K>
 __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s, __half *xs,
                                              float *xsum)
 {
+    constexpr int HI = RowsFmt<FMT>::kHiOff;
+    constexpr int G = RowsFmt<FMT>::kGroups;
     const int US = a.US;
     const int64_t kbase = (int64_t)s * US * 256;
     const uint16_t *xsl = a.x + kbase * a.B;
@@ -124,17 +158,17 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
         const int c = jc & 3, j = jc >> 2;
         uint32_t h[8];  // x[e0 .. e0+3], x[e0+32 .. e0+35] in natural order
         if (j < US_s && b < a.B) {
-            const int e0 = j * 256 + c * 64 + 4 * i;
+            const int e0 = j * 256 + rows_x_lo<FMT>(c, i);
             if (vec) {
                 const uint2 lo = *reinterpret_cast<const uint2 *>(xsl + e0);
-                const uint2 hi = *reinterpret_cast<const uint2 *>(xsl + e0 + 32);
+                const uint2 hi = *reinterpret_cast<const uint2 *>(xsl + e0 + HI);
                 h[0] = lo.x & 0xFFFFu; h[1] = lo.x >> 16; h[2] = lo.y & 0xFFFFu; h[3] = lo.y >> 16;
                 h[4] = hi.x & 0xFFFFu; h[5] = hi.x >> 16; h[6] = hi.y & 0xFFFFu; h[7] = hi.y >> 16;
             } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     h[q] = xsl[(int64_t)(e0 + q) * a.B + b];
-                    h[4 + q] = xsl[(int64_t)(e0 + 32 + q) * a.B + b];
+                    h[4 + q] = xsl[(int64_t)(e0 + HI + q) * a.B + b];
                 }
             }
         } else {
@@ -157,14 +191,30 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
                     __half2float(__ushort_as_half((unsigned short)h[5]))) +
                    (__half2float(__ushort_as_half((unsigned short)h[6])) +
                     __half2float(__ushort_as_half((unsigned short)h[7])));
+        if (G == 8) {
+            // 32-weight sub-blocks 2c (low nibbles) and 2c + 1: all 8 words of the chunk
 #pragma unroll
-        for (int off = 1; off < 8; off <<= 1) {
-            lo += __shfl_xor_sync(0xffffffffu, lo, off);
-            hi += __shfl_xor_sync(0xffffffffu, hi, off);
-        }
-        if (i == 0) {
-            xsum[rows_xsum_off<BP>(US, j, 2 * c, b)] = lo;
-            xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)] = hi;
+            for (int off = 1; off < 8; off <<= 1) {
+                lo += __shfl_xor_sync(0xffffffffu, lo, off);
+                hi += __shfl_xor_sync(0xffffffffu, hi, off);
+            }
+            if (i == 0) {
+                xsum[rows_xsum_off<BP, G>(US, j, 2 * c, b)] = lo;
+                xsum[rows_xsum_off<BP, G>(US, j, 2 * c + 1, b)] = hi;
+            }
+        } else {
+            // Q6_K: 16-weight groups, words 0-3 and 4-7 of the chunk; the low nibbles of chunk
+            // c = 2h + p are group 8h + 2p (+1 for words 4-7), the high nibbles 4 groups later
+#pragma unroll
+            for (int off = 1; off < 4; off <<= 1) {
+                lo += __shfl_xor_sync(0xffffffffu, lo, off);
+                hi += __shfl_xor_sync(0xffffffffu, hi, off);
+            }
+            if ((i & 3) == 0) {
+                const int g = 8 * (c >> 1) + 2 * (c & 1) + (i >> 2);
+                xsum[rows_xsum_off<BP, G>(US, j, g, b)] = lo;
+                xsum[rows_xsum_off<BP, G>(US, j, g + 4, b)] = hi;
+            }
         }
     }
 }
@@ -289,6 +339,166 @@ __device__ __forceinline__ void rows_q8_0(const uint8_t *u, const __half *xs, in
     }
 }
 
+// One Q5_K superblock against x (unit j of the slice).  The Q4_K arithmetic with 5-bit q: per qs
+// word, the low nibbles and the fifth bits of their weights are merged byte-wise into
+// wl = (q & 15) | h << 4 (the qh bit of sub-block 2c is bit 2c of each qh byte, moved to bit 4),
+// the high nibbles likewise into wh; bits 5-7 of each byte are then masked off, so each half of
+// (wl & 0x001F001F) is the fp16 subnormal q * 2^-24 of a whole 5-bit q.
+template <int BP>
+__device__ __forceinline__ void rows_q5k(const uint8_t *u, const __half *xs, const float *xsum,
+                                         int US, int j, float (&v)[BP])
+{
+    const uint4 hdr = *reinterpret_cast<const uint4 *>(u);
+    const uint32_t SC_lo = hdr.y & 0x3F3F3F3Fu;
+    const uint32_t MM_lo = hdr.z & 0x3F3F3F3Fu;
+    const uint32_t SC_hi = (hdr.w & 0x0F0F0F0Fu) | ((hdr.y >> 2) & 0x30303030u);
+    const uint32_t MM_hi = ((hdr.w >> 4) & 0x0F0F0F0Fu) | ((hdr.z >> 2) & 0x30303030u);
+    __half2 dd;
+    *reinterpret_cast<uint32_t *>(&dd) = hdr.x;
+    const float2 dm = __half22float2(dd);  // (d, dmin), exact
+    const float ds = dm.x * 16777216.0f;   // every q*x sum carries 2^-24
+    const uint4 h0 = *reinterpret_cast<const uint4 *>(u + 16);
+    const uint4 h1 = *reinterpret_cast<const uint4 *>(u + 32);
+    const uint32_t hq[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};  // qh bytes 4i..4i+3
+#pragma unroll
+    for (int b = 0; b < BP; ++b) v[b] = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t scw = c < 2 ? SC_lo : SC_hi;
+        const uint32_t mmw = c < 2 ? MM_lo : MM_hi;
+        const uint32_t sel = 0x7650u + 2u * (c & 1);
+        const float2 sc = __fadd2_rn(f2(__uint_as_float(__byte_perm(scw, 0x4B000000u, sel)),
+                                        __uint_as_float(__byte_perm(scw, 0x4B000000u, sel + 1))),
+                                     f2(-8388608.0f, -8388608.0f));
+        const float2 mm = __fadd2_rn(f2(__uint_as_float(__byte_perm(mmw, 0x4B000000u, sel)),
+                                        __uint_as_float(__byte_perm(mmw, 0x4B000000u, sel + 1))),
+                                     f2(-8388608.0f, -8388608.0f));
+        const float2 D = __fmul2_rn(f2(ds, ds), sc);      // scaled d*sc for sub-blocks 2c, 2c+1
+        const float2 M = __fmul2_rn(f2(dm.y, dm.y), mm);  // dmin*m for sub-blocks 2c, 2c+1
+        const uint4 q0 = *reinterpret_cast<const uint4 *>(u + 48 + 32 * c);
+        const uint4 q1 = *reinterpret_cast<const uint4 *>(u + 64 + 32 * c);
+        const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        float l0[BP], l1[BP], h0a[BP], h1a[BP];
+#pragma unroll
+        for (int b = 0; b < BP; ++b) l0[b] = l1[b] = h0a[b] = h1a[b] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t w = qw[i], hw = hq[i];
+            // bit 2c (low nibbles' fifth bit) and bit 2c + 1 (high nibbles') of each byte -> bit 4
+            const uint32_t t1 = (c == 0) ? hw << 4 : (c == 1) ? hw << 2 : (c == 2) ? hw : hw >> 2;
+            const uint32_t t2 = (c == 0) ? hw << 3 : (c == 1) ? hw << 1 : (c == 2) ? hw >> 1 : hw >> 3;
+            const uint32_t wl = (w & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
+            const uint32_t wh = ((w >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
+            const uint32_t qa = wl & 0x001F001Fu, qb = (wl >> 8) & 0x001F001Fu;  // low: e,e+2 / e+1,e+3
+            const uint32_t qc = wh & 0x001F001Fu, qd = (wh >> 8) & 0x001F001Fu;  // high
+#pragma unroll
+            for (int b = 0; b < BP; ++b) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xs + rows_x_off<BP>(US, j, c, i, b));
+                mfma2(l0[b], qa, xv.x);
+                mfma2(l1[b], qb, xv.y);
+                mfma2(h0a[b], qc, xv.z);
+                mfma2(h1a[b], qd, xv.w);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < BP; ++b) {
+            const float Xlo = xsum[rows_xsum_off<BP>(US, j, 2 * c, b)];
+            const float Xhi = xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)];
+            float t = v[b];
+            t = fmaf(D.x, l0[b] + l1[b], t);
+            t = fmaf(D.y, h0a[b] + h1a[b], t);
+            t = fmaf(-M.x, Xlo, t);
+            t = fmaf(-M.y, Xhi, t);
+            v[b] = t;
+        }
+    }
+}
+
+// One Q6_K superblock against x (unit j of the slice), from the lane's ring window: the
+// superblock starts `o` bytes (even, 0..14) into the 16-byte aligned window `win`, so its word k
+// is the funnel shift of window words o/4 + k and o/4 + k + 1 by 8 * (o % 4) bits.  When `tail` is
+// set (the tensor's last superblock, whose window was cut at the tensor's last 16-byte boundary)
+// the scales and d are read from `gblk`, the superblock in global memory.
+// Arithmetic: per 16-weight group t, sum (q - 32) x = sum q x - 32 X_t, q in 0..63 built like
+// Q5_K's: the low nibble of a ql byte and its two qh bits (bits 2p, 2p+1 of the qh byte for the
+// low nibbles of chunk c = 2h + p, bits 2p + 4, 2p + 5 for the high nibbles) merged into one byte.
+template <int BP>
+__device__ __forceinline__ void rows_q6k(const uint32_t *win, int o, bool tail, const uint8_t *gblk,
+                                         const __half *xs, const float *xsum, int US, int j,
+                                         float (&v)[BP])
+{
+    const uint32_t *wp = win + (o >> 2);
+    const uint32_t sh = (o & 2) ? 16u : 0u;
+    auto word = [&](int k) { return __funnelshift_r(wp[k], wp[k + 1], sh); };
+    uint32_t scw[4], dw;
+    if (!tail) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) scw[k] = word(48 + k);
+        dw = word(52);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            scw[k] = (uint32_t)gblk[192 + 4 * k] | ((uint32_t)gblk[193 + 4 * k] << 8) |
+                     ((uint32_t)gblk[194 + 4 * k] << 16) | ((uint32_t)gblk[195 + 4 * k] << 24);
+        dw = (uint32_t)gblk[208] | ((uint32_t)gblk[209] << 8);
+    }
+    const float ds = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu))) * 16777216.0f;
+#pragma unroll
+    for (int b = 0; b < BP; ++b) v[b] = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t hq[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hq[i] = word(32 + 8 * h + i);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int c = 2 * h + p;
+            uint32_t qw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qw[i] = word(16 * h + 8 * p + i);
+#pragma unroll
+            for (int hp = 0; hp < 2; ++hp) {
+                const int tlo = 8 * h + 2 * p + hp, thi = tlo + 4;  // scale groups
+                const float Dlo = ds * (float)(int8_t)(scw[tlo >> 2] >> (8 * (tlo & 3)));
+                const float Dhi = ds * (float)(int8_t)(scw[thi >> 2] >> (8 * (thi & 3)));
+                float l0[BP], l1[BP], h0a[BP], h1a[BP];
+#pragma unroll
+                for (int b = 0; b < BP; ++b) l0[b] = l1[b] = h0a[b] = h1a[b] = 0.0f;
+#pragma unroll
+                for (int i = 4 * hp; i < 4 * hp + 4; ++i) {
+                    const uint32_t w = qw[i], hw = hq[i];
+                    const uint32_t t1 = p ? hw << 2 : hw << 4;  // bits 2p, 2p+1 -> bits 4, 5
+                    const uint32_t t2 = p ? hw >> 2 : hw;       // bits 2p+4, 2p+5 -> bits 4, 5
+                    const uint32_t wl = (w & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
+                    const uint32_t wh = ((w >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
+                    const uint32_t qa = wl & 0x003F003Fu, qb = (wl >> 8) & 0x003F003Fu;
+                    const uint32_t qc = wh & 0x003F003Fu, qd = (wh >> 8) & 0x003F003Fu;
+#pragma unroll
+                    for (int b = 0; b < BP; ++b) {
+                        const uint4 xv =
+                            *reinterpret_cast<const uint4 *>(xs + rows_x_off<BP>(US, j, c, i, b));
+                        mfma2(l0[b], qa, xv.x);
+                        mfma2(l1[b], qb, xv.y);
+                        mfma2(h0a[b], qc, xv.z);
+                        mfma2(h1a[b], qd, xv.w);
+                    }
+                }
+                // d*sc_t * (sum q x - 32 X_t): the q x sums carry 2^-24, so 32 X_t is scaled by
+                // 2^-19 to match
+#pragma unroll
+                for (int b = 0; b < BP; ++b) {
+                    const float Xlo = xsum[rows_xsum_off<BP, 16>(US, j, tlo, b)];
+                    const float Xhi = xsum[rows_xsum_off<BP, 16>(US, j, thi, b)];
+                    float t = v[b];
+                    t = fmaf(Dlo, fmaf(-1.9073486328125e-06f, Xlo, l0[b] + l1[b]), t);
+                    t = fmaf(Dhi, fmaf(-1.9073486328125e-06f, Xhi, h0a[b] + h1a[b]), t);
+                    v[b] = t;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar)
 {
@@ -393,15 +603,18 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
 {
     constexpr int NW = RowsWarps<FMT, BP>::value;
     constexpr int UB = RowsFmt<FMT>::kUnitBytes;
-    constexpr int BOX = 32 * UB;  // bytes of one step: 32 rows x one unit
+    constexpr int LB = RowsFmt<FMT>::kLaneBytes;
+    constexpr bool PER_LANE = RowsFmt<FMT>::kPerLane;
+    constexpr int BOX = 32 * LB;  // ring bytes of one step: 32 rows x one unit
     constexpr int INNER = UB / 4; // u32 elements of one unit
     static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
+    static_assert(LB % 16 == 0, "bulk-copy destinations must be 16-byte aligned");
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     __half *xs = reinterpret_cast<__half *>(smem + NW * kRowsStages * BOX);
     float *xsum = reinterpret_cast<float *>(xs + (size_t)a.US * 256 * BP);
-    float *red = xsum + a.US * 8 * BP;  // [pair][32][BP] partial rows (bands with K parts)
+    float *red = xsum + a.US * RowsFmt<FMT>::kGroups * BP;  // [pair][32][BP] partial rows
     uint64_t *bars = reinterpret_cast<uint64_t *>(red + a.red_floats);
 
     const int s = blockIdx.x / a.Gs;
@@ -439,33 +652,66 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         ig_map = second ? MATS - 1 : 0;
     };
     if (iq < npairs) cursor_pair();
-    auto issue = [&](int i) {
-        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
-        mbar_arrive_expect_tx(bar, BOX);
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
-                    ig_row, bar);
+    auto advance = [&]() {
         if (++iu == iub) {
             iq += NW;
             if (iq < npairs) cursor_pair();
         }
     };
+    // one 2-D tensor copy of the step's 32 rows x one unit (lane 0 alone)
+    auto issue = [&](int i) {
+        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+        mbar_arrive_expect_tx(bar, BOX);
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
+                    ig_row, bar);
+        advance();
+    };
+    // per-lane copies (all 32 lanes): rows whose unit is not 16-byte aligned in W (Q6_K) cannot be
+    // described by a tensor map, so each lane copies the 16-byte aligned window [off & ~15,
+    // (off & ~15) + LB - 16) around its row's unit at byte off; windows never reach past the
+    // tensor's last 16-byte boundary (the last unit of the tensor may come up short: its tail is
+    // read from global memory by the consumer).  Lanes past the last row copy nothing.
+    auto issue_lanes = [&](int i) {
+        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+        const int64_t row = (int64_t)ig_row + lane;
+        uint32_t nb = 0;
+        const uint8_t *src = nullptr;
+        if (row < a.N) {
+            const int64_t ad = ((row * a.UPR + ucol0 + iu) * UB) & ~(int64_t)15;
+            const int64_t room = a.wend - ad;
+            nb = (uint32_t)(room < (LB - 16) ? room : (LB - 16));
+            src = a.w[ig_map] + ad;
+        }
+        const uint32_t tot = __reduce_add_sync(0xffffffffu, nb);
+        if (lane == 0) mbar_arrive_expect_tx(bar, tot);
+        __syncwarp();
+        if (nb) bulk_g2s_plain(smem_u32(myring + (i % kRowsStages) * BOX + lane * LB), src, nb, bar);
+        advance();
+    };
 
     // 1. weight prefetch (independent of the previous kernel on the stream): the first steps
     //    into the ring
     if (nsteps > 0 && lane == 0) {
+        if (!PER_LANE) {
 #pragma unroll
-        for (int m = 0; m < MATS; ++m)
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
+            for (int m = 0; m < MATS; ++m)
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
+        }
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
-        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+        if (!PER_LANE)
+            for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+    }
+    if (PER_LANE && nsteps > 0) {
+        __syncwarp();
+        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue_lanes(i);
     }
     // 2. programmatic dependent launch: let the next kernel start prefetching, then wait for the
     //    previous kernel's results before reading x or writing y
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // 3. x for this slice -> shared memory (fp16 in consumer order) and per-sub-block sums
-    rows_stage_x<BP>(a, s, US_s, xs, xsum);
+    rows_stage_x<BP, FMT>(a, s, US_s, xs, xsum);
     __syncthreads();
 
     int step = 0;
@@ -488,18 +734,36 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
                 failed = true;
                 break;
             }
-            const uint8_t *u = myring + (step % kRowsStages) * BOX + lane * UB;
+            const uint8_t *u = myring + (step % kRowsStages) * BOX + lane * LB;
             float v[BP];
-            if (FMT == kFmtQ4_K)
+            if (FMT == kFmtQ4_K) {
                 rows_q4k<BP>(u, xs, xsum, a.US, j, v);
-            else
+            } else if (FMT == kFmtQ5_K) {
+                rows_q5k<BP>(u, xs, xsum, a.US, j, v);
+            } else if (FMT == kFmtQ6_K) {
+                // this lane's row and unit: where its superblock sits in the window
+                const int g = q / bs.P;
+                const bool second = (MATS > 1) && g >= bs.Gm;
+                const int64_t row = R0 + 32 * (second ? g - bs.Gm : g) + lane;
+                const int64_t m = row * a.UPR + ucol0 + j;  // superblock index in the tensor
+                const int o = (int)((m * UB) & 15);
+                const bool tail = a.wtail && row == a.N - 1 && ucol0 + j == a.UPR - 1;
+                rows_q6k<BP>(reinterpret_cast<const uint32_t *>(u), o, tail,
+                             a.w[second ? MATS - 1 : 0] + m * UB, xs, xsum, a.US, j, v);
+            } else {
                 rows_q8_0<BP>(u, xs, a.US, j, v);
+            }
 #pragma unroll
             for (int b = 0; b < BP; ++b) acc[b] += v[b];
             __syncwarp();
-            if (lane == 0 && step + kRowsStages < nsteps) {
-                fence_proxy_async_smem();
-                issue(step + kRowsStages);
+            if (step + kRowsStages < nsteps) {
+                if (PER_LANE) {
+                    fence_proxy_async_smem();
+                    issue_lanes(step + kRowsStages);
+                } else if (lane == 0) {
+                    fence_proxy_async_smem();
+                    issue(step + kRowsStages);
+                }
             }
         }
         if (bs.P == 1 && MATS == 1) {

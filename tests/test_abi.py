@@ -43,7 +43,8 @@ def test_exports_every_declared_symbol(L):
 def test_weight_bytes(L, orc):
     for fmt, N, K in [(12, 17408, 5120), (12, 5120, 17408), (8, 12288, 5120), (12, 1024, 5120),
                       (8, 3, 96), (12, 0, 256), (12, 1, 300), (8, 1, 33), (7, 1, 256),
-                      (12, -1, 256), (12, 1, 0)]:
+                      (12, -1, 256), (12, 1, 0), (13, 17408, 5120), (14, 5120, 17408),
+                      (13, 3, 768), (14, 3, 768), (13, 1, 300), (14, 1, 32), (14, 0, 256)]:
         assert qg.qg_weight_bytes(fmt, N, K) == max(orc.weight_bytes(fmt, N, K), 0), (fmt, N, K)
 
 
@@ -82,6 +83,54 @@ def test_pack_q8_0_roundtrip(L, orc):
     assert np.array_equal(W, W2)
 
 
+def test_pack_q5k_roundtrips_through_oracle_unpack(L, orc):
+    rng = np.random.default_rng(5)
+    N, K = 3, 768
+    nsb, nsub = N * K // 256, N * K // 32
+    d = rng.integers(0, 65536, nsb, dtype=np.uint16)
+    dmin = rng.integers(0, 65536, nsb, dtype=np.uint16)
+    sc = rng.integers(0, 64, nsub, dtype=np.uint8)
+    m = rng.integers(0, 64, nsub, dtype=np.uint8)
+    q = rng.integers(0, 32, N * K, dtype=np.uint8)
+    W = qg.qg_pack_reference(13, N, K, d, dmin, sc, m, q)
+    f = orc.unpack_q5k(W, nsb)
+    assert np.array_equal(f["d"], d) and np.array_equal(f["dmin"], dmin)
+    assert np.array_equal(f["sc"].reshape(-1), sc) and np.array_equal(f["m"].reshape(-1), m)
+    assert np.array_equal(f["q"].reshape(-1), q)
+
+
+def test_pack_q6k_roundtrips_through_oracle_unpack(L, orc):
+    rng = np.random.default_rng(6)
+    N, K = 3, 768
+    nsb = N * K // 256
+    d = rng.integers(0, 65536, nsb, dtype=np.uint16)
+    sc = rng.integers(-128, 128, N * K // 16).astype(np.int8)
+    q = rng.integers(0, 64, N * K, dtype=np.uint8)
+    W = qg.qg_pack_reference(14, N, K, d, None, sc, None, q)
+    f = orc.unpack_q6k(W, nsb)
+    assert np.array_equal(f["d"], d)
+    assert np.array_equal(f["scales"].reshape(-1), sc)
+    assert np.array_equal(f["q"].reshape(-1).astype(np.int64), q.astype(np.int64) - 32)
+
+
+@pytest.mark.parametrize("fmt", [13, 14])
+def test_pack_kquant_bytes_roundtrip(L, orc, fmt):
+    """Random bytes -> oracle fields -> product packer == the same bytes (every byte of a Q5_K or
+    Q6_K superblock is a field bit)."""
+    N, K = 2, 512
+    W = synth.weights(fmt, N, K, seed=9)
+    nsb = N * K // 256
+    if fmt == 13:
+        f = orc.unpack_q5k(W, nsb)
+        W2 = qg.qg_pack_reference(13, N, K, f["d"], f["dmin"], f["sc"].reshape(-1),
+                                  f["m"].reshape(-1), f["q"].reshape(-1))
+    else:
+        f = orc.unpack_q6k(W, nsb)
+        W2 = qg.qg_pack_reference(14, N, K, f["d"], None, f["scales"].reshape(-1), None,
+                                  (f["q"].reshape(-1).astype(np.int64) + 32).astype(np.uint8))
+    assert np.array_equal(W, W2)
+
+
 def test_pack_range_checks(L):
     N, K = 1, 256
     ok = dict(d=np.zeros(1, np.uint16), dmin=np.zeros(1, np.uint16), sc=np.zeros(8, np.uint8),
@@ -93,6 +142,15 @@ def test_pack_range_checks(L):
         args[key][0] = bad
         with pytest.raises(qg.QgError) as e:
             qg.qg_pack_reference(12, N, K, **args)
+        assert e.value.status == qg.QG_ERR_RANGE
+    for fmt, qmax in [(13, 31), (14, 63)]:
+        q = np.zeros(256, np.uint8)
+        qg.qg_pack_reference(fmt, N, K, ok["d"], ok["dmin"], ok["sc"] if fmt == 13 else
+                             np.zeros(16, np.int8), ok["m"], q)
+        q[7] = qmax + 1
+        with pytest.raises(qg.QgError) as e:
+            qg.qg_pack_reference(fmt, N, K, ok["d"], ok["dmin"], ok["sc"] if fmt == 13 else
+                                 np.zeros(16, np.int8), ok["m"], q)
         assert e.value.status == qg.QG_ERR_RANGE
     q8 = np.zeros(32, np.int8)
     q8[5] = -128
@@ -137,6 +195,12 @@ def test_variant_checks(L):
     assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
     for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_TENSOR):
         assert L.qg_gemv_variant(FAKE, 8, 4, 96, FAKE, 1, FAKE, None, v) == qg.QG_ERR_VARIANT
+    # Q5_K / Q6_K: no four-lanes-per-unit kernel and no tensor-core kernel; 1..8 columns
+    for fmt in (13, 14):
+        for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_TENSOR):
+            assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 1, FAKE, None, v) == qg.QG_ERR_VARIANT
+        assert L.qg_gemv(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+        assert L.qg_gemv(FAKE, fmt, 4, 300, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
 
 
 def test_dequant_rejects_bad_arguments(L):
