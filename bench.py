@@ -499,7 +499,7 @@ def run_ncu_case(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="qg", choices=["qg", "reference"])
     ap.add_argument("--variant", type=int, default=0, help="QG_VARIANT_* (0 = library default)")
@@ -604,7 +604,7 @@ def main(argv=None):
                 n_c = max(args.table_steps, 3 * csc.copies)
                 gbs = c.algorithmic_bytes * n_c / s_c / 1e9
                 per_call[c.name] = {"N": c.N, "K": c.K, "B": c.B,
-                                    "fmt": "Q4_K" if c.fmt == synth.Q4_K else "Q8_0",
+                                    "fmt": synth.FMT_NAMES[c.fmt],
                                     "us": round(s_c * 1e6 / n_c, 3), "gbs": round(gbs, 1),
                                     "frac": round(gbs / hbm, 4),
                                     "splits": qg.qg_last_splits()}

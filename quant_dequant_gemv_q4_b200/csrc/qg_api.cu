@@ -256,6 +256,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     const size_t ring = (size_t)NW * kRowsStages * 32 * LB;
     const size_t tabs = tensor ? (size_t)NW * std::max(256, 32 * BP) * sizeof(float) : 0;  // per-warp tables
     const size_t bars = (size_t)NW * kRowsStages * 8;
+
     const int64_t UPR = K / 256;
     // K slices: the fewest for which x fits in shared memory and the row bands keep at least 85%
     // of their 32-row lanes busy (bands of N*S/SMs rows); otherwise the best such fraction
@@ -271,9 +272,9 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         const int64_t band_rows = (N + Gs - 1) / Gs;
         const int64_t groups = (int64_t)mats * ((band_rows + 31) / 32);
         const int red = (int)((mats == 1 ? NW : std::max<int64_t>(NW, groups)) * 32 * BP);
-        const size_t smem = ring + (size_t)US * (512 + 4 * groups_per_unit) * BP + tabs +
-                            (size_t)red * sizeof(float) + bars;
-        if (smem + 128 > (size_t)di.smem_optin) continue;
+        const size_t xbytes = (size_t)US * (512 + 4 * groups_per_unit) * BP;
+        const size_t smem = ring + xbytes + tabs + (size_t)red * sizeof(float) + bars;
+        if (smem > (size_t)di.smem_optin) continue;  // the kernels have no static shared memory
         const double util = ((double)N / (double)Gs) / (32.0 * (double)((N / Gs + 31) / 32 > 0 ? (N / Gs + 31) / 32 : 1));
         RowsPlan p;
         p.BP = BP;
@@ -383,7 +384,7 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(W), dims, strides,
                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
 }
 
@@ -426,6 +427,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     a.red_floats = p.red_floats;
     a.act = act;
     a.res = res;
+
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.G);
     cfg.blockDim = dim3(p.NW * 32);

@@ -267,16 +267,17 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     const int ucol0 = s * a.US;
     float *dtab = tabs + warp * MmaTab<BP>::value;
 
+    // K part p of a row group takes units p, p + P, ... (as in rows_gemv_kernel)
+    const int du = bs.P;
     auto pair_units = [&](int q, int &ua, int &ub) {
-        const int p = q % bs.P;
-        ua = (p * US_s) / bs.P;
-        ub = ((p + 1) * US_s) / bs.P;
+        ua = q % bs.P;
+        ub = US_s;
     };
     int nsteps = 0;
     for (int q = warp; q < npairs; q += NW) {
         int ua, ub;
         pair_units(q, ua, ub);
-        nsteps += ub - ua;
+        nsteps += (ub - ua + du - 1) / du;
     }
     uint8_t *myring = ring + warp * kRowsStages * BOX;
     const uint32_t bar0 = smem_u32(bars + warp * kRowsStages);
@@ -295,7 +296,8 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
         mbar_arrive_expect_tx(bar, BOX);
         tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
                     ig_row, bar);
-        if (++iu == iub) {
+        iu += du;
+        if (iu >= iub) {
             iq += NW;
             if (iq < npairs) cursor_pair();
         }
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
         float accM[BP];
 #pragma unroll
         for (int b = 0; b < BP; ++b) accM[b] = 0.0f;
-        for (int j = ua; j < ub; ++j, ++step) {
+        for (int j = ua; j < ub; j += du, ++step) {
             const bool ok = mbar_wait_bounded(bar0 + 8 * (step % kRowsStages),
                                               (uint32_t)((step / kRowsStages) & 1));
             if (!__all_sync(0xffffffffu, ok)) {
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     // 4. rows of the band: sum the K parts (and combine the pair) in part order, write once
     if (!any_failed && (bs.P > 1 || MATS > 1)) band_finish<BP, MATS>(a, bs, red, s, R0, rows);
     // 5. K slices: the last CTA of the band adds them up
-    if (a.S > 1) splitk_fixup<MATS>(a, cta, R0, rows);
+    if (a.S > 1) splitk_fixup<MATS>(a, cta, R0, rows, reinterpret_cast<int *>(xsum));
 }
 
 }  // namespace qg

@@ -560,19 +560,22 @@ __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &
 // counter, and the last of the S CTAs to arrive adds the S slices in slice order (so y does not
 // depend on arrival order), writes y and resets the counter for the next call.  Every CTA
 // arrives, also after a copy timeout, so the counters always return to zero.
+// `flag` is one int of shared memory that nothing else uses any more (the kernels pass their x
+// sums, which are dead once the steps are done), so the kernels need no static shared memory.
 template <int MATS>
-__device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_t R0, int rows)
+__device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_t R0, int rows,
+                                             int *flag)
 {
-    __shared__ int s_last;
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned prev = atomicAdd(a.cnt + band, 1u);
-        s_last = (prev == (unsigned)(a.S - 1)) ? 1 : 0;
-        if (s_last) a.cnt[band] = 0u;  // all S arrivals of this call are in
+        const int last = (prev == (unsigned)(a.S - 1)) ? 1 : 0;
+        *flag = last;
+        if (last) a.cnt[band] = 0u;  // all S arrivals of this call are in
     }
     __syncthreads();
-    if (!s_last) return;
+    if (!*flag) return;
     __threadfence();
     const int64_t NB = a.N * a.B;
     for (int t = threadIdx.x; t < rows * a.B; t += blockDim.x) {
@@ -602,6 +605,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     rows_gemv_kernel(const RowsArgs a, const __grid_constant__ WeightMaps<MATS> maps)
 {
     constexpr int NW = RowsWarps<FMT, BP>::value;
+    constexpr int NS = kRowsStages;
     constexpr int UB = RowsFmt<FMT>::kUnitBytes;
     constexpr int LB = RowsFmt<FMT>::kLaneBytes;
     constexpr bool PER_LANE = RowsFmt<FMT>::kPerLane;
@@ -612,7 +616,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
-    __half *xs = reinterpret_cast<__half *>(smem + NW * kRowsStages * BOX);
+    __half *xs = reinterpret_cast<__half *>(smem + NW * NS * BOX);
     float *xsum = reinterpret_cast<float *>(xs + (size_t)a.US * 256 * BP);
     float *red = xsum + a.US * RowsFmt<FMT>::kGroups * BP;  // [pair][32][BP] partial rows
     uint64_t *bars = reinterpret_cast<uint64_t *>(red + a.red_floats);
@@ -627,22 +631,25 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;  // first unit column of this slice
 
-    // this warp's pairs: warp, warp + NW, ...; steps run over the units of each pair in turn
+    // this warp's pairs: warp, warp + NW, ...; steps run over the units of each pair in turn.
+    // K part p of a row group takes the units p, p + P, p + 2P, ... of the slice, so the P warps
+    // of a group stream adjacent units of the same 32 rows at about the same time (measured
+    // faster than contiguous ranges of units per part: DRAM sees longer runs of each row).
+    const int du = bs.P;
     auto pair_units = [&](int q, int &ua, int &ub) {
-        const int p = q % bs.P;
-        ua = (p * US_s) / bs.P;
-        ub = ((p + 1) * US_s) / bs.P;
+        ua = q % bs.P;
+        ub = US_s;
     };
     int nsteps = 0;
     for (int q = warp; q < npairs; q += NW) {
         int ua, ub;
         pair_units(q, ua, ub);
-        nsteps += ub - ua;
+        nsteps += (ub - ua + du - 1) / du;
     }
-    uint8_t *myring = ring + warp * kRowsStages * BOX;
-    const uint32_t bar0 = smem_u32(bars + warp * kRowsStages);
-    // issue cursor (lane 0): pair iq, unit iu
-    int iq = warp, iu = 0, iub = 0;
+    uint8_t *myring = ring + warp * NS * BOX;
+    const uint32_t bar0 = smem_u32(bars + warp * NS);
+    // issue cursor (lane 0): pair iq, unit iu, ring slot islot
+    int iq = warp, iu = 0, iub = 0, islot = 0;
     int ig_row = 0, ig_map = 0;  // the pair's first row in its matrix, and its matrix
     auto cursor_pair = [&]() {
         pair_units(iq, iu, iub);
@@ -653,17 +660,18 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     };
     if (iq < npairs) cursor_pair();
     auto advance = [&]() {
-        if (++iu == iub) {
+        islot = (islot + 1 == NS) ? 0 : islot + 1;
+        iu += du;
+        if (iu >= iub) {
             iq += NW;
             if (iq < npairs) cursor_pair();
         }
     };
     // one 2-D tensor copy of the step's 32 rows x one unit (lane 0 alone)
-    auto issue = [&](int i) {
-        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+    auto issue = [&]() {
+        const uint32_t bar = bar0 + 8 * islot;
         mbar_arrive_expect_tx(bar, BOX);
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
-                    ig_row, bar);
+        tma_load_2d(smem_u32(myring + islot * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER, ig_row, bar);
         advance();
     };
     // per-lane copies (all 32 lanes): rows whose unit is not 16-byte aligned in W (Q6_K) cannot be
@@ -671,8 +679,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     // (off & ~15) + LB - 16) around its row's unit at byte off; windows never reach past the
     // tensor's last 16-byte boundary (the last unit of the tensor may come up short: its tail is
     // read from global memory by the consumer).  Lanes past the last row copy nothing.
-    auto issue_lanes = [&](int i) {
-        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+    auto issue_lanes = [&]() {
+        const uint32_t bar = bar0 + 8 * islot;
         const int64_t row = (int64_t)ig_row + lane;
         uint32_t nb = 0;
         const uint8_t *src = nullptr;
@@ -685,7 +693,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         const uint32_t tot = __reduce_add_sync(0xffffffffu, nb);
         if (lane == 0) mbar_arrive_expect_tx(bar, tot);
         __syncwarp();
-        if (nb) bulk_g2s_plain(smem_u32(myring + (i % kRowsStages) * BOX + lane * LB), src, nb, bar);
+        if (nb) bulk_g2s_plain(smem_u32(myring + islot * BOX + lane * LB), src, nb, bar);
         advance();
     };
 
@@ -697,14 +705,14 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
             for (int m = 0; m < MATS; ++m)
                 asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
         }
-        for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
+        for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         if (!PER_LANE)
-            for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+            for (int i = 0; i < NS && i < nsteps; ++i) issue();
     }
     if (PER_LANE && nsteps > 0) {
         __syncwarp();
-        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue_lanes(i);
+        for (int i = 0; i < NS && i < nsteps; ++i) issue_lanes();
     }
     // 2. programmatic dependent launch: let the next kernel start prefetching, then wait for the
     //    previous kernel's results before reading x or writing y
@@ -714,7 +722,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     rows_stage_x<BP, FMT>(a, s, US_s, xs, xsum);
     __syncthreads();
 
-    int step = 0;
+    int step = 0, cslot = 0;
+    uint32_t cphase = 0;  // consumer: ring slot and its phase parity
     bool failed = false;
     for (int q = warp; q < npairs && !failed; q += NW) {
         int ua, ub;
@@ -722,19 +731,23 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         float acc[BP];
 #pragma unroll
         for (int b = 0; b < BP; ++b) acc[b] = 0.0f;
-        for (int j = ua; j < ub; ++j, ++step) {
-            const bool ok = mbar_wait_bounded(bar0 + 8 * (step % kRowsStages),
-                                              (uint32_t)((step / kRowsStages) & 1));
+        for (int j = ua; j < ub; j += du, ++step) {
+            const bool ok = mbar_wait_bounded(bar0 + 8 * cslot, cphase);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) {
                     atomicExch(a.err, kErrCopyTimeout);
-                    for (int r = step + 1; r < nsteps && r < step + kRowsStages; ++r)
-                        (void)mbar_wait_bounded(bar0 + 8 * (r % kRowsStages), (uint32_t)((r / kRowsStages) & 1));
+                    // wait (bounded) for the copies still in flight before the CTA exits
+                    int r_slot = cslot;
+                    uint32_t r_phase = cphase;
+                    for (int r = step + 1; r < nsteps && r < step + NS; ++r) {
+                        if (++r_slot == NS) { r_slot = 0; r_phase ^= 1u; }
+                        (void)mbar_wait_bounded(bar0 + 8 * r_slot, r_phase);
+                    }
                 }
                 failed = true;
                 break;
             }
-            const uint8_t *u = myring + (step % kRowsStages) * BOX + lane * LB;
+            const uint8_t *u = myring + cslot * BOX + lane * LB;
             float v[BP];
             if (FMT == kFmtQ4_K) {
                 rows_q4k<BP>(u, xs, xsum, a.US, j, v);
@@ -756,15 +769,16 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
 #pragma unroll
             for (int b = 0; b < BP; ++b) acc[b] += v[b];
             __syncwarp();
-            if (step + kRowsStages < nsteps) {
+            if (step + NS < nsteps) {
                 if (PER_LANE) {
                     fence_proxy_async_smem();
-                    issue_lanes(step + kRowsStages);
+                    issue_lanes();
                 } else if (lane == 0) {
                     fence_proxy_async_smem();
-                    issue(step + kRowsStages);
+                    issue();
                 }
             }
+            if (++cslot == NS) { cslot = 0; cphase ^= 1u; }
         }
         if (bs.P == 1 && MATS == 1) {
             // a single K part of a single matrix: the row is complete, write it
@@ -788,7 +802,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     // 4. rows of the band: sum the K parts (and combine the pair) in part order, write once
     if (!any_failed && (bs.P > 1 || MATS > 1)) band_finish<BP, MATS>(a, bs, red, s, R0, rows);
     // 5. K slices: the last CTA of the band adds them up
-    if (a.S > 1) splitk_fixup<MATS>(a, cta, R0, rows);
+    if (a.S > 1) splitk_fixup<MATS>(a, cta, R0, rows, reinterpret_cast<int *>(xsum));
 }
 
 }  // namespace qg

@@ -180,4 +180,15 @@ WORKLOADS = {
     # batched verify of up to 8 draft tokens on the FFN gate
     "q4k_ffn_gate_verify": Workload("q4k_ffn_gate_verify", 4, tuple(
         Gemv(f"ffn_gate_b{b}", Q4_K, 17408, 5120, b, 0) for b in (1, 2, 4, 8))),
+    # the other K-quants of the dossier's quant mix on the same FFN tensors
+    "q5k_ffn_pair_b1": Workload("q5k_ffn_pair_b1", 5, (
+        Gemv("ffn_gate", Q5_K, 17408, 5120, 1, 0, 1e-3),
+        Gemv("ffn_down", Q5_K, 5120, 17408, 1, 1, 1e-3))),
+    "q6k_ffn_pair_b1": Workload("q6k_ffn_pair_b1", 6, (
+        Gemv("ffn_gate", Q6_K, 17408, 5120, 1, 0, 1e-3),
+        Gemv("ffn_down", Q6_K, 5120, 17408, 1, 1, 1e-3))),
+    "kquant_ffn_gate_b8": Workload("kquant_ffn_gate_b8", 7, (
+        Gemv("q5k_ffn_gate_b8", Q5_K, 17408, 5120, 8, 0),
+        Gemv("q6k_ffn_gate_b8", Q6_K, 17408, 5120, 8, 1))),
 }
+FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q6_K: "Q6_K", Q8_0: "Q8_0"}
