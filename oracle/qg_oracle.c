@@ -18,20 +18,24 @@
  *       recurrence ... #3513", Description: the accuracy yardstick is an exact f64 dequantized dot.
  *   GGML's block formats, which the pages name but do not spell out: the Q4_K 6-bit scale/min
  *       packing ("get_scale_min_k4" layout), the Q4_K nibble order, and Q8_0 = {half d; int8 qs[32]}
- *       with w = d*q.
+ *       with w = d*q.  The same dossier's quant mix also lists Q5_K and Q6_K (GGML's K-quants with a
+ *       fifth bit per weight, and with 6-bit weights and 16 int8 group scales); their layouts are
+ *       written out at orc_q5k_quant and orc_q6k_quant below.
  *
  * Definition computed (exact up to the final fp64 summation):
  *   w[n,k]  = the fp32 dequantized weight, computed exactly in fp64 and rounded ONCE to fp32
  *             (round-to-nearest-even).  For Q4_K, d*sc*q and dmin*m have at most 21 and 17
  *             significant bits, and their difference spans at most 50 bits, so the fp64 value is
- *             exact and the single cast is the correctly rounded fp32 weight.  For Q8_0, d*q is
- *             exact in fp32.
+ *             exact and the single cast is the correctly rounded fp32 weight.  Q5_K is the same
+ *             with 5-bit q (d*sc*q at most 22 bits).  Q6_K: d*sc*(q-32) has at most 25 significant
+ *             bits, exact in fp64, rounded once.  For Q8_0, d*q is exact in fp32.
  *   y[n,b]  = sum_k w[n,k] * x[k,b]    in fp64, k ascending (each product is exact in fp64);
  *   A[n,b]  = sum_k |w[n,k] * x[k,b]|  in fp64, the scale of the error bound
  *             |y_gpu - y| <= 1e-5 * A + 1e-6.
  *
- * Layouts: W is row-major, row n is K/256 consecutive 144-byte Q4_K superblocks (or K/32
- * consecutive 34-byte Q8_0 blocks); x is fp16 bits, x[k*B + b]; y and A are y[n*B + b].
+ * Layouts: W is row-major, row n is K/256 consecutive superblocks (144 B Q4_K, 176 B Q5_K,
+ * 210 B Q6_K) or K/32 consecutive 34-byte Q8_0 blocks; x is fp16 bits, x[k*B + b]; y and A are
+ * y[n*B + b].
  *
  * Build with -ffp-contract=off so that no product is fused into a sum.
  */
