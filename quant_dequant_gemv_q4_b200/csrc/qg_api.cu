@@ -250,7 +250,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         break;
     }
     if (tensor) {
-        LB = RowsFmt<kFmtQ4_K>::kLaneBytes;
+        LB = (fmt == kFmtQ5_K) ? MmaFmt<kFmtQ5_K>::kUnitBytes : MmaFmt<kFmtQ4_K>::kUnitBytes;
         NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
     }
     const size_t ring = (size_t)NW * kRowsStages * 32 * LB;
@@ -314,6 +314,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
     }
 #define QG_MMA1(bp) mma_gemv_kernel<bp, 1>
 #define QG_MMA2(bp) mma_gemv_kernel<bp, 2>
+#define QG_MMA5K1(bp) mma_gemv_kernel<bp, 1, kFmtQ5_K>
+#define QG_MMA5K2(bp) mma_gemv_kernel<bp, 2, kFmtQ5_K>
 #define QG_ROWS_Q4K1(bp) rows_gemv_kernel<kFmtQ4_K, bp, 1>
 #define QG_ROWS_Q4K2(bp) rows_gemv_kernel<kFmtQ4_K, bp, 2>
 #define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
@@ -322,6 +324,10 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_ROWS_Q5K2(bp) rows_gemv_kernel<kFmtQ5_K, bp, 2>
 #define QG_ROWS_Q6K1(bp) rows_gemv_kernel<kFmtQ6_K, bp, 1>
 #define QG_ROWS_Q6K2(bp) rows_gemv_kernel<kFmtQ6_K, bp, 2>
+    if (tensor && fmt == kFmtQ5_K) {
+        if (mats == 2) { QG_BP_SWITCH(QG_MMA5K2) }
+        QG_BP_SWITCH(QG_MMA5K1)
+    }
     if (tensor) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
         QG_BP_SWITCH16(QG_MMA1)
@@ -348,6 +354,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #undef QG_ROWS_Q801
 #undef QG_ROWS_Q4K2
 #undef QG_ROWS_Q4K1
+#undef QG_MMA5K2
+#undef QG_MMA5K1
 #undef QG_MMA2
 #undef QG_MMA1
 #undef QG_BP_SWITCH16
@@ -477,7 +485,8 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
 int auto_variant(int fmt, int64_t K, int B)
 {
     if (K % 256 != 0) return QG_VARIANT_GENERIC;
-    return (fmt == QG_FMT_Q4_K && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
+    return ((fmt == QG_FMT_Q4_K || fmt == QG_FMT_Q5_K) && B >= 2) ? QG_VARIANT_TENSOR
+                                                                   : QG_VARIANT_FACTORED;
 }
 
 int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
@@ -497,7 +506,8 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     int var = variant;
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
-    if (var == QG_VARIANT_TENSOR && fmt != QG_FMT_Q4_K) return QG_ERR_VARIANT;
+    if (var == QG_VARIANT_TENSOR && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K) return QG_ERR_VARIANT;
+    if (B > 8 && fmt != QG_FMT_Q4_K) return QG_ERR_BATCH;  // 9..16 columns: the Q4_K kernel only
     if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
     DeviceInfo di;
@@ -595,7 +605,7 @@ int gate_up_impl(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K, 
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;
+    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -627,7 +637,7 @@ int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;
+    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -829,7 +839,7 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
         return QG_ERR_ALIGN;
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;
+    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;

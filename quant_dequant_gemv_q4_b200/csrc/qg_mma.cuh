@@ -37,6 +37,20 @@ namespace qg {
 template <int BP> struct MmaWarps {
     static constexpr int value = BP >= 16 ? 8 : BP >= 8 ? 12 : 16;
 };
+
+// Formats of the tensor-core kernel: Q4_K, and Q5_K (the Q4_K superblock with a fifth-bit plane
+// qh[32] before qs).  kQs: offset of qs in the superblock; kHiScale: the fp16-subnormal scale of
+// the high-nibble half (Q4_K masks the high nibble in place, q * 2^-20; Q5_K shifts it down next
+// to its fifth bit, q * 2^-24).
+template <int FMT> struct MmaFmt;
+template <> struct MmaFmt<kFmtQ4_K> {
+    static constexpr int kUnitBytes = 144, kQs = 16;
+    static constexpr float kHiScale = 1048576.0f;
+};
+template <> struct MmaFmt<kFmtQ5_K> {
+    static constexpr int kUnitBytes = 176, kQs = 48;
+    static constexpr float kHiScale = 16777216.0f;
+};
 // n-tiles of 8 columns per mma (16 columns: two, sharing the unpacked A fragment)
 template <int BP> struct MmaNT {
     static constexpr int value = BP > 8 ? 2 : 1;
@@ -137,17 +151,37 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
 // the min term.  dtab: the warp's [8][32] table of D_j (scaled by 2^24 / 2^20 for the low /
 // high nibble halves), position (row % 8) * 4 + row / 8 so that rows g, g+8, g+16, g+24 are one
 // float4.
-template <int BP>
+// Q5_K: the A registers of one qs word w and its qh word hw (bytes l..l+3 of chunk c): the low
+// nibbles with their fifth bit (bit 2c of each qh byte) and the high nibbles with theirs (bit
+// 2c + 1), each merged into a byte as q = nibble | bit << 4 and read as fp16 subnormal pairs
+// q * 2^-24: lo0 / hi0 = bytes 0 and 2, lo1 / hi1 = bytes 1 and 3.
+template <int C>
+__device__ __forceinline__ void q5k_a_regs(uint32_t w, uint32_t hw, uint32_t &lo0, uint32_t &lo1,
+                                           uint32_t &hi0, uint32_t &hi1)
+{
+    const uint32_t t1 = (C == 0) ? hw << 4 : (C == 1) ? hw << 2 : (C == 2) ? hw : hw >> 2;
+    const uint32_t t2 = (C == 0) ? hw << 3 : (C == 1) ? hw << 1 : (C == 2) ? hw >> 1 : hw >> 3;
+    const uint32_t wl = (w & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
+    const uint32_t wh = ((w >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
+    lo0 = wl & 0x001F001Fu;
+    lo1 = __umulhi(wl, 1u << 24) & 0x001F001Fu;  // >> 8 on the FMA pipe
+    hi0 = wh & 0x001F001Fu;
+    hi1 = __umulhi(wh, 1u << 24) & 0x001F001Fu;
+}
+
+template <int BP, int FMT = kFmtQ4_K>
 __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
                                              int US, int j, float *dtab,
                                              float (&acc)[2][MmaNT<BP>::value][4], float (&accM)[BP],
                                              int lane)
 {
+    constexpr int UB = MmaFmt<FMT>::kUnitBytes;
+    constexpr int QS = MmaFmt<FMT>::kQs;
     const int g = lane >> 2, t = lane & 3;
     {
         // header of row `lane`: the GGML get_scale_min_k4 table decoded with 32-bit masks (byte k
         // of each word = sub-block k or k+4), d and dmin exact in fp32
-        const uint4 hdr = *reinterpret_cast<const uint4 *>(u0 + lane * 144);
+        const uint4 hdr = *reinterpret_cast<const uint4 *>(u0 + lane * UB);
         const uint32_t SC_lo = hdr.y & 0x3F3F3F3Fu;
         const uint32_t MM_lo = hdr.z & 0x3F3F3F3Fu;
         const uint32_t SC_hi = (hdr.w & 0x0F0F0F0Fu) | ((hdr.y >> 2) & 0x30303030u);
@@ -155,7 +189,7 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
         __half2 dd;
         *reinterpret_cast<uint32_t *>(&dd) = hdr.x;
         const float2 dm = __half22float2(dd);
-        const float2 dscale = f2(dm.x * 16777216.0f, dm.x * 1048576.0f);
+        const float2 dscale = f2(dm.x * 16777216.0f, dm.x * MmaFmt<FMT>::kHiScale);
         const int pos = (lane & 7) * 4 + (lane >> 3);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -198,9 +232,15 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
         const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * g);
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile) {
-            const uint8_t *rowA = u0 + (tile * 16 + g) * 144 + 16 + 32 * c + 8 * t;
-            const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);            // row tile*16 + g
-            const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * 144);  // row tile*16 + g + 8
+            const uint8_t *rowA = u0 + (tile * 16 + g) * UB + QS + 32 * c + 8 * t;
+            const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);           // row tile*16 + g
+            const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * UB);  // row tile*16 + g + 8
+            uint2 qhA = make_uint2(0u, 0u), qhB = make_uint2(0u, 0u);  // Q5_K: qh words 2t, 2t+1
+            if (FMT == kFmtQ5_K) {
+                const uint8_t *qhp = u0 + (tile * 16 + g) * UB + 16 + 8 * t;
+                qhA = *reinterpret_cast<const uint2 *>(qhp);
+                qhB = *reinterpret_cast<const uint2 *>(qhp + 8 * UB);
+            }
             float cl[MmaNT<BP>::value][4], ch[MmaNT<BP>::value][4];
 #pragma unroll
             for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
@@ -209,11 +249,20 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t wa = h ? wA.y : wA.x, wb = h ? wB.y : wB.x;
-                const uint32_t sa = __umulhi(wa, 1u << 24), sb = __umulhi(wb, 1u << 24);  // >> 8
-                const uint32_t l0 = wa & 0x000F000Fu, l1 = wb & 0x000F000Fu, l2 = sa & 0x000F000Fu,
-                               l3 = sb & 0x000F000Fu;
-                const uint32_t h0 = wa & 0x00F000F0u, h1 = wb & 0x00F000F0u, h2 = sa & 0x00F000F0u,
-                               h3 = sb & 0x00F000F0u;
+                uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
+                if (FMT == kFmtQ5_K) {
+                    const uint32_t ha = h ? qhA.y : qhA.x, hb = h ? qhB.y : qhB.x;
+                    switch (c) {  // c is a compile-time constant after unrolling
+                    case 0: q5k_a_regs<0>(wa, ha, l0, l2, h0, h2); q5k_a_regs<0>(wb, hb, l1, l3, h1, h3); break;
+                    case 1: q5k_a_regs<1>(wa, ha, l0, l2, h0, h2); q5k_a_regs<1>(wb, hb, l1, l3, h1, h3); break;
+                    case 2: q5k_a_regs<2>(wa, ha, l0, l2, h0, h2); q5k_a_regs<2>(wb, hb, l1, l3, h1, h3); break;
+                    default: q5k_a_regs<3>(wa, ha, l0, l2, h0, h2); q5k_a_regs<3>(wb, hb, l1, l3, h1, h3); break;
+                    }
+                } else {
+                    const uint32_t sa = __umulhi(wa, 1u << 24), sb = __umulhi(wb, 1u << 24);  // >> 8
+                    l0 = wa & 0x000F000Fu; l1 = wb & 0x000F000Fu; l2 = sa & 0x000F000Fu; l3 = sb & 0x000F000Fu;
+                    h0 = wa & 0x00F000F0u; h1 = wb & 0x00F000F0u; h2 = sa & 0x00F000F0u; h3 = sb & 0x00F000F0u;
+                }
 #pragma unroll
                 for (int nt = 0; nt < MmaNT<BP>::value; ++nt) {
                     mma_16816(cl[nt], l0, l1, l2, l3, xb[nt][0][h].x, xb[nt][0][h].y);
@@ -238,12 +287,12 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 // Shared memory of the tensor-core kernel, in order: ring [NW][2][32 x 144 B], x fragments
 // [US][16][BP][4] uint2, x sums [US][8][BP], per-warp tables [NW][256] floats, partial rows
 // [red_floats], mbarriers [NW][2].
-template <int BP, int MATS>
+template <int BP, int MATS, int FMT = kFmtQ4_K>
 __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     mma_gemv_kernel(const RowsArgs a, const __grid_constant__ WeightMaps<MATS> maps)
 {
     constexpr int NW = MmaWarps<BP>::value;
-    constexpr int UB = 144;
+    constexpr int UB = MmaFmt<FMT>::kUnitBytes;
     constexpr int BOX = 32 * UB;
     constexpr int INNER = UB / 4;
     static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
@@ -347,8 +396,8 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
                 failed = true;
                 break;
             }
-            mma_q4k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
-                             lane);
+            mma_q4k_step<BP, FMT>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
+                                  lane);
             __syncwarp();
             if (lane == 0 && step + kRowsStages < nsteps) {
                 fence_proxy_async_smem();

@@ -109,8 +109,8 @@ def test_dump_golden_superblocks(dev):
 SMALL_SHAPES = [(1, 256), (2, 512), (7, 1280), (33, 5120), (300, 768), (129, 2560)]
 
 
-@pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
-@pytest.mark.parametrize("variant", [0, 2, 3])
+@pytest.mark.parametrize("fmt,variant", [(Q5_K, 0), (Q5_K, 2), (Q5_K, 3), (Q5_K, 4),
+                                         (Q6_K, 0), (Q6_K, 2), (Q6_K, 3)])
 @pytest.mark.parametrize("N,K", SMALL_SHAPES)
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8])
 def test_gemv_small(dev, orc, fmt, variant, N, K, B):
@@ -131,6 +131,8 @@ def test_split_k(dev, orc, fmt, N, K, B):
     assert qg.qg_last_splits() > 1
     yref, A = orc.gemv(W, fmt, N, K, x, B)
     assert_within(y, yref, A, "split-K")
+    if fmt == Q5_K and B > 1:  # the CUDA-core kernel on the same split shape
+        assert_within(gpu_gemv(dev, W, fmt, N, K, x, 2), yref, A, "split-K, CUDA cores")
 
 
 def test_q5k_exact_integer_case(dev, orc):
@@ -144,7 +146,7 @@ def test_q5k_exact_integer_case(dev, orc):
     W = W.reshape(-1)
     x = rng.integers(-2, 3, size=(K, B)).astype(np.float16)
     yref, _ = orc.gemv(W, Q5_K, N, K, x, B)
-    for variant in (0, 2, 3):
+    for variant in (0, 2, 3, 4):
         y = gpu_gemv(dev, W, Q5_K, N, K, x, variant)
         assert np.array_equal(y.astype(np.float64), yref), variant
 
@@ -219,6 +221,9 @@ def test_launch_witness(dev):
         x = _t(synth.activations(K, 2, seed=1).view(np.uint16), dev)
         y = torch.empty((N, 2), dtype=torch.float32, device=dev)
         qg.qg_gemv(W, fmt, N, K, x, 2, y)
+        assert qg.qg_last_variant() == (qg.QG_VARIANT_TENSOR if fmt == Q5_K else qg.QG_VARIANT_FACTORED)
+        x1 = _t(synth.activations(K, 1, seed=1).view(np.uint16), dev)
+        qg.qg_gemv(W, fmt, N, K, x1, 1, y)
         assert qg.qg_last_variant() == qg.QG_VARIANT_FACTORED
         qg.qg_gemv_variant(W, fmt, N, K, x, 2, y, None, qg.QG_VARIANT_GENERIC)
         assert qg.qg_last_variant() == qg.QG_VARIANT_GENERIC
