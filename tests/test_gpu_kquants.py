@@ -260,3 +260,70 @@ def test_residual(dev, orc, fmt, N, K, B):
     y = run(dev, W, fmt, N, K, x, r, inplace=True)
     yref, A = orc.gemv(W, fmt, N, K, x, B)
     check(y, yref, A, r, f"fmt={fmt} N={N} K={K} B={B}")
+
+
+# ------------------------------------------------------------------------------------------------
+# Interface behaviour on the new formats
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
+def test_output_guards_untouched(dev, orc, fmt):
+    """y is written exactly in [0, N*B): sentinels on both sides stay intact (every variant)."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    N, K, B = 301, 1280, 3
+    W = synth.weights(fmt, N, K, seed=fmt + 4)
+    x = synth.activations(K, B, seed=4)
+    yref, A = orc.gemv(W, fmt, N, K, x, B)
+    for v in ((0, 2, 3, 4) if fmt == Q5_K else (0, 2, 3)):
+        buf = torch.full((N * B + 128,), 12345.0, dtype=torch.float32, device=dev)
+        y = buf[64:64 + N * B]
+        qg.qg_gemv_variant(_t(W, dev), fmt, N, K, _t(x.view(np.uint16), dev), B, y, None, v)
+        torch.cuda.synchronize()
+        b = buf.cpu().numpy()
+        assert np.all(b[:64] == 12345.0) and np.all(b[64 + N * B:] == 12345.0), v
+        assert_within(b[64:64 + N * B].reshape(N, B), yref, A, f"guarded fmt={fmt} v{v}")
+
+
+@pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_x_not_16_byte_aligned(dev, orc, fmt, B):
+    """x only 2-byte aligned: the staging falls back to element loads; results unchanged."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    N, K = 150, 2560
+    W = synth.weights(fmt, N, K, seed=B + fmt)
+    x = synth.activations(K, B, seed=B)
+    buf = torch.zeros(K * B + 8, dtype=torch.int16, device=dev)
+    buf[1:1 + K * B] = torch.from_numpy(x.view(np.int16).reshape(-1)).to(dev)
+    xd = buf[1:1 + K * B]
+    assert xd.data_ptr() % 16 != 0
+    yref, A = orc.gemv(W, fmt, N, K, x, B)
+    y = torch.empty((N, B), dtype=torch.float32, device=dev)
+    qg.qg_gemv(_t(W, dev), fmt, N, K, xd, B, y)
+    torch.cuda.synchronize()
+    assert_within(y.cpu().numpy(), yref, A, f"unaligned x fmt={fmt} B={B}")
+
+
+@pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
+def test_wide_b_rejected(dev, fmt):
+    import quant_dequant_gemv_q4_b200 as qg
+    W = synth.weights(fmt, 8, 256, seed=1)
+    x = synth.activations(256, 9, seed=1)
+    for v in (0, 2, 3):
+        with pytest.raises(qg.QgError) as e:
+            gpu_gemv(dev, W, fmt, 8, 256, x, v)
+        assert e.value.status == qg.QG_ERR_BATCH
+
+
+def test_q6k_tail_window_every_misalignment(dev, orc):
+    """The tensor's last Q6_K superblock sits at every even offset 0..14 past a 16-byte boundary
+    (N*K/256 mod 8 = 1..8): the cut last copy window and its header read from global memory."""
+    K = 256
+    for N in range(1, 9):  # N superblocks: the last starts at 210 * (N - 1)
+        for B in (1, 2):
+            W = synth.q6k_weights(N, K, seed=N)
+            x = synth.activations(K, B, seed=N)
+            yref, A = orc.gemv(W, Q6_K, N, K, x, B)
+            for v in (0, 3):
+                assert_within(gpu_gemv(dev, W, Q6_K, N, K, x, v), yref, A, f"N={N} B={B} v{v}")

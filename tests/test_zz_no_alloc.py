@@ -17,6 +17,10 @@ CASES = [
     (12, 300, 17408, 8),    # x for the whole K does not fit: split-K partial rows in scratch
     (12, 5120, 17408, 1),   # long-K down projection
     (8, 1000, 5120, 2),     # Q8_0
+    (13, 5120, 17408, 1),   # Q5_K, long K (split-K partial rows)
+    (13, 2000, 5120, 8),    # Q5_K on the tensor-core kernel
+    (14, 17408, 5120, 1),   # Q6_K, per-lane copy windows
+    (14, 300, 17408, 4),    # Q6_K, split K
 ]
 
 
