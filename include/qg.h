@@ -79,7 +79,7 @@ enum {
 };
 
 /* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses: when
- * K % 256 == 0, TENSOR for Q4_K and Q5_K with B >= 2 and FACTORED otherwise; GENERIC when
+ * K % 256 == 0, TENSOR for the K-quants with B >= 2 and FACTORED otherwise; GENERIC when
  * K % 256 != 0. */
 enum {
     QG_VARIANT_AUTO = 0,
@@ -98,10 +98,10 @@ enum {
     /* Any format and shape: one warp per row, plain loads, no shared-memory staging.  Used by
      * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0). */
     QG_VARIANT_GENERIC = 3,
-    /* Q4_K and Q5_K: the FACTORED arithmetic with the q*x products on the tensor cores
-     * (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the instruction are
-     * the B columns of x), so B = 1..8 cost the same (Q4_K: up to 16 columns as two 8-column
-     * tiles).  Same error bound as FACTORED.  Requires K % 256 == 0. */
+    /* The K-quants (Q4_K, Q5_K, Q6_K): the FACTORED arithmetic with the q*x products on the
+     * tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the
+     * instruction are the B columns of x), so B = 1..8 cost the same (Q4_K: up to 16 columns as
+     * two 8-column tiles).  Same error bound as FACTORED.  Requires K % 256 == 0. */
     QG_VARIANT_TENSOR = 4
 };
 
@@ -149,8 +149,8 @@ int qg_gemv_residual(const void *W, int fmt, int64_t N, int64_t K, const uint16_
                      const float *r, float *y, void *stream);
 
 /* qg_gemv with an explicit kernel variant (QG_VARIANT_*); QG_ERR_VARIANT for an unknown variant,
- * for DIRECT / FACTORED / TENSOR when K % 256 != 0, for TENSOR with Q6_K or Q8_0, and for DIRECT
- * with Q5_K or Q6_K.  FACTORED and GENERIC take every format. */
+ * for DIRECT / FACTORED / TENSOR when K % 256 != 0, for TENSOR with Q8_0, and for DIRECT with
+ * Q5_K or Q6_K.  FACTORED and GENERIC take every format. */
 int qg_gemv_variant(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
                     float *y, void *stream, int variant);
 

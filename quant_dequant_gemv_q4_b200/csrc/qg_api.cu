@@ -249,12 +249,20 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         NW = BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
         break;
     }
+    int tab_floats = 0;  // per-warp table of the tensor-core kernel
     if (tensor) {
-        LB = (fmt == kFmtQ5_K) ? MmaFmt<kFmtQ5_K>::kUnitBytes : MmaFmt<kFmtQ4_K>::kUnitBytes;
-        NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
+        if (fmt == kFmtQ6_K) {
+            LB = MmaFmt<kFmtQ6_K>::kUnitBytes;
+            NW = MmaWarpsF<kFmtQ6_K, 1>::value;
+            tab_floats = std::max(512, 32 * BP);
+        } else {
+            LB = (fmt == kFmtQ5_K) ? MmaFmt<kFmtQ5_K>::kUnitBytes : MmaFmt<kFmtQ4_K>::kUnitBytes;
+            NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
+            tab_floats = std::max(256, 32 * BP);
+        }
     }
     const size_t ring = (size_t)NW * kRowsStages * 32 * LB;
-    const size_t tabs = tensor ? (size_t)NW * std::max(256, 32 * BP) * sizeof(float) : 0;  // per-warp tables
+    const size_t tabs = (size_t)NW * tab_floats * sizeof(float);
     const size_t bars = (size_t)NW * kRowsStages * 8;
 
     const int64_t UPR = K / 256;
@@ -316,6 +324,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_MMA2(bp) mma_gemv_kernel<bp, 2>
 #define QG_MMA5K1(bp) mma_gemv_kernel<bp, 1, kFmtQ5_K>
 #define QG_MMA5K2(bp) mma_gemv_kernel<bp, 2, kFmtQ5_K>
+#define QG_MMA6K1(bp) mma_gemv_kernel<bp, 1, kFmtQ6_K>
+#define QG_MMA6K2(bp) mma_gemv_kernel<bp, 2, kFmtQ6_K>
 #define QG_ROWS_Q4K1(bp) rows_gemv_kernel<kFmtQ4_K, bp, 1>
 #define QG_ROWS_Q4K2(bp) rows_gemv_kernel<kFmtQ4_K, bp, 2>
 #define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
@@ -327,6 +337,10 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
     if (tensor && fmt == kFmtQ5_K) {
         if (mats == 2) { QG_BP_SWITCH(QG_MMA5K2) }
         QG_BP_SWITCH(QG_MMA5K1)
+    }
+    if (tensor && fmt == kFmtQ6_K) {
+        if (mats == 2) { QG_BP_SWITCH(QG_MMA6K2) }
+        QG_BP_SWITCH(QG_MMA6K1)
     }
     if (tensor) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
@@ -354,6 +368,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #undef QG_ROWS_Q801
 #undef QG_ROWS_Q4K2
 #undef QG_ROWS_Q4K1
+#undef QG_MMA6K2
+#undef QG_MMA6K1
 #undef QG_MMA5K2
 #undef QG_MMA5K1
 #undef QG_MMA2
@@ -410,7 +426,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     static_assert(offsetof(WeightMaps<2>, m) == 0 && sizeof(WeightMaps<1>) == sizeof(CUtensorMap),
                   "WeightMaps<1> is a prefix of WeightMaps<2>");
     std::memset(&maps, 0, sizeof(maps));
-    const bool per_lane = (fmt == kFmtQ6_K) && !p.tensor;  // rows not 16-byte multiples: no map
+    const bool per_lane = (fmt == kFmtQ6_K);  // rows not 16-byte multiples: no tensor map
     if (!per_lane) {
         if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
         if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
@@ -485,8 +501,7 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
 int auto_variant(int fmt, int64_t K, int B)
 {
     if (K % 256 != 0) return QG_VARIANT_GENERIC;
-    return ((fmt == QG_FMT_Q4_K || fmt == QG_FMT_Q5_K) && B >= 2) ? QG_VARIANT_TENSOR
-                                                                   : QG_VARIANT_FACTORED;
+    return (fmt != QG_FMT_Q8_0 && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
 }
 
 int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
@@ -506,7 +521,7 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     int var = variant;
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
-    if (var == QG_VARIANT_TENSOR && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K) return QG_ERR_VARIANT;
+    if (var == QG_VARIANT_TENSOR && fmt == QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (B > 8 && fmt != QG_FMT_Q4_K) return QG_ERR_BATCH;  // 9..16 columns: the Q4_K kernel only
     if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only

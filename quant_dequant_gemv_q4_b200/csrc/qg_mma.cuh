@@ -51,6 +51,10 @@ template <> struct MmaFmt<kFmtQ5_K> {
     static constexpr int kUnitBytes = 176, kQs = 48;
     static constexpr float kHiScale = 16777216.0f;
 };
+template <> struct MmaFmt<kFmtQ6_K> {  // rows arrive in 240-byte per-lane windows (qg_rows.cuh)
+    static constexpr int kUnitBytes = 240, kQs = 0;
+    static constexpr float kHiScale = 16777216.0f;
+};
 // n-tiles of 8 columns per mma (16 columns: two, sharing the unpacked A fragment)
 template <int BP> struct MmaNT {
     static constexpr int value = BP > 8 ? 2 : 1;
@@ -58,6 +62,14 @@ template <int BP> struct MmaNT {
 // floats of a warp's table: D_j [8][32], reused for the epilogue's [32][BP] rows
 template <int BP> struct MmaTab {
     static constexpr int value = 32 * BP > 256 ? 32 * BP : 256;
+};
+// Q6_K: 16 scale groups per superblock (D_t [16][32]); its per-lane copy windows (240 B a row)
+// leave shared memory for 8 warps
+template <int FMT, int BP> struct MmaTabF {
+    static constexpr int value = (FMT == kFmtQ6_K && MmaTab<BP>::value < 512) ? 512 : MmaTab<BP>::value;
+};
+template <int FMT, int BP> struct MmaWarpsF {
+    static constexpr int value = (FMT == kFmtQ6_K) ? 8 : MmaWarps<BP>::value;
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -90,7 +102,11 @@ __device__ __forceinline__ int mma_xf_swz(int c, int lh, int h, int BP)
 // Thread g stages the 4 consecutive x rows e..e+3 of group g = ((j*4 + c)*2 + lh)*8 + 2t + h
 // (all B columns, one contiguous run of 4*B halves, read with the widest aligned loads), writes
 // their BP fragments, and the 8 groups of one sub-block (8 consecutive lanes) add up its x sums.
-template <int BP>
+// Q6_K keeps the same fragment slots with its own weight order: chunk c = 2hf + p is
+// ql[64hf + 32p ..], k-tile h covers its words 4h .. 4h+3 (one 16-weight scale group), so
+//   e = 256j + 128(c >> 1) + 32(c & 1) + 64lh + 16h + 4t,
+// and the x sums are per 16-weight group 8(c >> 1) + 2(c & 1) + h + 4lh.
+template <int BP, int FMT = kFmtQ4_K>
 __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, uint2 *xf,
                                             float *xsum)
 {
@@ -104,7 +120,9 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
 #pragma unroll
         for (int q = 0; q < 4 * BP; ++q) xv[q] = 0u;
         if (j < US_s) {
-            const int e = j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
+            const int e = (FMT == kFmtQ6_K)
+                              ? j * 256 + 128 * (c >> 1) + 32 * (c & 1) + 64 * lh + 16 * h + 4 * t
+                              : j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
             const uint16_t *src = xsl + (int64_t)e * B;  // 4 * B contiguous halves
             const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
             if (B == BP && (8 * BP) % 16 == 0 && (addr & 15) == 0) {
@@ -133,9 +151,17 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
                          __half2float(__ushort_as_half((unsigned short)xv[1 * BP + col]))) +
                         (__half2float(__ushort_as_half((unsigned short)xv[2 * BP + col])) +
                          __half2float(__ushort_as_half((unsigned short)xv[3 * BP + col])));
+            if (FMT == kFmtQ6_K) {
+                // the 4 lanes t = 0..3 of (c, lh, h) (th = 2t + h): xor over th bits 1 and 2
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                if (t == 0)
+                    xsum[rows_xsum_off<BP, 16>(a.US, j, 8 * (c >> 1) + 2 * (c & 1) + h + 4 * lh, col)] = sum;
+            } else {
 #pragma unroll
-            for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            if (th == 0) xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, col)] = sum;
+                for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                if (th == 0) xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, col)] = sum;
+            }
         }
         const int swz = mma_xf_swz(c, lh, h, BP);
 #pragma unroll
@@ -284,16 +310,135 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
     }
 }
 
+// One Q6_K step: 32 rows x one superblock from the warp's per-lane windows at u0 (window of row
+// r at u0 + 240 r; its superblock starts o_r = (m_r * 210) mod 16 bytes in, m_r its superblock
+// index in the tensor).  Chunk c = 2hf + p is ql[64hf + 32p ..]; its k-tile kk (words 4kk .. 4kk+3)
+// is one 16-weight scale group for the low nibbles (group 8hf + 2p + kk) and one for the high
+// nibbles (4 groups later), so each k-tile's C fragments are scaled by one D_t per row.  A words:
+// thread (g, t) takes ql word 16hf + 8p + 4kk + t and qh word 32 + 8hf + 4kk + t of rows g and
+// g + 8 of the tile; their two high bits (bits 2p, 2p+1 for the low nibbles, 2p+4, 2p+5 for the
+// high ones) are merged byte-wise next to the nibbles and the 6-bit values read as fp16
+// subnormals q * 2^-24.  The -32 offset is applied per group through the x sums:
+// sum (q - 32) x = sum q x - 32 X_t.
+template <int BP>
+__device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
+                                             int US, int j, float *dtab,
+                                             float (&acc)[2][MmaNT<BP>::value][4], float (&accM)[BP],
+                                             int lane, const RowsArgs &a, int64_t row0, int unit,
+                                             const uint8_t *wbase)
+{
+    constexpr int LB = MmaFmt<kFmtQ6_K>::kUnitBytes;
+    const int g = lane >> 2, t = lane & 3;
+    {
+        // header of row `lane`: 16 int8 scales (bytes 192..207) and d (208..209)
+        const int64_t row = row0 + lane;
+        const int64_t m = row * a.UPR + unit;
+        const int o = (int)((m * 210) & 15);
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(u0 + lane * LB) + (o >> 2);
+        const uint32_t sh = (o & 2) ? 16u : 0u;
+        uint32_t scw[4], dw;
+        if (!(a.wtail && row == a.N - 1 && unit == a.UPR - 1)) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) scw[k] = __funnelshift_r(wp[48 + k], wp[49 + k], sh);
+            dw = __funnelshift_r(wp[52], wp[53], sh);
+        } else {
+            // the tensor's last superblock: its copy window stopped at the last 16-byte boundary
+            const uint8_t *gb = wbase + m * 210;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                scw[k] = (uint32_t)gb[192 + 4 * k] | ((uint32_t)gb[193 + 4 * k] << 8) |
+                         ((uint32_t)gb[194 + 4 * k] << 16) | ((uint32_t)gb[195 + 4 * k] << 24);
+            dw = (uint32_t)gb[208] | ((uint32_t)gb[209] << 8);
+        }
+        const float ds = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu))) * 16777216.0f;
+        const int pos = (lane & 7) * 4 + (lane >> 3);
+#pragma unroll
+        for (int tg = 0; tg < 16; ++tg) {
+            const float D = ds * (float)(int8_t)(scw[tg >> 2] >> (8 * (tg & 3)));
+            dtab[tg * 32 + pos] = D;
+            // -32 d sc_t X_t: the q x sums carry 2^-24, so -32 is -2^-19 against D
+#pragma unroll
+            for (int b = 0; b < BP; ++b)
+                accM[b] = fmaf(D * -1.9073486328125e-06f, xsum[rows_xsum_off<BP, 16>(US, j, tg, b)], accM[b]);
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int hf = c >> 1, p = c & 1;
+        uint2 xb[MmaNT<BP>::value][2][2];
+#pragma unroll
+        for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = (BP > 8) ? 8 * nt + g : g % BP;
+                    xb[nt][lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
+                }
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            // the two rows of this thread in the tile, their windows and misalignments
+            const int rA = tile * 16 + g, rB = rA + 8;
+            const int64_t mA = (row0 + rA) * a.UPR + unit, mB = (row0 + rB) * a.UPR + unit;
+            const int oA = (int)((mA * 210) & 15), oB = (int)((mB * 210) & 15);
+            const uint32_t *wa_p = reinterpret_cast<const uint32_t *>(u0 + rA * LB) + (oA >> 2);
+            const uint32_t *wb_p = reinterpret_cast<const uint32_t *>(u0 + rB * LB) + (oB >> 2);
+            const uint32_t sA = (oA & 2) ? 16u : 0u, sB = (oB & 2) ? 16u : 0u;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int ql = 16 * hf + 8 * p + 4 * kk + t, qh = 32 + 8 * hf + 4 * kk + t;
+                const uint32_t wa = __funnelshift_r(wa_p[ql], wa_p[ql + 1], sA);
+                const uint32_t ha = __funnelshift_r(wa_p[qh], wa_p[qh + 1], sA);
+                const uint32_t wb = __funnelshift_r(wb_p[ql], wb_p[ql + 1], sB);
+                const uint32_t hb = __funnelshift_r(wb_p[qh], wb_p[qh + 1], sB);
+                // bits 2p, 2p+1 (low nibbles) and 2p+4, 2p+5 (high nibbles) of each qh byte -> bits 4, 5
+                const uint32_t t1a = p ? ha << 2 : ha << 4, t2a = p ? ha >> 2 : ha;
+                const uint32_t t1b = p ? hb << 2 : hb << 4, t2b = p ? hb >> 2 : hb;
+                const uint32_t wla = (wa & 0x0F0F0F0Fu) | (t1a & 0xF0F0F0F0u);
+                const uint32_t wha = ((wa >> 4) & 0x0F0F0F0Fu) | (t2a & 0xF0F0F0F0u);
+                const uint32_t wlb = (wb & 0x0F0F0F0Fu) | (t1b & 0xF0F0F0F0u);
+                const uint32_t whb = ((wb >> 4) & 0x0F0F0F0Fu) | (t2b & 0xF0F0F0F0u);
+                const uint32_t l0 = wla & 0x003F003Fu, l1 = wlb & 0x003F003Fu;
+                const uint32_t l2 = (wla >> 8) & 0x003F003Fu, l3 = (wlb >> 8) & 0x003F003Fu;
+                const uint32_t h0 = wha & 0x003F003Fu, h1 = whb & 0x003F003Fu;
+                const uint32_t h2 = (wha >> 8) & 0x003F003Fu, h3 = (whb >> 8) & 0x003F003Fu;
+                const int tlo = 8 * hf + 2 * p + kk;
+                const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + tlo * 32 + 4 * g);
+                const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (tlo + 4) * 32 + 4 * g);
+                const float la = tile ? Dlo.z : Dlo.x, lb = tile ? Dlo.w : Dlo.y;
+                const float ha_s = tile ? Dhi.z : Dhi.x, hb_s = tile ? Dhi.w : Dhi.y;
+#pragma unroll
+                for (int nt = 0; nt < MmaNT<BP>::value; ++nt) {
+                    float cl[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ch[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    mma_16816(cl, l0, l1, l2, l3, xb[nt][0][kk].x, xb[nt][0][kk].y);
+                    mma_16816(ch, h0, h1, h2, h3, xb[nt][1][kk].x, xb[nt][1][kk].y);
+                    acc[tile][nt][0] = fmaf(ha_s, ch[0], fmaf(la, cl[0], acc[tile][nt][0]));
+                    acc[tile][nt][2] = fmaf(hb_s, ch[2], fmaf(lb, cl[2], acc[tile][nt][2]));
+                    if (BP > 1) {
+                        acc[tile][nt][1] = fmaf(ha_s, ch[1], fmaf(la, cl[1], acc[tile][nt][1]));
+                        acc[tile][nt][3] = fmaf(hb_s, ch[3], fmaf(lb, cl[3], acc[tile][nt][3]));
+                    }
+                }
+            }
+        }
+    }
+}
+
 // Shared memory of the tensor-core kernel, in order: ring [NW][2][32 x 144 B], x fragments
 // [US][16][BP][4] uint2, x sums [US][8][BP], per-warp tables [NW][256] floats, partial rows
 // [red_floats], mbarriers [NW][2].
 template <int BP, int MATS, int FMT = kFmtQ4_K>
-__global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
+__global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
     mma_gemv_kernel(const RowsArgs a, const __grid_constant__ WeightMaps<MATS> maps)
 {
-    constexpr int NW = MmaWarps<BP>::value;
-    constexpr int UB = MmaFmt<FMT>::kUnitBytes;
-    constexpr int BOX = 32 * UB;
+    constexpr int NW = MmaWarpsF<FMT, BP>::value;
+    constexpr int TAB = MmaTabF<FMT, BP>::value;
+    constexpr bool PER_LANE = (FMT == kFmtQ6_K);    // per-lane copy windows (rows kernel, Q6_K)
+    constexpr int UB = PER_LANE ? 210 : MmaFmt<FMT>::kUnitBytes;  // unit bytes in W
+    constexpr int LB = MmaFmt<FMT>::kUnitBytes;     // ring bytes per row
+    constexpr int GR = PER_LANE ? 16 : 8;           // x-sum groups per unit
+    constexpr int BOX = 32 * LB;
     constexpr int INNER = UB / 4;
     static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
 
@@ -301,8 +446,8 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     uint8_t *ring = smem;
     uint2 *xf = reinterpret_cast<uint2 *>(smem + NW * kRowsStages * BOX);
     float *xsum = reinterpret_cast<float *>(xf + (size_t)a.US * 16 * BP * 4);
-    float *tabs = xsum + a.US * 8 * BP;
-    float *red = tabs + NW * MmaTab<BP>::value;
+    float *tabs = xsum + a.US * GR * BP;
+    float *red = tabs + NW * TAB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(red + a.red_floats);
 
     const int s = blockIdx.x / a.Gs;
@@ -314,7 +459,7 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
     const int npairs = bs.G * bs.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ucol0 = s * a.US;
-    float *dtab = tabs + warp * MmaTab<BP>::value;
+    float *dtab = tabs + warp * TAB;
 
     // K part p of a row group takes units p, p + P, ... (as in rows_gemv_kernel)
     const int du = bs.P;
@@ -340,33 +485,62 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
         ig_map = second ? MATS - 1 : 0;
     };
     if (iq < npairs) cursor_pair();
-    auto issue = [&](int i) {
-        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
-        mbar_arrive_expect_tx(bar, BOX);
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
-                    ig_row, bar);
+    auto advance = [&]() {
         iu += du;
         if (iu >= iub) {
             iq += NW;
             if (iq < npairs) cursor_pair();
         }
     };
+    auto issue = [&](int i) {
+        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+        mbar_arrive_expect_tx(bar, BOX);
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
+                    ig_row, bar);
+        advance();
+    };
+    // Q6_K: per-lane bulk copies of the 16-byte aligned window around each row's unit (all 32
+    // lanes; the same windows as rows_gemv_kernel)
+    auto issue_lanes = [&](int i) {
+        const uint32_t bar = bar0 + 8 * (i % kRowsStages);
+        const int64_t row = (int64_t)ig_row + lane;
+        uint32_t nb = 0;
+        const uint8_t *src = nullptr;
+        if (row < a.N) {
+            const int64_t ad = ((row * a.UPR + ucol0 + iu) * UB) & ~(int64_t)15;
+            const int64_t room = a.wend - ad;
+            nb = (uint32_t)(room < (LB - 16) ? room : (LB - 16));
+            src = a.w[ig_map] + ad;
+        }
+        const uint32_t tot = __reduce_add_sync(0xffffffffu, nb);
+        if (lane == 0) mbar_arrive_expect_tx(bar, tot);
+        __syncwarp();
+        if (nb) bulk_g2s_plain(smem_u32(myring + (i % kRowsStages) * BOX + lane * LB), src, nb, bar);
+        advance();
+    };
 
     // 1. weight prefetch (independent of the previous kernel on the stream)
     if (nsteps > 0 && lane == 0) {
+        if (!PER_LANE) {
 #pragma unroll
-        for (int m = 0; m < MATS; ++m)
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
+            for (int m = 0; m < MATS; ++m)
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
+        }
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
-        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+        if (!PER_LANE)
+            for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+    }
+    if (PER_LANE && nsteps > 0) {
+        __syncwarp();
+        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue_lanes(i);
     }
     // 2. programmatic dependent launch: let the next kernel start prefetching, then wait for the
     //    previous kernel's results before reading x or writing y
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // 3. x fragments and sub-block sums of this slice
-    mma_stage_x<BP>(a, s, US_s, xf, xsum);
+    mma_stage_x<BP, FMT>(a, s, US_s, xf, xsum);
     __syncthreads();
 
     int step = 0;
@@ -396,12 +570,25 @@ __global__ void __launch_bounds__(MmaWarps<BP>::value * 32, 1)
                 failed = true;
                 break;
             }
-            mma_q4k_step<BP, FMT>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
-                                  lane);
+            if (FMT == kFmtQ6_K) {
+                const int gq = q / bs.P;
+                const bool second = (MATS > 1) && gq >= bs.Gm;
+                const int64_t row0 = R0 + 32 * (second ? gq - bs.Gm : gq);
+                mma_q6k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
+                                 lane, a, row0, ucol0 + j, a.w[second ? MATS - 1 : 0]);
+            } else {
+                mma_q4k_step<BP, FMT>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc,
+                                      accM, lane);
+            }
             __syncwarp();
-            if (lane == 0 && step + kRowsStages < nsteps) {
-                fence_proxy_async_smem();
-                issue(step + kRowsStages);
+            if (step + kRowsStages < nsteps) {
+                if (PER_LANE) {
+                    fence_proxy_async_smem();
+                    issue_lanes(step + kRowsStages);
+                } else if (lane == 0) {
+                    fence_proxy_async_smem();
+                    issue(step + kRowsStages);
+                }
             }
         }
         if (failed) break;

@@ -195,9 +195,7 @@ def test_variant_checks(L):
     assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
     for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_TENSOR):
         assert L.qg_gemv_variant(FAKE, 8, 4, 96, FAKE, 1, FAKE, None, v) == qg.QG_ERR_VARIANT
-    # Q5_K / Q6_K: no four-lanes-per-unit kernel; the tensor-core kernel takes Q5_K, not Q6_K;
-    # 1..8 columns
-    assert L.qg_gemv_variant(FAKE, 14, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
+    # Q5_K / Q6_K: no four-lanes-per-unit kernel; 1..8 columns on every kernel
     for fmt in (13, 14):
         assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_DIRECT) == qg.QG_ERR_VARIANT
         assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None, qg.QG_VARIANT_TENSOR) in (

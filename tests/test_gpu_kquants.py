@@ -110,7 +110,7 @@ SMALL_SHAPES = [(1, 256), (2, 512), (7, 1280), (33, 5120), (300, 768), (129, 256
 
 
 @pytest.mark.parametrize("fmt,variant", [(Q5_K, 0), (Q5_K, 2), (Q5_K, 3), (Q5_K, 4),
-                                         (Q6_K, 0), (Q6_K, 2), (Q6_K, 3)])
+                                         (Q6_K, 0), (Q6_K, 2), (Q6_K, 3), (Q6_K, 4)])
 @pytest.mark.parametrize("N,K", SMALL_SHAPES)
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8])
 def test_gemv_small(dev, orc, fmt, variant, N, K, B):
@@ -131,7 +131,7 @@ def test_split_k(dev, orc, fmt, N, K, B):
     assert qg.qg_last_splits() > 1
     yref, A = orc.gemv(W, fmt, N, K, x, B)
     assert_within(y, yref, A, "split-K")
-    if fmt == Q5_K and B > 1:  # the CUDA-core kernel on the same split shape
+    if B > 1:  # the CUDA-core kernel on the same split shape
         assert_within(gpu_gemv(dev, W, fmt, N, K, x, 2), yref, A, "split-K, CUDA cores")
 
 
@@ -161,7 +161,7 @@ def test_q6k_exact_integer_case(dev, orc):
     W = W.reshape(-1)
     x = rng.integers(-2, 3, size=(K, B)).astype(np.float16)
     yref, _ = orc.gemv(W, Q6_K, N, K, x, B)
-    for variant in (0, 2, 3):
+    for variant in (0, 2, 3, 4):
         y = gpu_gemv(dev, W, Q6_K, N, K, x, variant)
         assert np.array_equal(y.astype(np.float64), yref), variant
 
@@ -186,6 +186,7 @@ def test_q6k_near_zero_weights(dev, orc):
     s = np.abs(np.repeat(sc.astype(np.float64), 16)) * 2.0 ** -7
     Af = (s * (q.astype(np.float64) + 32.0)).reshape(N, K) @ np.abs(x.astype(np.float64))
     assert_within(gpu_gemv(dev, W, Q6_K, N, K, x, 2), yref, Af, "factored, near-zero")
+    assert_within(gpu_gemv(dev, W, Q6_K, N, K, x, 4), yref, Af, "tensor cores, near-zero")
 
 
 # ------------------------------------------------------------------------------------------------
@@ -221,7 +222,7 @@ def test_launch_witness(dev):
         x = _t(synth.activations(K, 2, seed=1).view(np.uint16), dev)
         y = torch.empty((N, 2), dtype=torch.float32, device=dev)
         qg.qg_gemv(W, fmt, N, K, x, 2, y)
-        assert qg.qg_last_variant() == (qg.QG_VARIANT_TENSOR if fmt == Q5_K else qg.QG_VARIANT_FACTORED)
+        assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
         x1 = _t(synth.activations(K, 1, seed=1).view(np.uint16), dev)
         qg.qg_gemv(W, fmt, N, K, x1, 1, y)
         assert qg.qg_last_variant() == qg.QG_VARIANT_FACTORED
@@ -275,7 +276,7 @@ def test_output_guards_untouched(dev, orc, fmt):
     W = synth.weights(fmt, N, K, seed=fmt + 4)
     x = synth.activations(K, B, seed=4)
     yref, A = orc.gemv(W, fmt, N, K, x, B)
-    for v in ((0, 2, 3, 4) if fmt == Q5_K else (0, 2, 3)):
+    for v in (0, 2, 3, 4):
         buf = torch.full((N * B + 128,), 12345.0, dtype=torch.float32, device=dev)
         y = buf[64:64 + N * B]
         qg.qg_gemv_variant(_t(W, dev), fmt, N, K, _t(x.view(np.uint16), dev), B, y, None, v)
@@ -325,5 +326,5 @@ def test_q6k_tail_window_every_misalignment(dev, orc):
             W = synth.q6k_weights(N, K, seed=N)
             x = synth.activations(K, B, seed=N)
             yref, A = orc.gemv(W, Q6_K, N, K, x, B)
-            for v in (0, 3):
+            for v in (0, 2, 3, 4):
                 assert_within(gpu_gemv(dev, W, Q6_K, N, K, x, v), yref, A, f"N={N} B={B} v{v}")
