@@ -1,4 +1,5 @@
-// qg_mma.cuh -- the tensor-core streaming GEMV of libqg (sm_100a) for Q4_K, B = 1..8 columns.
+// qg_mma.cuh -- the tensor-core streaming GEMV of libqg (sm_100a) for the K-quants (Q4_K, Q5_K,
+// Q6_K), B = 1..8 columns (Q4_K: up to 16).
 //
 // Operation (HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle), second prompt, "SPEC"):
 //   y[n,b] = sum_k dequant(W)[n,k] * x[k,b], fp32 accumulation ("PHYSICS & CONTRACT"), Q4_K
@@ -26,6 +27,8 @@
 //     by D_j of its row and added to the warp's accumulators.
 // The scales come from a per-warp table: lane l decodes row l's header (as in the CUDA-core
 // kernel), writes D_j for its row, and folds -M_j * sum(x over j) into its own per-row sum.
+// Q5_K and Q6_K keep this skeleton; their high-bit planes are merged into the A words byte-wise
+// (q5k_a_regs, mma_q6k_step), and Q6_K scales each 16-weight k-tile by its own group's D_t.
 #pragma once
 
 #include "qg_rows.cuh"

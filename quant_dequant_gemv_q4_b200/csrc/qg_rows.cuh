@@ -2,19 +2,20 @@
 //
 // Operation (HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle), second prompt, "SPEC"):
 //   y[n,b] = sum_k dequant(W)[n,k] * x[k,b] with the format chosen by a flag, fp32 accumulation
-//   ("PHYSICS & CONTRACT"), Q4_K w = d*sc*q - dmin*m ("QUANTIZATION MIX"), Q8_0 w = d*q.
+//   ("PHYSICS & CONTRACT"), Q4_K w = d*sc*q - dmin*m ("QUANTIZATION MIX"), Q8_0 w = d*q; the
+//   dossier's mix also holds Q5_K (5-bit q) and Q6_K (w = d*sc*(q - 32), 16-weight scale groups).
 //
 // Mapping.  CTA c of K slice s owns a band of consecutive rows [R0, R1) and the slice's units.
 // Its warps take (row group, K part) pairs: a row group is 32 consecutive rows of the band, a K
-// part an equal share of the slice's 256-weight units.  Lane l of a warp owns row 32g + l of
-// its group and decodes that row's whole unit (all 8 sub-blocks) per step, so the scale/min table
-// is decoded once per 256 weights with SWAR masks and every x read is a broadcast (all lanes read
-// the same unit of x).  One 2-D TMA tensor copy (cp.async.bulk.tensor.2d) per step brings 32 rows
-// x one unit (144 B for Q4_K, 272 B for Q8_0; both odd multiples of 16 B, so 8 consecutive lanes
-// reading 16 B from 8 rows hit 8 different bank groups) into the warp's double-buffered ring.
-// When all warps are done, the K parts of each row are added in shared memory in part order and
-// the band's rows are written once: no atomics and no scratch (with S > 1 slices, each slice
-// writes partial rows and a second kernel adds them in slice order).
+// part every P-th of the slice's 256-weight units.  Lane l of a warp owns row 32g + l of its
+// group and decodes that row's whole unit per step, so the scale/min table is decoded once per
+// 256 weights with SWAR masks and every x read is a broadcast (all lanes read the same unit of
+// x).  One 2-D TMA tensor copy (cp.async.bulk.tensor.2d) per step brings 32 rows x one unit (144 B
+// Q4_K, 176 B Q5_K, 272 B Q8_0: odd multiples of 16 B, so 8 consecutive lanes reading 16 B from
+// 8 rows hit 8 different bank groups) into the warp's double-buffered ring; Q6_K rows (210 B per
+// unit) take one bulk copy per lane.  When all warps are done, the K parts of each row are added
+// in shared memory in part order and the band's rows are written once: no atomics (with S > 1
+// slices, each slice writes partial rows and the band's last CTA adds them in slice order).
 //
 // Arithmetic (factored form).  With D_j = d*sc_j and M_j = dmin*m_j (both exact in fp32),
 //   sum_i w_i x_i = sum_j [ D_j * sum_{i in j} q_i x_i  -  M_j * sum_{i in j} x_i ].
