@@ -473,14 +473,20 @@ def run_reference(args):
 
 
 def run_ncu_case(args):
-    """The headline tensor, one copy on the device: 3 launches at B=1, then 3 at B=8."""
+    """The headline tensor, one copy on the device: 3 launches at B=1, then 3 at B=8.  With
+    --ncu-fmt 13 or 14 the same tensor shape in Q5_K / Q6_K instead (3 launches at B=1, then 3 at
+    B=8)."""
     import torch
     from quant_dequant_gemv_q4_b200 import build as qbuild
     qbuild.build()
     import quant_dequant_gemv_q4_b200 as qg
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    for call in (HEADLINE, HEADLINE_B8):
+    calls = (HEADLINE, HEADLINE_B8)
+    if args.ncu_fmt != synth.Q4_K:
+        calls = tuple(synth.Gemv(f"ffn_gate_b{b}", args.ncu_fmt, HEADLINE.N, HEADLINE.K, b, 0)
+                      for b in (1, 8))
+    for call in calls:
         wl = synth.Workload("ncu", HEADLINE_SEED, (call,))
         W, x = wl.inputs(call)
         Wd = torch.from_numpy(W).to(device)
@@ -512,6 +518,8 @@ def main(argv=None):
     ap.add_argument("--ncu-case", action="store_true",
                     help="launch the headline call 3x at B=1 then 3x at B=8 on one weight copy "
                          "and exit (the small case an ncu capture runs; nothing is timed)")
+    ap.add_argument("--ncu-fmt", type=int, default=12,
+                    help="--ncu-case format: 12 Q4_K (default), 13 Q5_K, 14 Q6_K")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
