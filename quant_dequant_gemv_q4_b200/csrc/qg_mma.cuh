@@ -532,11 +532,11 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
         for (int i = 0; i < kRowsStages; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
         if (!PER_LANE)
-            for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue(i);
+            for (int i = 0; i < kPreStages && i < nsteps; ++i) issue(i);
     }
     if (PER_LANE && nsteps > 0) {
         __syncwarp();
-        for (int i = 0; i < kRowsStages && i < nsteps; ++i) issue_lanes(i);
+        for (int i = 0; i < kPreStages && i < nsteps; ++i) issue_lanes(i);
     }
     // 2. programmatic dependent launch: let the next kernel start prefetching, then wait for the
     //    previous kernel's results before reading x or writing y
@@ -544,6 +544,12 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // 3. x fragments and sub-block sums of this slice
     mma_stage_x<BP, FMT>(a, s, US_s, xf, xsum);
+    // the rest of the ring, once this warp's x loads have returned (as in rows_gemv_kernel)
+    if (PER_LANE) {
+        for (int i = kPreStages; i < kRowsStages && i < nsteps; ++i) issue_lanes(i);
+    } else if (lane == 0) {
+        for (int i = kPreStages; i < kRowsStages && i < nsteps; ++i) issue(i);
+    }
     __syncthreads();
 
     int step = 0;
