@@ -122,6 +122,24 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
 int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
             void *stream);
 
+/* qg_gemv for a caller whose activations live in host memory: enqueues on `stream` the copy of
+ * x_host into library-owned device scratch, the GEMV (the default kernel variant) and the copy
+ * of y back to y_host, so one call does what a host-side caller would otherwise do in three.
+ *   W        device, as for qg_gemv (weights stay resident on the GPU)
+ *   x_host   host, fp16 bits [K][B], 2-byte aligned; read by the copy engine when the stream
+ *            reaches the call
+ *   y_host   host, fp32 [N][B], 4-byte aligned; valid after the stream has been synchronized
+ *   fmt, N, K, B, stream as for qg_gemv.
+ * With page-locked (pinned) host buffers nothing is copied by a separate operation: a small
+ * kernel reads x_host into the scratch (chained to the GEMV, whose weight prefetch overlaps it)
+ * and the GEMV writes y straight into y_host.  Pageable buffers take two stream copies, which the
+ * CUDA runtime stages (the call may then block the host).  The scratch (K*B*2 + N*B*4 bytes) is one
+ * pair of buffers per (device, stream), allocated on first use and grown when a larger call
+ * comes (never during stream capture: QG_ERR_NOMEM then); calls on one stream share it, in
+ * stream order.  Errors as qg_gemv; argument errors are found before anything is enqueued. */
+int qg_gemv_host(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x_host, int B,
+                 float *y_host, void *stream);
+
 /* The FFN gate/up pair on one x, fused with its activation:
  *     h[n,b] = silu(gate[n,b]) * up[n,b],  gate = dequant(Wg) . x,  up = dequant(Wu) . x,
  *     silu(v) = v / (1 + e^-v)

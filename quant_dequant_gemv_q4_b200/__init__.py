@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.qg_gemv_variant.restype = I
         L.qg_gemv_noalloc.argtypes = [P, I, I64, I64, P, I, P, P]
         L.qg_gemv_noalloc.restype = I
+        L.qg_gemv_host.argtypes = [P, I, I64, I64, P, I, P, P]
+        L.qg_gemv_host.restype = I
         L.qg_gemv_gate_up_silu.argtypes = [P, P, I, I64, I64, P, I, P, P]
         L.qg_gemv_gate_up_silu.restype = I
         L.qg_gemv_residual.argtypes = [P, I, I64, I64, P, I, P, P, P]
@@ -136,6 +138,13 @@ def qg_gemv(W, fmt: int, N: int, K: int, x, B: int, y, stream=None) -> None:
     """Enqueue y = dequant(W) . x (all device pointers / CUDA tensors)."""
     _ok(lib().qg_gemv(_ptr(W), int(fmt), int(N), int(K), _ptr(x), int(B), _ptr(y),
                       _stream(stream)), "qg_gemv")
+
+
+def qg_gemv_host(W, fmt: int, N: int, K: int, x_host, B: int, y_host, stream=None) -> None:
+    """Enqueue x_host -> device, y = dequant(W) . x, y -> y_host (W on the device; x_host, y_host
+    host memory: pinned CPU tensors or numpy arrays).  y_host is valid after the stream syncs."""
+    _ok(lib().qg_gemv_host(_ptr(W), int(fmt), int(N), int(K), _ptr(x_host), int(B), _ptr(y_host),
+                           _stream(stream)), "qg_gemv_host")
 
 
 def qg_gemv_variant(W, fmt: int, N: int, K: int, x, B: int, y, stream=None,

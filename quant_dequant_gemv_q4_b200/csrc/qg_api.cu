@@ -670,9 +670,113 @@ int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *
     return QG_OK;
 }
 
+// The device address of page-locked host memory (registered or allocated with the CUDA
+// runtime), or nullptr for pageable memory.
+void *device_view_of_host(const void *p)
+{
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        (void)cudaGetLastError();  // an unknown pointer: clear the error, treat it as pageable
+        return nullptr;
+    }
+    if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
+    return at.devicePointer;
+}
+
+// Device scratch for x and y of qg_gemv_host: one pair per (device, stream), grown on demand.
+struct IoBuf {
+    void *x = nullptr, *y = nullptr;
+    size_t xb = 0, yb = 0;
+};
+std::map<std::pair<int, void *>, IoBuf> g_io;
+
+int get_iobuf(int dev, void *stream, size_t xb, size_t yb, IoBuf *out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    IoBuf &b = g_io[{dev, stream}];
+    if (b.xb >= xb && b.yb >= yb && b.x && b.y) {
+        *out = b;
+        return QG_OK;
+    }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap) != cudaSuccess)
+        return QG_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return QG_ERR_NOMEM;  // cannot grow while capturing
+    if (b.x || b.y) {
+        // queued work on this stream may still use the old buffers
+        if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QG_ERR_CUDA;
+        cudaFree(b.x);
+        cudaFree(b.y);
+    }
+    const size_t nx = std::max(xb, b.xb), ny = std::max(yb, b.yb);
+    b = IoBuf();
+    void *px = nullptr, *py = nullptr;
+    if (cudaMalloc(&px, nx) != cudaSuccess) return QG_ERR_NOMEM;
+    if (cudaMalloc(&py, ny) != cudaSuccess) {
+        cudaFree(px);
+        return QG_ERR_NOMEM;
+    }
+    b.x = px;
+    b.y = py;
+    b.xb = nx;
+    b.yb = ny;
+    *out = b;
+    return QG_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int qg_gemv_host(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x_host, int B,
+                 float *y_host, void *stream)
+{
+    int rc = check_common(W, fmt, N, K);
+    if (rc != QG_OK) return rc;
+    if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
+    // 9..16 columns run on the Q4_K tensor-core kernel only (rows of whole 256-weight units)
+    if (B > 8 && (fmt != QG_FMT_Q4_K || K % 256 != 0)) return QG_ERR_BATCH;
+    if (N == 0) return QG_OK;
+    if (!x_host || !y_host) return QG_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x_host) % 2 != 0 || reinterpret_cast<uintptr_t>(y_host) % 4 != 0)
+        return QG_ERR_ALIGN;
+    DeviceInfo di;
+    int dev = 0;
+    if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    const size_t xb = (size_t)K * (size_t)B * sizeof(uint16_t), yb = (size_t)N * (size_t)B * sizeof(float);
+    IoBuf io;
+    if ((rc = get_iobuf(dev, stream, xb, yb, &io)) != QG_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Page-locked host memory is readable and writable from the device: x is then read by a
+    // small kernel chained to the GEMV (no separate copy operation on the stream) and y is
+    // written by the GEMV straight into y_host.  Pageable memory takes stream copies.
+    const void *xdev_host = device_view_of_host(x_host);
+    void *ydev_host = device_view_of_host(y_host);
+    if (xdev_host) {
+        const int64_t n = K * B;
+        const int64_t pieces = (n + 7) / 8;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((pieces + 255) / 256));
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const uint16_t *src = static_cast<const uint16_t *>(xdev_host);
+        uint16_t *dst = static_cast<uint16_t *>(io.x);
+        if (cudaLaunchKernelEx(&cfg, host_x_copy_kernel, src, dst, n) != cudaSuccess) return QG_ERR_CUDA;
+    } else if (cudaMemcpyAsync(io.x, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+        return QG_ERR_CUDA;
+    }
+    float *ydst = ydev_host ? static_cast<float *>(ydev_host) : static_cast<float *>(io.y);
+    rc = gemv_impl(W, fmt, N, K, static_cast<const uint16_t *>(io.x), B, ydst, stream, QG_VARIANT_AUTO);
+    if (rc != QG_OK) return rc;
+    if (!ydev_host && cudaMemcpyAsync(y_host, io.y, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return QG_ERR_CUDA;
+    return QG_OK;
+}
 
 int qg_gemv_residual(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
                      const float *r, float *y, void *stream)

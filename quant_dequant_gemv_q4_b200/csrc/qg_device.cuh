@@ -886,6 +886,37 @@ __global__ void rowwise_gemv_kernel(const uint8_t *W, int64_t N, int64_t K, cons
 }
 
 // ------------------------------------------------------------------------------------------------
+// x from page-locked host memory into device scratch (qg_gemv_host).  Each thread reads one
+// 16-byte piece (or, unaligned, 8 halves one by one) of the host copy first, which depends on no
+// earlier work, then waits for the previous kernel on the stream before it overwrites the scratch
+// that kernel may still be reading; it lets the next kernel (the GEMV) launch at once, so the
+// GEMV's weight prefetch overlaps the copy.
+// ------------------------------------------------------------------------------------------------
+__global__ void host_x_copy_kernel(const uint16_t *src, uint16_t *dst, int64_t n)
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int64_t i0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0;
+    uint16_t v[8];
+    uint4 q = make_uint4(0u, 0u, 0u, 0u);
+    const bool whole = aligned && i0 + 8 <= n;
+    if (whole) {
+        q = *reinterpret_cast<const uint4 *>(src + i0);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = (i0 + k < n) ? src[i0 + k] : (uint16_t)0;
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (whole) {
+        *reinterpret_cast<uint4 *>(dst + i0) = q;
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (i0 + k < n) dst[i0 + k] = v[k];
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
 // Bandwidth probes.
 // ------------------------------------------------------------------------------------------------
 __global__ void hbm_copy_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t n16)

@@ -257,3 +257,18 @@ def test_batch_width_limits(L):
     assert L.qg_gemv_noalloc(FAKE, 8, 4, 256, FAKE, 16, FAKE, None) == qg.QG_ERR_BATCH
     assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 8, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
     assert L.qg_gemv_residual(FAKE, 8, 4, 256, FAKE, 12, FAKE, FAKE, None) == qg.QG_ERR_BATCH
+
+
+def test_gemv_host_rejects_bad_arguments(L):
+    """qg_gemv_host checks its arguments before any device call or copy."""
+    f = L.qg_gemv_host
+    assert f(FAKE, 99, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_FMT
+    assert f(FAKE, 12, 4, 300, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
+    assert f(FAKE, 12, 4, 256, FAKE, 0, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, 8, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # 9..16: Q4_K only
+    assert f(FAKE, 14, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, 12, 4, 256, 0, 1, FAKE, None) == qg.QG_ERR_NULL
+    assert f(FAKE, 12, 4, 256, FAKE, 1, 0, None) == qg.QG_ERR_NULL
+    assert f(FAKE, 12, 4, 256, FAKE + 1, 1, FAKE, None) == qg.QG_ERR_ALIGN
+    assert f(FAKE, 12, 4, 256, FAKE, 1, FAKE + 2, None) == qg.QG_ERR_ALIGN
+    assert f(None, 12, 0, 256, None, 1, None, None) == qg.QG_OK  # N == 0: nothing to do

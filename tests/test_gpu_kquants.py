@@ -328,3 +328,31 @@ def test_q6k_tail_window_every_misalignment(dev, orc):
             yref, A = orc.gemv(W, Q6_K, N, K, x, B)
             for v in (0, 2, 3, 4):
                 assert_within(gpu_gemv(dev, W, Q6_K, N, K, x, v), yref, A, f"N={N} B={B} v{v}")
+
+
+# ------------------------------------------------------------------------------------------------
+# Host-buffer entry point
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt,N,K,B", [(12, 1000, 5120, 1), (12, 300, 2560, 12), (13, 129, 2560, 4),
+                                       (14, 77, 5120, 1), (8, 200, 96, 3)])
+@pytest.mark.parametrize("pinned", [True, False])
+def test_gemv_host_matches_device_call(dev, orc, fmt, N, K, B, pinned):
+    """qg_gemv_host (x and y in host memory) gives the same bits as qg_gemv on device buffers."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    W = synth.weights(fmt, N, K, seed=N + B)
+    x = synth.activations(K, B, seed=K + B)
+    Wd = _t(W, dev)
+    y_dev = gpu_gemv(dev, W, fmt, N, K, x, 0)
+    xh = torch.from_numpy(x.view(np.uint16).copy())
+    yh = torch.full((N, B), float("nan"), dtype=torch.float32)
+    if pinned:
+        xh, yh = xh.pin_memory(), yh.pin_memory()
+    s = torch.cuda.current_stream()
+    for _ in range(2):  # the second call reuses the scratch
+        qg.qg_gemv_host(Wd, fmt, N, K, xh, B, yh, s)
+    s.synchronize()
+    assert np.array_equal(yh.numpy().view(np.uint32), y_dev.view(np.uint32))
+    yref, A = orc.gemv(W, fmt, N, K, x, B)
+    assert_within(yh.numpy(), yref, A, f"host fmt={fmt}")
