@@ -1,11 +1,16 @@
-// qg_device.cuh -- device code of libqg: block-format decoding, the streaming GEMV kernel, the
-// split-K second pass, the dequant dump, a plain per-row kernel and bandwidth probes (sm_100a).
+// qg_device.cuh -- device code of libqg shared by the kernels (PTX wrappers: mbarriers, bulk
+// copies, timers), plus the kernels that are not the default streaming ones: the four-lanes-per-
+// unit kernel of QG_VARIANT_DIRECT (stream_gemv_kernel) and its split-K second pass, the dequant
+// dumps, the plain per-row kernel of QG_VARIANT_GENERIC, the host-x copy of qg_gemv_host, and
+// bandwidth probes (sm_100a).  The default kernels are in qg_rows.cuh (CUDA cores) and qg_mma.cuh
+// (tensor cores).
 //
 // Operation (HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle), second prompt, "SPEC"):
 //   y[n,b] = sum_k dequant(W)[n,k] * x[k,b], format chosen per call by a flag; fp32 accumulation
-//   ("PHYSICS & CONTRACT"); Q4_K w = d*sc*q - dmin*m ("QUANTIZATION MIX"); Q8_0 w = d*q.
+//   ("PHYSICS & CONTRACT"); Q4_K w = d*sc*q - dmin*m ("QUANTIZATION MIX"); Q8_0 w = d*q; Q5_K and
+//   Q6_K (the same mix) in the dumps and the per-row kernel.
 //
-// Work decomposition of the streaming kernel.  A "unit" is 256 consecutive weights of one row:
+// Work decomposition of stream_gemv_kernel (Q4_K and Q8_0).  A "unit" is 256 consecutive weights of one row:
 // one Q4_K superblock (144 B) or eight Q8_0 blocks (272 B).  Both are 16-byte multiples, so any
 // run of whole units of a row is a legal bulk-copy source.  The K axis may be cut into S slices
 // (only when x for the whole of K would not fit in shared memory); slice s of row n is a
