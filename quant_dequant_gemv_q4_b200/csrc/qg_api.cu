@@ -266,24 +266,25 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     const size_t bars = (size_t)NW * kRowsStages * 8;
 
     const int64_t UPR = K / 256;
-    // K slices: the fewest for which x fits in shared memory and the row bands keep at least 85%
-    // of their 32-row lanes busy (bands of N*S/SMs rows); otherwise the best such fraction.
-    // The 16-warp CUDA-core kernels (B = 1) instead take one slice when that keeps 70% of the
-    // lanes busy, else, among the slicings with 85% busy lanes and at least 12 (row group, K
-    // part) pairs, the one with the fewest 32-row steps per CTA (or NW times the steps of the
-    // busiest warp, if more).  Measured: a call takes about 3.3 us + 0.11 us per step of a CTA,
-    // plus about 1.5 us for the cross-CTA sum when K is sliced.
-    const bool step_rule = !tensor && NW == 16;
-    RowsPlan first85{};
-    RowsPlan step_best{};
-    int64_t step_best_cost = INT64_MAX;
+    // K slices.  Among the slicings whose shared memory fits (and, past one slice, whose slices
+    // keep at least 5 units of a row, so that each row is still read in long runs), the least
+    //   cost = max(steps of a CTA, NW * steps of its busiest warp) + [S > 1] * 16 * 144 / UB
+    // in 32-row steps: a call took about 3.3 us + 0.11 us per step of a CTA, plus about 1.8 us
+    // (16 Q4_K steps) for the cross-CTA sum of K slices, when measured over slicings of the FFN,
+    // attention and SSM shapes at B = 1 and 8 (the warp term covers bands with too few (row
+    // group, K part) pairs to keep every warp streaming).  Ties: fewer steps, then fewer slices.
+    // The tensor-core kernel only takes slicings with at most one pair per warp.  If no slicing
+    // qualifies, the one with the most busy lanes.
+    const int UB = tensor ? (fmt == kFmtQ5_K ? 176 : fmt == kFmtQ6_K ? 210 : 144)
+                          : (fmt == kFmtQ6_K ? 210 : LB);
+    double best_cost = 1e300;
+    int64_t best_steps = INT64_MAX;
+    RowsPlan util_best{};
     for (int64_t S0 = 1; S0 <= std::min<int64_t>(UPR, 64); ++S0) {
         const int64_t US = (UPR + S0 - 1) / S0;
         const int64_t S = (UPR + US - 1) / US;
         if (S != S0) continue;  // the same slicing as a smaller S0
         const int64_t Gs = std::max<int64_t>(1, std::min<int64_t>(di.sms / S, N));
-        // partial rows are kept in shared memory only when a band has several K parts, and then
-        // there is at most one (row group, part) pair per warp
         // partial rows: one (group, part) pair per warp, or, for the gate/up pair, every group of
         // both matrices when there are more groups than warps
         const int64_t band_rows = (N + Gs - 1) / Gs;
@@ -303,25 +304,23 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         p.red_floats = red;
         p.smem = smem;
         p.tensor = tensor;
-        if (step_rule) {
-            if (S == 1 && util >= 0.70) return p;
-            const int64_t P = std::max<int64_t>(1, std::min<int64_t>(NW / std::max<int64_t>(groups, 1), US));
-            const int64_t warp_steps = ((groups * P + NW - 1) / NW) * ((US + P - 1) / P);
-            const int64_t cost = std::max<int64_t>(groups * US, NW * warp_steps);
-            if (util >= 0.85 && groups * P >= 12 && cost < step_best_cost) {
-                step_best_cost = cost;
-                step_best = p;
-            }
-        }
-        if (util >= 0.85 && first85.smem == 0) first85 = p;
         if (util > best_util) {
             best_util = util;
+            util_best = p;
+        }
+        if (S > 1 && US < 5) continue;
+        const int64_t P = std::max<int64_t>(1, std::min<int64_t>(NW / std::max<int64_t>(groups, 1), US));
+        if (tensor && groups * P > NW) continue;  // measured slower: tensor-core warps with two pairs
+        const int64_t warp_steps = ((groups * P + NW - 1) / NW) * ((US + P - 1) / P);
+        const int64_t steps = groups * US;
+        const double cost = (double)std::max<int64_t>(steps, NW * warp_steps) + (S > 1 ? 16.0 * 144.0 / UB : 0.0);
+        if (cost < best_cost || (cost == best_cost && steps < best_steps)) {
+            best_cost = cost;
+            best_steps = steps;
             best = p;
         }
-        if (!step_rule && first85.smem != 0) break;
     }
-    if (step_rule && step_best.smem != 0) return step_best;
-    if (first85.smem != 0) return first85;
+    if (best.smem == 0) best = util_best;
     return best;  // smem == 0 if nothing fits
 }
 

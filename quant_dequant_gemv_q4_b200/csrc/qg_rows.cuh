@@ -561,6 +561,22 @@ __device__ __forceinline__ void band_finish(const RowsArgs &a, const BandShape &
     }
 }
 
+// sum_{s < S} p[s * stride], added in slice order; the loads go out eight at a time, so the last
+// CTA of a band waits for ceil(S / 8) round trips to L2 rather than S.
+__device__ __forceinline__ float slice_sum(const float *p, int64_t stride, int S)
+{
+    float sum = 0.0f;
+    for (int s0 = 0; s0 < S; s0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = (s0 + j < S) ? __ldcg(p + (int64_t)(s0 + j) * stride) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (s0 + j < S) sum += v[j];
+    }
+    return sum;
+}
+
 // Split-K across CTAs without a second kernel.  CTA (slice s, band) has written its band's
 // partial rows to out = part[s][mats][N][B]; each makes its writes visible and bumps the band's
 // counter, and the last of the S CTAs to arrive adds the S slices in slice order (so y does not
@@ -588,11 +604,7 @@ __device__ __forceinline__ void splitk_fixup(const RowsArgs &a, int band, int64_
         const int64_t idx = R0 * a.B + t;
         float v[MATS];
 #pragma unroll
-        for (int m = 0; m < MATS; ++m) {
-            float sum = 0.0f;
-            for (int s2 = 0; s2 < a.S; ++s2) sum += __ldcg(a.out + ((int64_t)s2 * MATS + m) * NB + idx);
-            v[m] = sum;
-        }
+        for (int m = 0; m < MATS; ++m) v[m] = slice_sum(a.out + (int64_t)m * NB + idx, (int64_t)MATS * NB, a.S);
         if (MATS == 2) a.y[idx] = a.act ? silu_mul(v[0], v[MATS - 1]) : v[0];
         else a.y[idx] = a.res ? v[0] + a.res[idx] : v[0];
     }
