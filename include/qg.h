@@ -197,6 +197,26 @@ int qg_last_variant(void);
 /* Number of K slices the last GEMV of the calling thread used (1 = no split-K second pass). */
 int qg_last_splits(void);
 
+/* The launch plan a call would use, computed on the host; no GPU work and no allocation.
+ * Arguments as qg_gemv_variant's (fmt, N >= 1, K, B, variant), plus:
+ *   mats        1 for qg_gemv / qg_gemv_variant / qg_gemv_residual, 2 for qg_gemv_gate_up_silu
+ *               (then variant must be QG_VARIANT_AUTO);
+ *   sms, smem_optin
+ *               the device's multiprocessor count and opt-in shared memory per block in bytes;
+ *               if either is <= 0, the current device's (which needs a GPU: QG_ERR_CUDA
+ *               without one);
+ *   out         host array of 6 int64_t, written on success:
+ *               {variant launched (QG_VARIANT_*, AUTO resolved), K slices S, 256-weight units
+ *                per slice (K/32 blocks for QG_VARIANT_GENERIC), CTAs launched, warps per CTA,
+ *                dynamic shared memory per CTA in bytes}.
+ * The slice count of the streaming kernels is the slicing with the least modelled cost in 32-row
+ * steps: max(steps of a CTA, warps x steps of its busiest warp), plus a fixed charge for the
+ * cross-CTA sum when K is sliced; this call lets a caller or a test see the choice.
+ * Returns QG_OK, or the argument error the call itself would return (QG_ERR_FMT, _SHAPE, _BATCH,
+ * _VARIANT, _NULL for out == NULL), or QG_ERR_SHAPE if no plan fits the shared memory. */
+int qg_plan(int fmt, int64_t N, int64_t K, int B, int variant, int mats, int sms, int smem_optin,
+            int64_t *out);
+
 /* Reads and clears the device error word of the workspace that (current device, stream) uses;
  * synchronizes the stream.  *flag = 0 if no device-side timeout happened, else a nonzero code. */
 int qg_device_error(void *stream, int *flag);

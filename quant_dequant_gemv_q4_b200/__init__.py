@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.qg_last_variant.restype = I
         L.qg_last_splits.argtypes = []
         L.qg_last_splits.restype = I
+        L.qg_plan.argtypes = [I, I64, I64, I, I, I, I, I, ctypes.POINTER(I64)]
+        L.qg_plan.restype = I
         L.qg_device_error.argtypes = [P, ctypes.POINTER(I)]
         L.qg_device_error.restype = I
         L.qg_hbm_copy.argtypes = [P, P, SZ, P]
@@ -207,6 +209,17 @@ def qg_last_variant() -> int:
 
 def qg_last_splits() -> int:
     return int(lib().qg_last_splits())
+
+
+def qg_plan(fmt: int, N: int, K: int, B: int, variant: int = 0, mats: int = 1, sms: int = 0,
+            smem_optin: int = 0) -> dict:
+    """The launch plan of a call (host only): variant, K slices, units per slice, CTAs, warps per
+    CTA, dynamic shared memory bytes.  sms / smem_optin <= 0: the current device's."""
+    out = (ctypes.c_int64 * 6)()
+    _ok(lib().qg_plan(int(fmt), int(N), int(K), int(B), int(variant), int(mats), int(sms),
+                      int(smem_optin), out), "qg_plan")
+    keys = ("variant", "splits", "units_per_slice", "ctas", "warps", "smem")
+    return dict(zip(keys, (int(v) for v in out)))
 
 
 def qg_device_error(stream=None) -> int:

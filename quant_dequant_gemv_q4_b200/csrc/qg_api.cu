@@ -280,7 +280,9 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     double best_cost = 1e300;
     int64_t best_steps = INT64_MAX;
     RowsPlan util_best{};
-    for (int64_t S0 = 1; S0 <= std::min<int64_t>(UPR, 64); ++S0) {
+    // at most 64 slices, and no more slices than SMs (every slice gets at least one CTA per wave)
+    const int64_t max_slices = std::min<int64_t>(std::min<int64_t>(UPR, 64), std::max(di.sms, 1));
+    for (int64_t S0 = 1; S0 <= max_slices; ++S0) {
         const int64_t US = (UPR + S0 - 1) / S0;
         const int64_t S = (UPR + US - 1) / US;
         if (S != S0) continue;  // the same slicing as a smaller S0
@@ -525,6 +527,23 @@ int auto_variant(int fmt, int64_t K, int B)
     return (fmt != QG_FMT_Q8_0 && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
 }
 
+// The kernel variant a GEMV call runs (QG_VARIANT_AUTO resolved), or the argument error.
+int resolve_variant(int fmt, int64_t K, int B, int variant, int *var_out)
+{
+    // the streaming kernels need rows of whole 256-weight units (16-byte multiples): always for
+    // Q4_K, K % 256 == 0 for Q8_0
+    const bool streamable = (K % 256 == 0);
+    int var = variant;
+    if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
+    if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
+    if (var == QG_VARIANT_TENSOR && fmt == QG_FMT_Q8_0) return QG_ERR_VARIANT;
+    if (B > 8 && fmt != QG_FMT_Q4_K) return QG_ERR_BATCH;  // 9..16 columns: the Q4_K kernel only
+    if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
+    *var_out = var;
+    return QG_OK;
+}
+
 int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
               void *stream, int variant)
 {
@@ -536,16 +555,8 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     if (!x || !y) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
         return QG_ERR_ALIGN;
-    // the streaming kernels need rows of whole 256-weight units (16-byte multiples): always for
-    // Q4_K, K % 256 == 0 for Q8_0
-    const bool streamable = (K % 256 == 0);
-    int var = variant;
-    if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
-    if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
-    if (var == QG_VARIANT_TENSOR && fmt == QG_FMT_Q8_0) return QG_ERR_VARIANT;
-    if (B > 8 && fmt != QG_FMT_Q4_K) return QG_ERR_BATCH;  // 9..16 columns: the Q4_K kernel only
-    if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
+    int var = 0;
+    if ((rc = resolve_variant(fmt, K, B, variant, &var)) != QG_OK) return rc;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -855,6 +866,54 @@ int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, voi
 int qg_last_variant(void) { return t_last_variant; }
 
 int qg_last_splits(void) { return t_last_splits; }
+
+int qg_plan(int fmt, int64_t N, int64_t K, int B, int variant, int mats, int sms, int smem_optin,
+            int64_t *out)
+{
+    if (!out) return QG_ERR_NULL;
+    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K && fmt != QG_FMT_Q8_0)
+        return QG_ERR_FMT;
+    const int64_t bw = (fmt == QG_FMT_Q8_0) ? 32 : 256;
+    if (N < 1 || K < 1 || K % bw != 0 || (mats != 1 && mats != 2)) return QG_ERR_SHAPE;
+    if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
+    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TENSOR) return QG_ERR_VARIANT;
+    int var = 0, rc = QG_OK;
+    if (mats == 2) {
+        // the gate/up pair: the variant qg_gemv would take, rows of whole units
+        if (variant != QG_VARIANT_AUTO) return QG_ERR_VARIANT;
+        if (K % 256 != 0) return QG_ERR_SHAPE;
+        var = auto_variant(fmt, K, B);
+        if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
+    } else if ((rc = resolve_variant(fmt, K, B, variant, &var)) != QG_OK) {
+        return rc;
+    }
+    DeviceInfo di;
+    if (sms > 0 && smem_optin > 0) {
+        di.sms = sms;
+        di.smem_optin = smem_optin;
+    } else {
+        int dev = 0;
+        if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
+    }
+    if (var == QG_VARIANT_GENERIC) {
+        const int64_t blocks = std::min<int64_t>((N + 7) / 8, (int64_t)di.sms * 8);
+        const int64_t o[6] = {var, 1, K / bw, blocks, 8, 0};
+        std::memcpy(out, o, sizeof(o));
+        return QG_OK;
+    }
+    if (var == QG_VARIANT_DIRECT) {
+        const Plan p = make_plan(fmt, kVarDirect, N, K, B, di);
+        if ((size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+        const int64_t o[6] = {var, p.S, p.US, p.G, kWarps, (int64_t)p.smem};
+        std::memcpy(out, o, sizeof(o));
+        return QG_OK;
+    }
+    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR, mats);
+    if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
+    const int64_t o[6] = {var, p.S, p.US, p.G, p.NW, (int64_t)p.smem};
+    std::memcpy(out, o, sizeof(o));
+    return QG_OK;
+}
 
 int qg_device_error(void *stream, int *flag)
 {
