@@ -198,6 +198,18 @@ __device__ __forceinline__ void q5k_a_regs(uint32_t w, uint32_t hw, uint32_t &lo
     hi1 = __umulhi(wh, 1u << 24) & 0x001F001Fu;
 }
 
+// Row of a 16-row tile that fragment row g (lane >> 2) of mma.m16n8k16 stands for, in the Q4_K /
+// Q5_K steps: 2 (g mod 4) + g / 4.  Each half-warp's 8-byte A loads then read rows {0, 2, 4, 6}
+// or {1, 3, 5, 7}, which start 16 or 24 banks apart at the 144- and 176-byte row strides of the
+// ring (36 and 44 words), so the loads are free of bank conflicts; rows g = 0..3 in order would
+// start 4 (Q4_K) or 12 (Q5_K) banks apart and collide two-way.  Rows are independent outputs,
+// so the map only decides where each C fragment row lands.
+template <int FMT>
+__device__ __forceinline__ int mma_frag_row(int g)
+{
+    return (FMT == kFmtQ6_K) ? g : 2 * (g & 3) + (g >> 2);
+}
+
 template <int BP, int FMT = kFmtQ4_K>
 __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
                                              int US, int j, float *dtab,
@@ -207,6 +219,7 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
     constexpr int UB = MmaFmt<FMT>::kUnitBytes;
     constexpr int QS = MmaFmt<FMT>::kQs;
     const int g = lane >> 2, t = lane & 3;
+    const int pr = mma_frag_row<FMT>(g);  // the tile row of fragment row g
     {
         // header of row `lane`: the GGML get_scale_min_k4 table decoded with 32-bit masks (byte k
         // of each word = sub-block k or k+4), d and dmin exact in fp32
@@ -257,16 +270,16 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
                     const int col = (BP > 8) ? 8 * nt + g : g % BP;
                     xb[nt][lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
                 }
-        const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * g);
-        const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * g);
+        const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * pr);
+        const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * pr);
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile) {
-            const uint8_t *rowA = u0 + (tile * 16 + g) * UB + QS + 32 * c + 8 * t;
-            const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);           // row tile*16 + g
-            const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * UB);  // row tile*16 + g + 8
+            const uint8_t *rowA = u0 + (tile * 16 + pr) * UB + QS + 32 * c + 8 * t;
+            const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);           // row tile*16 + pr
+            const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * UB);  // row tile*16 + pr + 8
             uint2 qhA = make_uint2(0u, 0u), qhB = make_uint2(0u, 0u);  // Q5_K: qh words 2t, 2t+1
             if (FMT == kFmtQ5_K) {
-                const uint8_t *qhp = u0 + (tile * 16 + g) * UB + 16 + 8 * t;
+                const uint8_t *qhp = u0 + (tile * 16 + pr) * UB + 16 + 8 * t;
                 qhA = *reinterpret_cast<const uint2 *>(qhp);
                 qhB = *reinterpret_cast<const uint2 *>(qhp + 8 * UB);
             }
@@ -603,7 +616,7 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
         if (failed) break;
         // C fragments -> rows (row = lane) through the warp's table, plus the lane's min term
         {
-            const int g = lane >> 2, t = lane & 3;
+            const int pr = mma_frag_row<FMT>(lane >> 2), t = lane & 3;
 #pragma unroll
             for (int tile = 0; tile < 2; ++tile)
 #pragma unroll
@@ -611,7 +624,7 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int col = 8 * nt + 2 * t + (i & 1);
-                        if (col < BP) dtab[(tile * 16 + g + 8 * (i >> 1)) * BP + col] = acc[tile][nt][i];
+                        if (col < BP) dtab[(tile * 16 + pr + 8 * (i >> 1)) * BP + col] = acc[tile][nt][i];
                     }
         }
         __syncwarp();
