@@ -156,13 +156,13 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
     // consecutive lanes, which then add their halves into the chunk's two sub-block sums
     const int nchunk = 32 * BP * US;  // a multiple of 32: every lane of a warp takes part
     const bool vec = (BP == 1) && ((reinterpret_cast<uintptr_t>(xsl) & 7) == 0);
-    for (int t = threadIdx.x; t < nchunk; t += blockDim.x) {
+    // x[e0 .. e0+3], x[e0+HI .. e0+HI+3] of chunk t in natural order (zero past the slice)
+    auto load = [&](int t, uint32_t (&h)[8]) {
         const int i = t & 7;
         const int jcb = t >> 3;
         const int b = jcb % BP;
         const int jc = jcb / BP;
         const int c = jc & 3, j = jc >> 2;
-        uint32_t h[8];  // x[e0 .. e0+3], x[e0+32 .. e0+35] in natural order
         if (j < US_s && b < a.B) {
             const int e0 = j * 256 + rows_x_lo<FMT>(c, i);
             if (vec) {
@@ -181,6 +181,14 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
 #pragma unroll
             for (int q = 0; q < 8; ++q) h[q] = 0;
         }
+    };
+    // chunk t into shared memory, and its group sums (all 32 lanes of the warp together)
+    auto store = [&](int t, const uint32_t (&h)[8]) {
+        const int i = t & 7;
+        const int jcb = t >> 3;
+        const int b = jcb % BP;
+        const int jc = jcb / BP;
+        const int c = jc & 3, j = jc >> 2;
         uint4 v;  // group order (e, e+2, e+1, e+3)
         v.x = h[0] | (h[2] << 16);
         v.y = h[1] | (h[3] << 16);
@@ -222,6 +230,23 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
                 xsum[rows_xsum_off<BP, G>(US, j, g + 4, b)] = hi;
             }
         }
+    };
+    // two chunks per pass where a thread has two: both loads go out before either is used, so
+    // the pass waits for one round trip to L2 rather than two (the condition is uniform per warp:
+    // nchunk and blockDim.x are multiples of 32)
+    const int nthr = blockDim.x;
+    int t = threadIdx.x;
+    for (; t + nthr < nchunk; t += 2 * nthr) {
+        uint32_t ha[8], hb[8];
+        load(t, ha);
+        load(t + nthr, hb);
+        store(t, ha);
+        store(t + nthr, hb);
+    }
+    for (; t < nchunk; t += nthr) {
+        uint32_t h[8];
+        load(t, h);
+        store(t, h);
     }
 }
 
