@@ -44,11 +44,19 @@ HEADLINE_SEED = 4  # the batched-verify workload's seed
 FALLBACK_HBM_GBS = 6650.0
 
 
-def kernel_source_hash() -> str:
+# The sources the headline's CUDA-core kernel (rows_gemv_kernel) is built and launched from: its
+# device code and the host planner/launcher.  The tensor-core kernel's file (qg_mma.cuh) and the
+# host packer are not among them, so a change there leaves the headline's DRAM capture valid.
+ROWS_KERNEL_FILES = ("qg_api.cu", "qg_device.cuh", "qg_rows.cuh")
+MMA_KERNEL_FILES = ROWS_KERNEL_FILES + ("qg_mma.cuh",)  # the B >= 2 tensor-core kernel
+
+
+def kernel_source_hash(files=None) -> str:
+    """sha256 (16 hex digits) of the library's CUDA/C++ sources, or of the named ones only."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quant_dequant_gemv_q4_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".cpp", ".h")):
+        if f.endswith((".cu", ".cuh", ".cpp", ".h")) and (files is None or f in files):
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
@@ -394,15 +402,16 @@ def hbm_probe(device, nbytes=1 << 30, reps=10):
     return res
 
 
-def load_traffic(kernel_hash: str) -> dict | None:
-    """DRAM bytes per launch from a committed ncu capture summary, if it was taken on the current
-    kernel sources (same hash); else None."""
+def load_traffic(rows_hash: str) -> dict | None:
+    """DRAM bytes per launch of the headline kernel from a committed ncu capture summary, if it
+    was taken on the current sources of that kernel (same hash of ROWS_KERNEL_FILES); else
+    None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("kernel_hash") != kernel_hash:
+    if d.get("rows_kernel_hash") != rows_hash:
         return None
     return d
 
@@ -503,7 +512,9 @@ def run_ncu_case(args):
             qg.qg_gemv_variant(Wd, call.fmt, call.N, call.K, xd, call.B, yd, s, args.variant)
         torch.cuda.synchronize()
         del Wd, xd, yd
-    print(json.dumps({"ncu_case": "done", "kernel_hash": kernel_source_hash()}), flush=True)
+    print(json.dumps({"ncu_case": "done", "kernel_hash": kernel_source_hash(),
+                      "rows_kernel_hash": kernel_source_hash(ROWS_KERNEL_FILES),
+                      "mma_kernel_hash": kernel_source_hash(MMA_KERNEL_FILES)}), flush=True)
     return 0
 
 
@@ -564,7 +575,8 @@ def main(argv=None):
     per_launch_s = secs / (args.steps * launches)
     achieved = cs.bytes_per_step / launches / per_launch_s / 1e9
     khash = kernel_source_hash()
-    traffic = load_traffic(khash)
+    rows_hash = kernel_source_hash(ROWS_KERNEL_FILES)
+    traffic = load_traffic(rows_hash)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4),
                 "traffic": (traffic or {}).get("bytes_per_launch"),
@@ -680,6 +692,7 @@ def main(argv=None):
         "cpu_baseline": cpu,
         "hbm_probe": probe,
         "kernel_hash": khash,
+        "rows_kernel_hash": rows_hash,
         "workloads": table,
     }
     print(json.dumps(line), flush=True)
