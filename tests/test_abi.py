@@ -272,3 +272,20 @@ def test_gemv_host_rejects_bad_arguments(L):
     assert f(FAKE, 12, 4, 256, FAKE + 1, 1, FAKE, None) == qg.QG_ERR_ALIGN
     assert f(FAKE, 12, 4, 256, FAKE, 1, FAKE + 2, None) == qg.QG_ERR_ALIGN
     assert f(None, 12, 0, 256, None, 1, None, None) == qg.QG_OK  # N == 0: nothing to do
+
+
+def test_binding_constants_match_the_header():
+    """Every QG_* enum value and #define number of include/qg.h has the same value in the
+    binding (the binding restates them; this keeps the two from drifting)."""
+    src = open(os.path.join(ROOT, "include", "qg.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    values = {}
+    for body in re.findall(r"enum\s*\{(.*?)\}", src, flags=re.S):
+        for name, val in re.findall(r"(QG_\w+)\s*=\s*(\d+)", body):
+            values[name] = int(val)
+    for m in re.finditer(r"#define\s+(QG_\w+)\s+\((\d+)u\s*<<\s*(\d+)\)", src):
+        values[m.group(1)] = int(m.group(2)) << int(m.group(3))
+    assert {"QG_FMT_Q4_K", "QG_VARIANT_TENSOR", "QG_ERR_SCRATCH", "QG_OK"} <= set(values)
+    for name, val in values.items():
+        assert hasattr(qg, name), name
+        assert getattr(qg, name) == val, (name, getattr(qg, name), val)
