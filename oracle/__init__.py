@@ -23,6 +23,7 @@ Q8_0 = 8  # GGML type id of the Q8_0 block format
 Q4_K = 12  # GGML type id of the Q4_K superblock format
 Q5_K = 13  # GGML type id of the Q5_K superblock format
 Q6_K = 14  # GGML type id of the Q6_K superblock format
+IQ4_XS = 23  # GGML type id of the IQ4_XS superblock format (non-linear 4-bit codebook)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qg_oracle.c")
@@ -67,6 +68,10 @@ def lib():
         L.orc_unpack_q5k.restype = I
         L.orc_unpack_q6k.argtypes = [P, I64, P, P, P]
         L.orc_unpack_q6k.restype = I
+        L.orc_unpack_iq4xs.argtypes = [P, I64, P, P, P]
+        L.orc_unpack_iq4xs.restype = I
+        L.orc_iq4_level.argtypes = [I]
+        L.orc_iq4_level.restype = I
         _lib = L
     return _lib
 
@@ -191,3 +196,20 @@ def unpack_q6k(W: np.ndarray, nsb: int) -> dict:
     q = np.empty((nsb, 256), np.int8)
     _check(lib().orc_unpack_q6k(_ptr(W), nsb, _ptr(d), _ptr(scales), _ptr(q)), "unpack_q6k")
     return {"d": d, "scales": scales, "q": q}
+
+
+def unpack_iq4xs(W: np.ndarray, nsb: int) -> dict:
+    """Field view of nsb IQ4_XS superblocks: d (fp16 bits), ls [nsb, 8] (stored 6-bit scales; the
+    multiplier is ls - 32), idx [nsb, 256] codebook indices 0..15."""
+    W = np.ascontiguousarray(W, dtype=np.uint8)
+    assert W.size >= nsb * 136
+    d = np.empty(nsb, np.uint16)
+    ls = np.empty((nsb, 8), np.uint8)
+    idx = np.empty((nsb, 256), np.uint8)
+    _check(lib().orc_unpack_iq4xs(_ptr(W), nsb, _ptr(d), _ptr(ls), _ptr(idx)), "unpack_iq4xs")
+    return {"d": d, "ls": ls, "idx": idx}
+
+
+def iq4_level(v: int) -> int:
+    """The oracle's codebook level of index v."""
+    return int(lib().orc_iq4_level(int(v)))

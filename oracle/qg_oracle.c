@@ -20,7 +20,9 @@
  *       packing ("get_scale_min_k4" layout), the Q4_K nibble order, and Q8_0 = {half d; int8 qs[32]}
  *       with w = d*q.  The same dossier's quant mix also lists Q5_K and Q6_K (GGML's K-quants with a
  *       fifth bit per weight, and with 6-bit weights and 16 int8 group scales); their layouts are
- *       written out at orc_q5k_quant and orc_q6k_quant below.
+ *       written out at orc_q5k_quant and orc_q6k_quant below.  The dossier's second prompt
+ *       ("SPEC", "OUTPUT") also names IQ4_XS, GGML's 4-bit format whose indices select values of
+ *       a fixed 16-entry non-linear codebook; its layout is written out at orc_iq4xs_index.
  *
  * Definition computed (exact up to the final fp64 summation):
  *   w[n,k]  = the fp32 dequantized weight, computed exactly in fp64 and rounded ONCE to fp32
@@ -28,13 +30,14 @@
  *             significant bits, and their difference spans at most 50 bits, so the fp64 value is
  *             exact and the single cast is the correctly rounded fp32 weight.  Q5_K is the same
  *             with 5-bit q (d*sc*q at most 22 bits).  Q6_K: d*sc*(q-32) has at most 25 significant
- *             bits, exact in fp64, rounded once.  For Q8_0, d*q is exact in fp32.
+ *             bits, exact in fp64, rounded once.  For Q8_0, d*q is exact in fp32.  IQ4_XS:
+ *             d*(ls-32)*v has at most 11 + 5 + 7 = 23 significant bits, exact in fp32.
  *   y[n,b]  = sum_k w[n,k] * x[k,b]    in fp64, k ascending (each product is exact in fp64);
  *   A[n,b]  = sum_k |w[n,k] * x[k,b]|  in fp64, the scale of the error bound
  *             |y_gpu - y| <= 1e-5 * A + 1e-6.
  *
  * Layouts: W is row-major, row n is K/256 consecutive superblocks (144 B Q4_K, 176 B Q5_K,
- * 210 B Q6_K) or K/32 consecutive 34-byte Q8_0 blocks; x is fp16 bits, x[k*B + b]; y and A are
+ * 210 B Q6_K, 136 B IQ4_XS) or K/32 consecutive 34-byte Q8_0 blocks; x is fp16 bits, x[k*B + b]; y and A are
  * y[n*B + b].
  *
  * Build with -ffp-contract=off so that no product is fused into a sum.
@@ -49,6 +52,7 @@
 #define ORC_Q4_K 12
 #define ORC_Q5_K 13
 #define ORC_Q6_K 14
+#define ORC_IQ4_XS 23
 
 #define ORC_OK 0
 #define ORC_EINVAL 1
@@ -184,6 +188,46 @@ static void orc_dequant_q6k_block(const uint8_t *blk, float *w)
     }
 }
 
+/* IQ4_XS: 256 weights in 136 bytes: fp16 d (0-1), a little-endian uint16 scales_h (2-3),
+ * scales_l[4] (4-7), qs[128] (8-135).  Sub-block j (32 weights, j = 0..7) has the 6-bit scale
+ *   ls_j = (nibble j % 2 of scales_l[j / 2]: the low nibble for even j, the high for odd j)
+ *          + 16 * (bits 2j, 2j+1 of scales_h),
+ * and weight i of sub-block j = i / 32, with r = i % 32, has the 4-bit index held by
+ * qs[16j + r % 16]: its low nibble for r < 16, its high nibble for r >= 16.  The index selects
+ * one of sixteen fixed integer levels (the codebook below, spaced more finely near zero), and
+ *   w = d * (ls_j - 32) * codebook[index],
+ * at most 23 significant bits: exact in fp32. */
+static const int orc_iq4_levels[16] = {-127, -104, -83, -65, -49, -35, -22, -10,
+                                       1,    13,   25,  38,  53,  69,  89,  113};
+
+static int orc_iq4xs_scale(const uint8_t *blk, int j)
+{
+    int scales_h = blk[2] | (blk[3] << 8);
+    int low = (blk[4 + j / 2] >> (4 * (j % 2))) & 15;
+    int high = (scales_h >> (2 * j)) & 3;
+    return low + 16 * high;
+}
+
+static int orc_iq4xs_index(const uint8_t *qs, int i)
+{
+    int j = i / 32;
+    int r = i % 32;
+    uint8_t byte = qs[16 * j + (r % 16)];
+    return (r < 16) ? (byte & 15) : (byte >> 4);
+}
+
+static void orc_dequant_iq4xs_block(const uint8_t *blk, float *w)
+{
+    double d = orc_half_to_double((uint16_t)(blk[0] | (blk[1] << 8)));
+    const uint8_t *qs = blk + 8;
+    for (int i = 0; i < 256; ++i) {
+        int ls = orc_iq4xs_scale(blk, i / 32);
+        int v = orc_iq4_levels[orc_iq4xs_index(qs, i)];
+        double exact = d * (double)(ls - 32) * (double)v;
+        w[i] = (float)exact;
+    }
+}
+
 /* One Q8_0 block (34 bytes) -> 32 fp32 weights, w = d * q. */
 static void orc_dequant_q8_0_block(const uint8_t *blk, float *w)
 {
@@ -208,6 +252,9 @@ static int orc_block_geometry(int fmt, int64_t K, int64_t *block_w, int64_t *blo
     } else if (fmt == ORC_Q6_K) {
         *block_w = 256;
         *block_b = 210;
+    } else if (fmt == ORC_IQ4_XS) {
+        *block_w = 256;
+        *block_b = 136;
     } else {
         return ORC_EINVAL;
     }
@@ -237,6 +284,8 @@ static void orc_dequant_row(int fmt, const uint8_t *W, int64_t n, int64_t K, flo
             orc_dequant_q5k_block(row + t * bb, w + t * bw);
         else if (fmt == ORC_Q6_K)
             orc_dequant_q6k_block(row + t * bb, w + t * bw);
+        else if (fmt == ORC_IQ4_XS)
+            orc_dequant_iq4xs_block(row + t * bb, w + t * bw);
         else
             orc_dequant_q8_0_block(row + t * bb, w + t * bw);
     }
@@ -369,3 +418,20 @@ int orc_unpack_q6k(const uint8_t *W, int64_t nsb, uint16_t *d, int8_t *scales, i
     }
     return ORC_OK;
 }
+
+/* Field view of IQ4_XS superblocks: d[s] (fp16 bits), ls[8s + j] (6-bit sub-block scales, the
+ * stored value: the multiplier is ls - 32), idx[256s + i] (codebook indices 0..15). */
+int orc_unpack_iq4xs(const uint8_t *W, int64_t nsb, uint16_t *d, uint8_t *ls, uint8_t *idx)
+{
+    if (!W || !d || !ls || !idx || nsb < 0) return ORC_EINVAL;
+    for (int64_t s = 0; s < nsb; ++s) {
+        const uint8_t *blk = W + s * 136;
+        d[s] = (uint16_t)(blk[0] | (blk[1] << 8));
+        for (int j = 0; j < 8; ++j) ls[8 * s + j] = (uint8_t)orc_iq4xs_scale(blk, j);
+        for (int i = 0; i < 256; ++i) idx[256 * s + i] = (uint8_t)orc_iq4xs_index(blk + 8, i);
+    }
+    return ORC_OK;
+}
+
+/* The codebook level of index v (0..15), for checking it against the format's printed table. */
+int orc_iq4_level(int v) { return (v >= 0 && v < 16) ? orc_iq4_levels[v] : 0; }

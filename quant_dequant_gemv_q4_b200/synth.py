@@ -20,6 +20,10 @@ weight's five bits once).
 Q6_K superblock bytes (210 per 256 weights): bytes 0-207 uniform random (uniform 6-bit q, stored
 q - 32 in -32..31, and uniform int8 scales per 16 weights), bytes 208-209 = fp16 d ~ U(1e-5, 2e-4).
 
+IQ4_XS superblock bytes (136 per 256 weights): bytes 0-1 = fp16 d ~ U(2e-5, 2e-4), bytes 2-135
+uniform random: uniform 6-bit sub-block scales (scales_h and scales_l hold each scale's six bits
+once) and uniform 4-bit codebook indices.
+
 Activations: x fp16 [K, B] with entries N(0, 1) drawn in fp64 and rounded once to fp16; for the
 "massive activation" FFN inputs each entry is independently, with probability 1e-3, multiplied by
 100 before that rounding.
@@ -37,9 +41,10 @@ Q8_0 = 8
 Q4_K = 12
 Q5_K = 13
 Q6_K = 14
+IQ4_XS = 23
 
-BLOCK_WEIGHTS = {Q4_K: 256, Q8_0: 32, Q5_K: 256, Q6_K: 256}
-BLOCK_BYTES = {Q4_K: 144, Q8_0: 34, Q5_K: 176, Q6_K: 210}
+BLOCK_WEIGHTS = {Q4_K: 256, Q8_0: 32, Q5_K: 256, Q6_K: 256, IQ4_XS: 256}
+BLOCK_BYTES = {Q4_K: 144, Q8_0: 34, Q5_K: 176, Q6_K: 210, IQ4_XS: 136}
 
 
 def _rng(seed: int, tensor_id: int, purpose: int) -> np.random.Generator:
@@ -103,6 +108,17 @@ def q6k_weights(N: int, K: int, seed: int, tensor_id: int = 0, d_range=(1e-5, 2e
     return blk.reshape(-1)
 
 
+def iq4xs_weights(N: int, K: int, seed: int, tensor_id: int = 0, d_range=(2e-5, 2e-4)) -> np.ndarray:
+    """Random IQ4_XS tensor [N, K] as raw bytes (uint8, N*K/256*136)."""
+    assert K % 256 == 0
+    g = _rng(seed, tensor_id, 0)
+    nsb = N * (K // 256)
+    blk = g.integers(0, 256, size=(nsb, 136), dtype=np.uint8)
+    d = g.uniform(d_range[0], d_range[1], size=nsb).astype(np.float16)
+    blk[:, 0:2] = d.view(np.uint8).reshape(nsb, 2)
+    return blk.reshape(-1)
+
+
 def weights(fmt: int, N: int, K: int, seed: int, tensor_id: int = 0) -> np.ndarray:
     if fmt == Q4_K:
         return q4k_weights(N, K, seed, tensor_id)
@@ -112,6 +128,8 @@ def weights(fmt: int, N: int, K: int, seed: int, tensor_id: int = 0) -> np.ndarr
         return q5k_weights(N, K, seed, tensor_id)
     if fmt == Q6_K:
         return q6k_weights(N, K, seed, tensor_id)
+    if fmt == IQ4_XS:
+        return iq4xs_weights(N, K, seed, tensor_id)
     raise ValueError(f"unknown format {fmt}")
 
 
@@ -191,4 +209,4 @@ WORKLOADS = {
         Gemv("q5k_ffn_gate_b8", Q5_K, 17408, 5120, 8, 0),
         Gemv("q6k_ffn_gate_b8", Q6_K, 17408, 5120, 8, 1))),
 }
-FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q6_K: "Q6_K", Q8_0: "Q8_0"}
+FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q6_K: "Q6_K", Q8_0: "Q8_0", IQ4_XS: "IQ4_XS"}

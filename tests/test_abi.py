@@ -285,7 +285,8 @@ def test_binding_constants_match_the_header():
             values[name] = int(val)
     for m in re.finditer(r"#define\s+(QG_\w+)\s+\((\d+)u\s*<<\s*(\d+)\)", src):
         values[m.group(1)] = int(m.group(2)) << int(m.group(3))
-    assert {"QG_FMT_Q4_K", "QG_VARIANT_TENSOR", "QG_ERR_SCRATCH", "QG_OK"} <= set(values)
+    assert {"QG_FMT_Q4_K", "QG_VARIANT_TENSOR", "QG_ERR_SCRATCH", "QG_OK",
+            "QG_NOALLOC_SCRATCH_BYTES"} <= set(values)
     for name, val in values.items():
         assert hasattr(qg, name), name
         assert getattr(qg, name) == val, (name, getattr(qg, name), val)

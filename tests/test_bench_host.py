@@ -73,7 +73,23 @@ def test_reference_arm_line():
                         "d2h_bytes_per_step": 0}
 
 
-def test_reference_arm_other_ranks_are_silent():
-    r = _run_bench(["--impl", "reference", "--steps", "1", "--ref-seconds", "1"],
-                   {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
-    assert r.returncode == 0 and r.stdout.strip() == ""
+def test_gpus_flag_launches_replica_ranks():
+    """--gpus 2 without a launcher starts two ranks under torch.distributed.run (rendezvous on
+    127.0.0.1; the reference arm joins a gloo group on every rank), and rank 0 alone prints."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl",
+                        "reference", "--steps", "1", "--warmup", "3", "--ref-seconds", "1"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+    assert d["config"] == bench.bench_config(2)
+
+
+def test_gpus_flag_must_match_the_launcher():
+    """Under a launcher, --gpus must equal WORLD_SIZE (no silent single-rank run)."""
+    r = _run_bench(["--gpus", "4", "--impl", "reference", "--steps", "1"],
+                   {"WORLD_SIZE": "2", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode == 2 and "WORLD_SIZE" in r.stderr

@@ -15,6 +15,7 @@ from conftest import read_golden
 from quant_dequant_gemv_q4_b200 import synth
 
 Q4_K, Q8_0 = 12, 8
+IQ4_XS = 23
 
 
 def _hexbytes(tokens):
@@ -232,12 +233,91 @@ def test_q8_0_exact_integer_case(orc):
 
 # --- the GEMV as a whole ------------------------------------------------------------------------
 
-@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14])
+def _numpy_dequant(W, fmt, N, K):
+    """An independent restatement of the block layouts in numpy (vectorized, written from the
+    format readings, sharing nothing with the oracle's C): the exact weight in fp64, rounded once
+    to fp32."""
+    W = np.asarray(W, np.uint8)
+    if fmt == Q8_0:
+        blk = W.reshape(-1, 34)
+        d = blk[:, 0:2].copy().view(np.float16).astype(np.float64)       # [nb, 1]
+        q = blk[:, 2:].view(np.int8).astype(np.float64)                  # [nb, 32]
+        return (d * q).astype(np.float32).reshape(N, K)
+    i = np.arange(256)
+    if fmt in (Q4_K, 13):
+        UB = 144 if fmt == Q4_K else 176
+        blk = W.reshape(-1, UB)
+        d = blk[:, 0:2].copy().view(np.float16).astype(np.float64)
+        dmin = blk[:, 2:4].copy().view(np.float16).astype(np.float64)
+        s = blk[:, 4:16].astype(np.int64)
+        sc = np.empty((blk.shape[0], 8), np.int64)
+        m = np.empty((blk.shape[0], 8), np.int64)
+        sc[:, :4], m[:, :4] = s[:, 0:4] & 63, s[:, 4:8] & 63
+        sc[:, 4:] = (s[:, 8:12] & 15) | ((s[:, 0:4] >> 6) << 4)
+        m[:, 4:] = (s[:, 8:12] >> 4) | ((s[:, 4:8] >> 6) << 4)
+        c, r = i // 64, i % 64
+        qs0 = 16 if fmt == Q4_K else 48
+        byte = blk[:, qs0 + 32 * c + r % 32].astype(np.int64)
+        q = np.where(r < 32, byte & 15, byte >> 4)
+        if fmt == 13:
+            hbit = (blk[:, 16 + r % 32].astype(np.int64) >> (2 * c + (r >= 32))) & 1
+            q = q + 16 * hbit
+        j = i // 32
+        w = d * sc[:, j] * q - dmin * m[:, j]
+        return w.astype(np.float32).reshape(N, K)
+    if fmt == IQ4_XS:
+        levels = np.array([-127, -104, -83, -65, -49, -35, -22, -10,
+                           1, 13, 25, 38, 53, 69, 89, 113], np.float64)
+        blk = W.reshape(-1, 136)
+        d = blk[:, 0:2].copy().view(np.float16).astype(np.float64)
+        sh = blk[:, 2].astype(np.int64) | (blk[:, 3].astype(np.int64) << 8)
+        jj = np.arange(8)
+        ls = ((blk[:, 4 + jj // 2].astype(np.int64) >> (4 * (jj % 2))) & 15) | \
+            (((sh[:, None] >> (2 * jj)) & 3) << 4)
+        j, r = i // 32, i % 32
+        byte = blk[:, 8 + 16 * j + r % 16].astype(np.int64)
+        idx = np.where(r < 16, byte & 15, byte >> 4)
+        w = d * (ls[:, j] - 32) * levels[idx]
+        return w.astype(np.float32).reshape(N, K)
+    # Q6_K
+    blk = W.reshape(-1, 210)
+    h, r = i // 128, i % 128
+    t, l = r // 32, r % 32
+    ql = blk[:, 64 * h + l + 32 * (t % 2)].astype(np.int64)
+    lo = np.where(t < 2, ql & 15, ql >> 4)
+    hi = (blk[:, 128 + 32 * h + l].astype(np.int64) >> (2 * t)) & 3
+    q = lo | (hi << 4)
+    sc = blk[:, 192:208].view(np.int8).astype(np.float64)
+    d = blk[:, 208:210].copy().view(np.float16).astype(np.float64)
+    w = d * sc[:, i // 16] * (q - 32)
+    return w.astype(np.float32).reshape(N, K)
+
+
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14, IQ4_XS])
+def test_dequant_matches_independent_numpy_unpack(orc, fmt):
+    """The oracle's unpack + dequant equals the numpy restatement bit for bit on random bytes
+    (every field uniform: sign, exponent and mantissa of d/dmin included)."""
+    N, K = 6, 2048
+    rng = np.random.default_rng(100 + fmt)
+    W = rng.integers(0, 256, size=orc.weight_bytes(fmt, N, K), dtype=np.uint8)
+    # keep d and dmin finite (an fp16 inf/NaN propagates differently in any two codes)
+    UB = {Q4_K: 144, 13: 176, 14: 210, Q8_0: 34, IQ4_XS: 136}[fmt]
+    blk = W.reshape(-1, UB)
+    for off in ([208] if fmt == 14 else [0, 2] if fmt in (Q4_K, 13) else [0]):
+        blk[:, off + 1] &= 0x7B  # exponent < 31
+    got = orc.dequant(W, fmt, N, K)
+    want = _numpy_dequant(W, fmt, N, K)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32)) or \
+        np.array_equal(got, want)  # +0 / -0 from d < 0 (see the signed-zero reading)
+
+
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14, IQ4_XS])
 @pytest.mark.parametrize("N,K", [(1, 256), (2, 512), (3, 256), (3, 512)])
 def test_brute_force_tiny(orc, fmt, N, K):
-    """Oracle y and A equal a numpy fp64 matmul of the dequantized matrix, for B = 1..8."""
+    """Oracle y and A equal a numpy fp64 matmul of the matrix dequantized by the independent
+    numpy unpack, for B = 1..8."""
     W = synth.weights(fmt, N, K, seed=N * 1000 + K)
-    Wf = orc.dequant(W, fmt, N, K).astype(np.float64)
+    Wf = _numpy_dequant(W, fmt, N, K).astype(np.float64)
     for B in range(1, 9):
         x = synth.activations(K, B, seed=B)
         y, A = orc.gemv(W, fmt, N, K, x, B)
@@ -256,7 +336,7 @@ def test_rows_subset_matches_full(orc):
     assert np.array_equal(ys, y[rows]) and np.array_equal(As, A[rows])
 
 
-@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14])
+@pytest.mark.parametrize("fmt", [Q4_K, Q8_0, 13, 14, IQ4_XS])
 def test_linearity(orc, fmt):
     """y(2x) = 2 y(x) and y(x/8) = y(x)/8 exactly (power-of-two scalings are exact in fp16 for
     these magnitudes); y(x1) + y(x2) = y(x1 + x2) for x1, x2 with disjoint supports."""
@@ -436,3 +516,92 @@ def test_q6k_exact_integer_case(orc):
     y, _ = orc.gemv(W.reshape(-1), Q6_K, N, K, x, B)
     q = orc.unpack_q6k(W.reshape(-1), W.shape[0])["q"].astype(np.int64).reshape(N, K)
     assert np.array_equal(y, (q @ x.astype(np.int64)).astype(np.float64))
+
+
+# ------------------------------------------------------------------------------------------------
+# IQ4_XS (named by the T4 dossier's second prompt, "SPEC" and "OUTPUT"; layout: the reading in
+# tests/golden/iq4xs_superblock.txt)
+# ------------------------------------------------------------------------------------------------
+
+def _iq4xs_golden_block():
+    g = read_golden("iq4xs_superblock.txt")
+    blk = np.zeros(136, np.uint8)
+    d = int(g["d"][0][0], 16)
+    sh = int(g["scales_h"][0][0], 16)
+    blk[0:2] = [d & 0xFF, d >> 8]
+    blk[2:4] = [sh & 0xFF, sh >> 8]
+    blk[4:8] = [int(v, 16) for v in g["scales_l"][0]]
+    blk[8:136] = np.arange(128, dtype=np.uint8)
+    return blk, g
+
+
+def test_iq4xs_codebook_is_the_formats(orc):
+    g = read_golden("iq4xs_superblock.txt")
+    assert [orc.iq4_level(v) for v in range(16)] == [int(v) for v in g["level"][0]]
+
+
+def test_iq4xs_superblock_golden(orc):
+    blk, g = _iq4xs_golden_block()
+    f = orc.unpack_iq4xs(blk, 1)
+    assert f["ls"][0].tolist() == [int(v) for v in g["ls"][0]]
+    w = orc.dequant(blk, IQ4_XS, 1, 256)[0]
+    for i, v in g["w"]:
+        assert w[int(i)] == np.float32(float(v)), i
+    # d = 0.5 halves every weight (exact)
+    blk[0:2] = [0x00, 0x38]
+    assert np.array_equal(orc.dequant(blk, IQ4_XS, 1, 256)[0], w / 2)
+
+
+def test_iq4xs_each_scale_bit_moves_one_sub_block(orc):
+    """Setting scale bit k of sub-block j adds 2^k to ls_j: exactly the 32 weights of sub-block j
+    change, each by d * 2^k * level.  Bits 0-3 of ls_j are nibble j % 2 of scales_l[j // 2], bits 4-5
+    are bits 2j, 2j+1 of scales_h."""
+    blk, _ = _iq4xs_golden_block()
+    blk[2:8] = 0
+    base = orc.dequant(blk, IQ4_XS, 1, 256)[0].astype(np.float64)
+    lev = np.array([orc.iq4_level(v) for v in range(16)], np.float64)
+    idx = orc.unpack_iq4xs(blk, 1)["idx"][0].astype(np.int64)
+    for j in range(8):
+        for k in range(6):
+            b2 = blk.copy()
+            if k < 4:
+                b2[4 + j // 2] |= 1 << (k + 4 * (j % 2))
+            else:
+                bit = 2 * j + (k - 4)
+                b2[2 + bit // 8] |= 1 << (bit % 8)
+            diff = orc.dequant(b2, IQ4_XS, 1, 256)[0].astype(np.float64) - base
+            want = np.zeros(256)
+            want[32 * j:32 * j + 32] = (2 ** k) * lev[idx[32 * j:32 * j + 32]]
+            assert np.array_equal(diff, want), (j, k)
+
+
+def test_iq4xs_each_nibble_is_one_weight(orc):
+    """Nibble h of qs[16j + l] holds weight 32j + 16h + l: changing it changes that weight only."""
+    blk, _ = _iq4xs_golden_block()
+    blk[2:4] = 0
+    blk[4:8] = 0x11  # every ls_j = 1: multiplier -31, no zero sub-block
+    blk[8:136] = 0x88  # every index 8 (level 1)
+    base = orc.dequant(blk, IQ4_XS, 1, 256)[0]
+    for j in (0, 3, 7):
+        for l in (0, 9, 15):
+            for h in (0, 1):
+                b2 = blk.copy()
+                b2[8 + 16 * j + l] = (0x8F if h == 0 else 0xF8)  # one nibble -> index 15
+                w = orc.dequant(b2, IQ4_XS, 1, 256)[0]
+                changed = np.nonzero(w != base)[0].tolist()
+                assert changed == [32 * j + 16 * h + l], (j, l, h)
+
+
+def test_iq4xs_exact_integer_case(orc):
+    """d = 1 and integer x: w = (ls - 32) * level is an integer, so y is an exact integer sum."""
+    rng = np.random.default_rng(23)
+    N, K, B = 3, 1024, 2
+    W = synth.iq4xs_weights(N, K, seed=23).reshape(-1, 136).copy()
+    W[:, 0:2] = np.array([0x00, 0x3C], np.uint8)
+    x = rng.integers(-8, 9, size=(K, B)).astype(np.float16)
+    y, _ = orc.gemv(W.reshape(-1), IQ4_XS, N, K, x, B)
+    f = orc.unpack_iq4xs(W.reshape(-1), W.shape[0])
+    lev = np.array([orc.iq4_level(v) for v in range(16)], np.int64)
+    wint = ((f["ls"].astype(np.int64) - 32).repeat(32, axis=1) * lev[f["idx"].astype(np.int64)])
+    wint = wint.reshape(N, K)
+    assert np.array_equal(y, (wint @ x.astype(np.int64)).astype(np.float64))
