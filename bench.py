@@ -231,8 +231,14 @@ class CallSet:
 
 
 def time_callset(cs: CallSet, steps: int, warmup: int, variant: int, clocks: ClockSampler | None):
-    """Time exactly `steps` steps (each: the call list on the next weight copy) replayed from CUDA
-    graphs; returns (seconds on this rank, per-step ms, kernels per step)."""
+    """Time exactly `steps` steps (each: the call list on the next weight copy) from one CUDA
+    graph; returns (seconds on this rank, ms per step).
+
+    The graph holds `lead` untimed calls, the start event, the `steps` timed calls and the end
+    event (event-record nodes, cudaEventRecordExternal), so the timed region opens while the GPU
+    is already streaming: neither the graph's launch nor its upload (done by the warm-up replays,
+    which run the whole graph) falls inside it, and every timed call is a steady-state call on a
+    fresh weight copy."""
     import torch
     stream = torch.cuda.Stream(device=cs.device)
     R = cs.copies
@@ -240,39 +246,34 @@ def time_callset(cs: CallSet, steps: int, warmup: int, variant: int, clocks: Clo
         for r in range(min(R, 2)):
             cs.launch(r, stream, variant)  # allocates the workspace of this stream
     stream.synchronize()
-    g_full = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_full, stream=stream):
-        for r in range(R):
-            cs.launch(r, stream, variant)
-    rem = steps % R
-    g_rem = None
-    if rem:
-        g_rem = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_rem, stream=stream):
-            for r in range(rem):
-                cs.launch(r, stream, variant)
+    lead = max(R, 8)
+    start = torch.cuda.Event(enable_timing=True, external=True)
+    end = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(lead):
+            cs.launch(i % R, stream, variant)
+        start.record(stream)
+        for i in range(steps):
+            cs.launch((lead + i) % R, stream, variant)
+        end.record(stream)
+    # warm-up: whole-graph replays until at least `warmup` steps have run (at least one replay,
+    # which uploads the graph)
     with torch.cuda.stream(stream):
-        for _ in range(max(1, -(-warmup // R))):
-            g_full.replay()
+        for _ in range(max(1, -(-warmup // (lead + steps)))):
+            graph.replay()
     stream.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     ctx = clocks if clocks is not None else _null()
     with ctx:
         barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            start.record(stream)
-            for _ in range(steps // R):
-                g_full.replay()
-            if g_rem is not None:
-                g_rem.replay()
-            end.record(stream)
-        end.synchronize()
+            graph.replay()
+        stream.synchronize()
         torch.cuda.synchronize()
         barrier()
     secs = start.elapsed_time(end) / 1e3
-    del g_full, g_rem
+    del graph
     return secs, secs * 1e3 / steps
 
 
@@ -442,6 +443,14 @@ def oracle_sample_rate(call: synth.Gemv, seed: int, seconds: float):
 
 def run_reference(args):
     world, rank, _ = dist_env()
+    if world > 1:
+        # every rank joins the launcher's rendezvous once (gloo: no GPU work on this arm); rank 0
+        # alone then times the oracle and prints
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("gloo", timeout=timedelta(seconds=300))
+        dist.barrier()
+        dist.destroy_process_group()
     if rank != 0:
         return 0
     import oracle
@@ -518,6 +527,22 @@ def run_ncu_case(args):
     return 0
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_replicas(n: int, argv: list[str]) -> int:
+    """Run this script as n local ranks under torch.distributed.run (rendezvous on 127.0.0.1);
+    returns the launcher's exit code.  Rank 0 prints the JSON line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 # ------------------------------------------------------------------------------------------------
 def main(argv=None):
     ap = argparse.ArgumentParser()
@@ -539,6 +564,15 @@ def main(argv=None):
                     help="--ncu-case format: 12 Q4_K (default), 13 Q5_K, 14 Q6_K")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+
+    # --gpus N > 1 started without a launcher: run N replica processes under torch.distributed.run
+    # (one per GPU), each with these same arguments
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_replicas(args.gpus, sys.argv[1:] if argv is None else list(argv))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        return 2
 
     if args.impl == "reference":
         return run_reference(args)

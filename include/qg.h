@@ -27,6 +27,12 @@
  *                bits are bits 2t, 2t+1 of qh[32h + l]; w = d*scales[i/16]*(q - 32), q in 0..63.
  *                (The T4 dossier's "QUANTIZATION MIX" lists Q5_K and Q6_K next to Q4_K.)
  *   QG_FMT_Q8_0: 32 weights in 34 bytes {fp16 d; i8 qs[32]}, w = d*q.
+ *   QG_FMT_IQ4_XS: 256 weights in 136 bytes {fp16 d; u16 scales_h; u8 scales_l[4]; u8 qs[128]}
+ *                (named by the same dossier's second prompt, "SPEC").  Sub-block j = i/32 has the
+ *                6-bit scale ls_j = nibble (j%2) of scales_l[j/2] + 16 * bits 2j..2j+1 of
+ *                scales_h; weight i's 4-bit index is the low (r < 16) or high (r >= 16) nibble of
+ *                qs[16j + r%16], r = i%32; w = d*(ls_j - 32)*level[index] with the format's
+ *                non-linear levels {-127,-104,-83,-65,-49,-35,-22,-10,1,13,25,38,53,69,89,113}.
  *   The flag values are GGML's type ids.
  *
  * Layouts: W row-major, row n = K/256 consecutive superblocks (K-quants) or K/32 consecutive
@@ -34,9 +40,12 @@
  * their transpose.
  *
  * Ownership: every pointer is the caller's; the library never frees caller memory.  The library
- * owns one small workspace per (device, stream) for split rows (partial sums, arrival counters,
- * an error word), allocated with cudaMalloc the first time a stream needs one of that size and
- * kept until process exit.  Make the first call on a stream outside CUDA-graph capture.
+ * owns one small workspace per (device, stream handle) for split rows (partial sums, arrival
+ * counters, an error word), allocated with cudaMalloc the first time a stream needs one of that
+ * size and kept until process exit: it is not released when the stream is destroyed, and a new
+ * stream that happens to get a destroyed stream's handle reuses that workspace (safe, since the
+ * calls on one stream are ordered).  qg_gemv_host's x/y scratch follows the same rule.  Make the
+ * first call on a stream outside CUDA-graph capture.
  *
  * Errors: every call returns a qg_status.  Argument errors are found on the host before anything
  * is enqueued.  Launch errors return QG_ERR_CUDA.  Faults of the asynchronous work surface at the
@@ -60,7 +69,7 @@ extern "C" {
 #endif
 
 /* Block formats (GGML type ids). */
-enum { QG_FMT_Q8_0 = 8, QG_FMT_Q4_K = 12, QG_FMT_Q5_K = 13, QG_FMT_Q6_K = 14 };
+enum { QG_FMT_Q8_0 = 8, QG_FMT_Q4_K = 12, QG_FMT_Q5_K = 13, QG_FMT_Q6_K = 14, QG_FMT_IQ4_XS = 23 };
 
 /* Status codes. */
 enum {
@@ -72,15 +81,15 @@ enum {
     QG_ERR_ALIGN = 5,   /* W not 16-byte aligned, x not 2-byte aligned or y not 4-byte aligned */
     QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
     QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
-    QG_ERR_RANGE = 8,   /* a packer field is out of range (sc, m > 63; q above 15 / 31 / 63 for
-                           Q4_K / Q5_K / Q6_K; Q8_0 q = -128) */
+    QG_ERR_RANGE = 8,   /* a packer field is out of range (sc, m > 63; q above 15 / 31 / 63 / 15
+                           for Q4_K / Q5_K / Q6_K / IQ4_XS; Q8_0 q = -128) */
     QG_ERR_VARIANT = 9, /* unknown kernel variant, or a variant that does not take this format */
     QG_ERR_SCRATCH = 10 /* qg_gemv_noalloc: the call needs more scratch than its fixed array holds */
 };
 
 /* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses: when
- * K % 256 == 0, TENSOR for the K-quants with B >= 2 and FACTORED otherwise; GENERIC when
- * K % 256 != 0. */
+ * K % 256 == 0, TENSOR for the K-quants (Q4_K, Q5_K, Q6_K) with B >= 2 and FACTORED otherwise;
+ * GENERIC when K % 256 != 0. */
 enum {
     QG_VARIANT_AUTO = 0,
     /* Each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m) (Q4_K; the
@@ -93,10 +102,14 @@ enum {
      * d*sc*q and dmin*m nearly cancel.  Q6_K: per 16-weight group,
      * y = sum_t (d*sc_t)*(sum(q*x) - 32*sum(x)), the same kind of bound with 32*|d*sc*x| in place
      * of |dmin*m*x|.  Q8_0: the block scale d is applied per 32 weights (error relative to
-     * sum|w*x|).  Requires K % 256 == 0. */
+     * sum|w*x|).  IQ4_XS: per 32-weight sub-block, y = sum_j d*(ls_j - 32)*(sum(u*x) - 128*sum(x))
+     * with u = level + 128 (1..241), the same kind of bound with (|level| + 128)*|x| in place of
+     * |level*x|.  Requires K % 256 == 0. */
     QG_VARIANT_FACTORED = 2,
     /* Any format and shape: one warp per row, plain loads, no shared-memory staging.  Used by
-     * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0). */
+     * AUTO for Q8_0 tensors whose rows are not 16-byte multiples (K % 256 != 0).  IQ4_XS weights
+     * are exact in fp32, so FACTORED's offset form (see below) and GENERIC differ only in their
+     * summation. */
     QG_VARIANT_GENERIC = 3,
     /* The K-quants (Q4_K, Q5_K, Q6_K): the FACTORED arithmetic with the q*x products on the
      * tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the
@@ -111,7 +124,7 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
 
 /* y = dequant(W) . x on the device.
  *   W      device, qg_weight_bytes(fmt, N, K) bytes, 16-byte aligned, read only
- *   fmt    QG_FMT_Q4_K, QG_FMT_Q5_K, QG_FMT_Q6_K or QG_FMT_Q8_0
+ *   fmt    QG_FMT_Q4_K, QG_FMT_Q5_K, QG_FMT_Q6_K, QG_FMT_IQ4_XS or QG_FMT_Q8_0
  *   N, K   rows and reduction length; N >= 0 (N == 0 does nothing); K >= 1, K % block == 0
  *   x      device, fp16 bits [K][B], 2-byte aligned, read only
  *   B      number of columns: 1..8; 1..16 for Q4_K with K % 256 == 0 (9..16 columns run on the
@@ -126,8 +139,10 @@ int qg_gemv(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int
  * x_host into library-owned device scratch, the GEMV (the default kernel variant) and the copy
  * of y back to y_host, so one call does what a host-side caller would otherwise do in three.
  *   W        device, as for qg_gemv (weights stay resident on the GPU)
- *   x_host   host, fp16 bits [K][B], 2-byte aligned; read by the copy engine when the stream
- *            reaches the call
+ *   x_host   host, fp16 bits [K][B], 2-byte aligned; filled by the host before the call.  With
+ *            a pinned buffer it may be read while the kernel queued just before the call on the
+ *            stream is still finishing (the copy overlaps that kernel's tail), so x_host must not
+ *            be written by device work queued on the stream before the call
  *   y_host   host, fp32 [N][B], 4-byte aligned; valid after the stream has been synchronized
  *   fmt, N, K, B, stream as for qg_gemv.
  * With page-locked (pinned) host buffers nothing is copied by a separate operation: a small
@@ -184,6 +199,8 @@ int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, voi
  *   Q6_K: d[N*K/256] fp16 bits; sc = the int8 group scales [N*K/16] (two's-complement bytes);
  *         dmin and m are ignored; q = uint8 [N*K] stored values 0..63 (w = d*sc*(q - 32)).
  *   Q8_0: d[N*K/32] fp16 bits; dmin, sc, m are ignored; q = int8 [N*K] in -127..127.
+ *   IQ4_XS: d[N*K/256] fp16 bits; sc = the stored 6-bit sub-block scales ls [N*K/32] (<= 63; the
+ *         multiplier is ls - 32); dmin and m are ignored; q = uint8 [N*K] codebook indices 0..15.
  *   out   host, qg_weight_bytes(fmt, N, K) bytes.
  * All pointers are host pointers.  QG_ERR_RANGE if a field is out of range (out is then
  * unspecified). */
@@ -233,12 +250,12 @@ int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
 
 /* qg_gemv without any allocation.  The pages have no counterpart of this entry point; it exists
  * for callers that cannot let a library call cudaMalloc: a host framework or plugin interface
- * that owns all device memory through its own pool, a decode loop that cannot afford the
- * device-wide synchronization an allocation may cause, or code recorded into a CUDA graph (an
- * allocation during capture is an error).  The caller passes inputs and outputs exactly as for
- * qg_gemv (same arguments, layouts, preconditions and results, default kernel variant); the
- * kernel's scratch (an error word, one arrival counter per row band when K is split, the split-K
- * partial rows) lives in one file-scope device array of QG_NOALLOC_SCRATCH_BYTES per GPU.
+ * that owns all device memory through its own pool, or a decode loop that cannot afford the
+ * device-wide synchronization an allocation may cause.  The caller passes inputs and outputs
+ * exactly as for qg_gemv (same arguments, layouts, preconditions and results, default kernel
+ * variant); the kernel's scratch (an error word, one arrival counter per row band when K is
+ * split, the split-K partial rows) lives in one file-scope device array of
+ * QG_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that loads the library holds until exit.
  *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library routine.  The counters
  *     start at zero (the array is zero-initialized) and every call leaves them at zero again (the
  *     last CTA of a band resets its counter); the partial rows are written before they are read.
@@ -250,10 +267,18 @@ int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
  *   - QG_ERR_SCRATCH if the call needs more scratch than the array holds (this happens only when
  *     x for the whole of K does not fit in shared memory and N*B is large: the split-K partial
  *     rows need S*N*B*4 bytes); nothing is enqueued then.
- *   - Device-side copy timeouts are not reported by this entry point (qg_device_error reads the
- *     allocating path's workspaces only). */
+ *   - qg_last_variant / qg_last_splits report its launch like qg_gemv's.
+ *   - Device-side copy timeouts go to the array's error word: read them with
+ *     qg_noalloc_device_error (qg_device_error reads the allocating entry points' workspaces). */
 int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B,
                     float *y, void *stream);
+
+/* Reads and clears the error word of qg_gemv_noalloc's fixed array on the current device, after
+ * synchronizing `stream` (the stream of the calls to check; NULL = the legacy default stream).
+ * *flag = 0 if no device-side timeout happened (or no qg_gemv_noalloc call has run on this
+ * device), else a nonzero code; a nonzero word also clears the array's band counters.  No
+ * counterpart on the pages; it allocates nothing (plain copies to and from the array). */
+int qg_noalloc_device_error(void *stream, int *flag);
 
 /* Static text for a status code. */
 const char *qg_status_string(int status);

@@ -19,6 +19,7 @@ QG_FMT_Q8_0 = 8
 QG_FMT_Q4_K = 12
 QG_FMT_Q5_K = 13
 QG_FMT_Q6_K = 14
+QG_FMT_IQ4_XS = 23
 
 QG_VARIANT_AUTO = 0
 QG_VARIANT_DIRECT = 1
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.qg_plan.restype = I
         L.qg_device_error.argtypes = [P, ctypes.POINTER(I)]
         L.qg_device_error.restype = I
+        L.qg_noalloc_device_error.argtypes = [P, ctypes.POINTER(I)]
+        L.qg_noalloc_device_error.restype = I
         L.qg_hbm_copy.argtypes = [P, P, SZ, P]
         L.qg_hbm_copy.restype = I
         L.qg_hbm_read.argtypes = [P, SZ, P, P]
@@ -181,7 +184,8 @@ def qg_dequant_f32(W, fmt: int, N: int, K: int, out, stream=None) -> None:
 
 def qg_pack_reference(fmt: int, N: int, K: int, d, dmin, sc, m, q) -> np.ndarray:
     """Host bit packer: fields (numpy) -> uint8 tensor bytes (Q6_K: sc are the int8 group scales,
-    q the stored values 0..63; dmin, m unused)."""
+    q the stored values 0..63; IQ4_XS: sc are the stored 6-bit sub-block scales, q the codebook
+    indices; dmin, m unused for both)."""
     out = np.empty(qg_weight_bytes(fmt, N, K), dtype=np.uint8)
     d = np.ascontiguousarray(d, dtype=np.uint16)
     args = [d]
@@ -193,6 +197,10 @@ def qg_pack_reference(fmt: int, N: int, K: int, d, dmin, sc, m, q) -> np.ndarray
     elif fmt == QG_FMT_Q6_K:
         dmin = m = None
         sc = np.ascontiguousarray(np.asarray(sc).astype(np.int8).view(np.uint8))
+        q = np.ascontiguousarray(q, dtype=np.uint8)
+    elif fmt == QG_FMT_IQ4_XS:
+        dmin = m = None
+        sc = np.ascontiguousarray(sc, dtype=np.uint8)
         q = np.ascontiguousarray(q, dtype=np.uint8)
     else:
         dmin = sc = m = None
@@ -225,6 +233,14 @@ def qg_plan(fmt: int, N: int, K: int, B: int, variant: int = 0, mats: int = 1, s
 def qg_device_error(stream=None) -> int:
     flag = ctypes.c_int(0)
     _ok(lib().qg_device_error(_stream(stream), ctypes.byref(flag)), "qg_device_error")
+    return flag.value
+
+
+def qg_noalloc_device_error(stream=None) -> int:
+    """Reads and clears the error word of qg_gemv_noalloc's fixed array (0: no timeout)."""
+    flag = ctypes.c_int(0)
+    _ok(lib().qg_noalloc_device_error(_stream(stream), ctypes.byref(flag)),
+        "qg_noalloc_device_error")
     return flag.value
 
 

@@ -244,6 +244,10 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         groups_per_unit = RowsFmt<kFmtQ6_K>::kGroups;
         NW = BP >= 4 ? RowsWarps<kFmtQ6_K, 4>::value : RowsWarps<kFmtQ6_K, 1>::value;
         break;
+    case kFmtIQ4_XS:
+        LB = RowsFmt<kFmtIQ4_XS>::kLaneBytes;
+        NW = BP >= 8 ? RowsWarps<kFmtIQ4_XS, 8>::value : RowsWarps<kFmtIQ4_XS, 1>::value;
+        break;
     default:
         LB = RowsFmt<kFmtQ8_0>::kLaneBytes;
         NW = BP >= 4 ? RowsWarps<kFmtQ8_0, 4>::value : RowsWarps<kFmtQ8_0, 1>::value;
@@ -276,7 +280,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     // The tensor-core kernel only takes slicings with at most one pair per warp.  If no slicing
     // qualifies, the one with the most busy lanes.
     const int UB = tensor ? (fmt == kFmtQ5_K ? 176 : fmt == kFmtQ6_K ? 210 : 144)
-                          : (fmt == kFmtQ6_K ? 210 : LB);
+                          : (fmt == kFmtQ6_K ? 210 : fmt == kFmtIQ4_XS ? 136 : LB);
     double best_cost = 1e300;
     int64_t best_steps = INT64_MAX;
     RowsPlan util_best{};
@@ -357,6 +361,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_ROWS_Q5K2(bp) rows_gemv_kernel<kFmtQ5_K, bp, 2>
 #define QG_ROWS_Q6K1(bp) rows_gemv_kernel<kFmtQ6_K, bp, 1>
 #define QG_ROWS_Q6K2(bp) rows_gemv_kernel<kFmtQ6_K, bp, 2>
+#define QG_ROWS_IQ41(bp) rows_gemv_kernel<kFmtIQ4_XS, bp, 1>
+#define QG_ROWS_IQ42(bp) rows_gemv_kernel<kFmtIQ4_XS, bp, 2>
     if (tensor && fmt == kFmtQ5_K) {
         if (mats == 2) { QG_BP_SWITCH(QG_MMA5K2) }
         QG_BP_SWITCH(QG_MMA5K1)
@@ -381,8 +387,14 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
         if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q6K2) }
         QG_BP_SWITCH(QG_ROWS_Q6K1)
     }
+    if (fmt == kFmtIQ4_XS) {
+        if (mats == 2) { QG_BP_SWITCH(QG_ROWS_IQ42) }
+        QG_BP_SWITCH(QG_ROWS_IQ41)
+    }
     if (mats == 2) { QG_BP_SWITCH(QG_ROWS_Q4K2) }
     QG_BP_SWITCH(QG_ROWS_Q4K1)
+#undef QG_ROWS_IQ42
+#undef QG_ROWS_IQ41
 #undef QG_ROWS_Q6K2
 #undef QG_ROWS_Q6K1
 #undef QG_ROWS_Q5K2
@@ -449,7 +461,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     static_assert(offsetof(WeightMaps<2>, m) == 0 && sizeof(WeightMaps<1>) == sizeof(CUtensorMap),
                   "WeightMaps<1> is a prefix of WeightMaps<2>");
     std::memset(&maps, 0, sizeof(maps));
-    const bool per_lane = (fmt == kFmtQ6_K);  // rows not 16-byte multiples: no tensor map
+    const bool per_lane = (fmt == kFmtQ6_K || fmt == kFmtIQ4_XS);  // units not 16-byte aligned: no tensor map
     if (!per_lane) {
         if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
         if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
@@ -492,7 +504,8 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
 
 int check_common(const void *W, int fmt, int64_t N, int64_t K)
 {
-    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K && fmt != QG_FMT_Q8_0)
+    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K && fmt != QG_FMT_Q8_0 &&
+        fmt != QG_FMT_IQ4_XS)
         return QG_ERR_FMT;
     const int64_t bw = (fmt == QG_FMT_Q8_0) ? 32 : 256;
     if (N < 0 || K < 1 || K % bw != 0) return QG_ERR_SHAPE;
@@ -512,6 +525,7 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
     case kFmtQ4_K: rowwise_gemv_kernel<kFmtQ4_K><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
     case kFmtQ5_K: rowwise_gemv_kernel<kFmtQ5_K><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
     case kFmtQ6_K: rowwise_gemv_kernel<kFmtQ6_K><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
+    case kFmtIQ4_XS: rowwise_gemv_kernel<kFmtIQ4_XS><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
     default: rowwise_gemv_kernel<kFmtQ8_0><<<(unsigned)blocks, threads, 0, st>>>(w, N, K, x, B, y); break;
     }
     return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
@@ -524,7 +538,8 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
 int auto_variant(int fmt, int64_t K, int B)
 {
     if (K % 256 != 0) return QG_VARIANT_GENERIC;
-    return (fmt != QG_FMT_Q8_0 && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
+    const bool has_tensor = (fmt == QG_FMT_Q4_K || fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K);
+    return (has_tensor && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
 }
 
 // The kernel variant a GEMV call runs (QG_VARIANT_AUTO resolved), or the argument error.
@@ -536,7 +551,7 @@ int resolve_variant(int fmt, int64_t K, int B, int variant, int *var_out)
     int var = variant;
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
-    if (var == QG_VARIANT_TENSOR && fmt == QG_FMT_Q8_0) return QG_ERR_VARIANT;
+    if (var == QG_VARIANT_TENSOR && (fmt == QG_FMT_Q8_0 || fmt == QG_FMT_IQ4_XS)) return QG_ERR_VARIANT;
     if (B > 8 && fmt != QG_FMT_Q4_K) return QG_ERR_BATCH;  // 9..16 columns: the Q4_K kernel only
     if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
@@ -847,14 +862,17 @@ int qg_dequant_f32(const void *W, int fmt, int64_t N, int64_t K, float *out, voi
         const int64_t threads = nsb * 4;
         dequant_q4k_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
             static_cast<const uint8_t *>(W), nsb, out);
-    } else if (fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K) {
+    } else if (fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K || fmt == QG_FMT_IQ4_XS) {
         const int64_t nsb = N * (K / 256);
         const int64_t threads = nsb * 16;
         const unsigned grid = (unsigned)((threads + 255) / 256);
+        const uint8_t *w = static_cast<const uint8_t *>(W);
         if (fmt == QG_FMT_Q5_K)
-            dequant_kq_kernel<kFmtQ5_K><<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(W), nsb, out);
+            dequant_kq_kernel<kFmtQ5_K><<<grid, 256, 0, st>>>(w, nsb, out);
+        else if (fmt == QG_FMT_Q6_K)
+            dequant_kq_kernel<kFmtQ6_K><<<grid, 256, 0, st>>>(w, nsb, out);
         else
-            dequant_kq_kernel<kFmtQ6_K><<<grid, 256, 0, st>>>(static_cast<const uint8_t *>(W), nsb, out);
+            dequant_kq_kernel<kFmtIQ4_XS><<<grid, 256, 0, st>>>(w, nsb, out);
     } else {
         const int64_t nblk = N * (K / 32);
         dequant_q8_0_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(
@@ -871,7 +889,8 @@ int qg_plan(int fmt, int64_t N, int64_t K, int B, int variant, int mats, int sms
             int64_t *out)
 {
     if (!out) return QG_ERR_NULL;
-    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K && fmt != QG_FMT_Q8_0)
+    if (fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K && fmt != QG_FMT_Q8_0 &&
+        fmt != QG_FMT_IQ4_XS)
         return QG_ERR_FMT;
     const int64_t bw = (fmt == QG_FMT_Q8_0) ? 32 : 256;
     if (N < 1 || K < 1 || K % bw != 0 || (mats != 1 && mats != 2)) return QG_ERR_SHAPE;
@@ -990,11 +1009,11 @@ const char *qg_status_string(int status)
 
 // ---------------------------------------------------------------------------------------------
 // Allocation-free entry point.  Some callers cannot let a library call cudaMalloc: a host
-// framework or plugin interface that owns every device allocation through its own pool, a
-// decode loop that cannot afford the device-wide synchronization cudaMalloc may cause, code
-// recorded into a CUDA graph (allocating during capture is an error).  qg_gemv_noalloc runs
-// the same streaming kernel with its scratch (arrival counters, split-row partial sums, split-K
-// partial rows) in the fixed file-scope device array below instead of a cudaMalloc'd workspace.
+// framework or plugin interface that owns every device allocation through its own pool, or a
+// decode loop that cannot afford the device-wide synchronization cudaMalloc may cause.
+// qg_gemv_noalloc runs the same streaming kernel with its scratch (error word, arrival counters,
+// split-K partial rows) in the fixed file-scope device array below instead of a cudaMalloc'd
+// workspace.
 // ---------------------------------------------------------------------------------------------
 namespace {
 
@@ -1043,12 +1062,20 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (var == QG_VARIANT_GENERIC) return launch_rowwise(W, fmt, N, K, x, B, y, st, di);  // no scratch
+    if (var == QG_VARIANT_GENERIC) {  // no scratch
+        rc = launch_rowwise(W, fmt, N, K, x, B, y, st, di);
+        if (rc == QG_OK) {
+            t_last_variant = QG_VARIANT_GENERIC;
+            t_last_splits = 1;
+        }
+        return rc;
+    }
 
     const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
-    // one fixed layout for every call: kNoallocCounters band counters, then the partial rows
+    // one fixed layout for every call: the error word, kNoallocCounters band counters, then the
+    // partial rows
     const size_t ncnt = kNoallocCounters;
     if ((size_t)p.Gs > kNoallocCounters) return QG_ERR_SCRATCH;
     if (ws_bytes_for(ncnt, 0, part_f) > QG_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH;
@@ -1065,5 +1092,34 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     if ((rc = launch_rows(W, fmt, N, K, x, B, y, st, di, dev, p, ws.err, ws.cnt, ws.part, false)) !=
         QG_OK)
         return rc;
+    t_last_variant = var;
+    t_last_splits = p.S;
+    return QG_OK;
+}
+
+// The fixed array's error word (and, after a timeout, its band counters): read with plain copies
+// to and from the array's cached device address, so this allocates nothing either.
+extern "C" int qg_noalloc_device_error(void *stream, int *flag)
+{
+    if (!flag) return QG_ERR_NULL;
+    *flag = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QG_ERR_CUDA;
+    uint8_t *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_noalloc_base.find(dev);
+        if (it == g_noalloc_base.end()) return QG_OK;  // no call on this device yet
+        base = it->second;
+    }
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QG_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, base, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QG_ERR_CUDA;
+    if (v != 0) {
+        // a warp that gave up left its band unfinished: clear the error word and the counters
+        if (cudaMemset(base, 0, ws_bytes_for(kNoallocCounters, 0, 0) - 256) != cudaSuccess)
+            return QG_ERR_CUDA;
+    }
+    *flag = v;
     return QG_OK;
 }

@@ -40,6 +40,14 @@ constexpr int kFmtQ8_0 = 8;
 constexpr int kFmtQ4_K = 12;
 constexpr int kFmtQ5_K = 13;
 constexpr int kFmtQ6_K = 14;
+constexpr int kFmtIQ4_XS = 23;
+
+// IQ4_XS codebook: the sixteen integer levels of the format, each stored biased by +128 as one
+// unsigned byte (levels -127 .. 113 -> 1 .. 241), four per word in index order.
+constexpr uint32_t kIq4Lut0 = 0x3F2D1801u;  // levels of indices 0..3:   -127 -104  -83  -65
+constexpr uint32_t kIq4Lut1 = 0x766A5D4Fu;  // indices 4..7:              -49  -35  -22  -10
+constexpr uint32_t kIq4Lut2 = 0xA6998D81u;  // indices 8..11:               1   13   25   38
+constexpr uint32_t kIq4Lut3 = 0xF1D9C5B5u;  // indices 12..15:             53   69   89  113
 
 constexpr int kVarDirect = 1;
 constexpr int kVarFactored = 2;
@@ -798,11 +806,43 @@ __device__ __forceinline__ float q6k_weight(const uint8_t *blk, int i)
     return __fmul_rn(D, (float)(q - 32));
 }
 
+// IQ4_XS {fp16 d; u16 scales_h; u8 scales_l[4]; u8 qs[128]}: sub-block j = i / 32 has the 6-bit
+// ls_j = nibble (j % 2) of scales_l[j / 2] + 16 * bits 2j..2j+1 of scales_h; weight i's index is
+// the low (r < 16) or high (r >= 16) nibble of qs[16j + r % 16], r = i % 32;
+// w = d * (ls_j - 32) * level[index], exact in fp32 (d*(ls-32) has at most 16 significant bits,
+// the level at most 7).
+__device__ __forceinline__ int iq4_level(int v)
+{
+    const uint32_t w = (v < 8) ? ((v < 4) ? kIq4Lut0 : kIq4Lut1) : ((v < 12) ? kIq4Lut2 : kIq4Lut3);
+    return (int)((w >> (8 * (v & 3))) & 0xFFu) - 128;
+}
+
+__device__ __forceinline__ float iq4xs_weight(const uint8_t *blk, int i)
+{
+    const int j = i >> 5, r = i & 31;
+    const int sh = blk[2] | (blk[3] << 8);
+    const int ls = ((blk[4 + (j >> 1)] >> (4 * (j & 1))) & 15) | (((sh >> (2 * j)) & 3) << 4);
+    const uint8_t qb = blk[8 + 16 * j + (r & 15)];
+    const int v = iq4_level((r < 16) ? (qb & 15) : (qb >> 4));
+    return __fmul_rn(__fmul_rn(half_bits_to_float(blk), (float)(ls - 32)), (float)v);
+}
+
+template <int FMT> struct KqBlock {
+    static constexpr int kBytes = (FMT == kFmtQ5_K) ? 176 : (FMT == kFmtQ6_K) ? 210 : 136;
+};
+
+template <int FMT>
+__device__ __forceinline__ float kq_weight(const uint8_t *blk, int i)
+{
+    return (FMT == kFmtQ5_K) ? q5k_weight(blk, i) : (FMT == kFmtQ6_K) ? q6k_weight(blk, i)
+                                                                        : iq4xs_weight(blk, i);
+}
+
 // dump: thread t writes the 16 weights of group t % 16 of superblock t / 16
 template <int FMT>
 __global__ void dequant_kq_kernel(const uint8_t *W, int64_t nsb, float *out)
 {
-    constexpr int SB = (FMT == kFmtQ5_K) ? 176 : 210;
+    constexpr int SB = KqBlock<FMT>::kBytes;
     const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (t >= nsb * 16) return;
     const int64_t sb = t >> 4;
@@ -810,8 +850,7 @@ __global__ void dequant_kq_kernel(const uint8_t *W, int64_t nsb, float *out)
     const uint8_t *blk = W + sb * SB;
     float *o = out + sb * 256 + 16 * g;
 #pragma unroll 4
-    for (int e = 0; e < 16; ++e)
-        o[e] = (FMT == kFmtQ5_K) ? q5k_weight(blk, 16 * g + e) : q6k_weight(blk, 16 * g + e);
+    for (int e = 0; e < 16; ++e) o[e] = kq_weight<FMT>(blk, 16 * g + e);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -855,8 +894,8 @@ __global__ void rowwise_gemv_kernel(const uint8_t *W, int64_t N, int64_t K, cons
                     }
                 }
             }
-        } else if (FMT == kFmtQ5_K || FMT == kFmtQ6_K) {
-            constexpr int SB = (FMT == kFmtQ5_K) ? 176 : 210;
+        } else if (FMT == kFmtQ5_K || FMT == kFmtQ6_K || FMT == kFmtIQ4_XS) {
+            constexpr int SB = KqBlock<FMT>::kBytes;
             const int64_t nsb = K / 256;
             // lane -> (superblock, 16-weight group)
             for (int64_t it = lane; it < nsb * 16; it += 32) {
@@ -865,8 +904,7 @@ __global__ void rowwise_gemv_kernel(const uint8_t *W, int64_t N, int64_t K, cons
                 const uint8_t *blk = W + (n * nsb + sb) * SB;
                 const int64_t k0 = sb * 256 + 16 * g;
                 for (int e = 0; e < 16; ++e) {
-                    const float wv = (FMT == kFmtQ5_K) ? q5k_weight(blk, 16 * g + e)
-                                                       : q6k_weight(blk, 16 * g + e);
+                    const float wv = kq_weight<FMT>(blk, 16 * g + e);
                     for (int b = 0; b < B; ++b)
                         acc[b] = fmaf(wv, __half2float(__ushort_as_half(x[(k0 + e) * B + b])), acc[b]);
                 }
@@ -892,10 +930,12 @@ __global__ void rowwise_gemv_kernel(const uint8_t *W, int64_t N, int64_t K, cons
 
 // ------------------------------------------------------------------------------------------------
 // x from page-locked host memory into device scratch (qg_gemv_host).  Each thread reads one
-// 16-byte piece (or, unaligned, 8 halves one by one) of the host copy first, which depends on no
-// earlier work, then waits for the previous kernel on the stream before it overwrites the scratch
-// that kernel may still be reading; it lets the next kernel (the GEMV) launch at once, so the
-// GEMV's weight prefetch overlaps the copy.
+// 16-byte piece (or, unaligned, 8 halves one by one) of the host copy first, then waits for the
+// previous kernel on the stream before it overwrites the scratch that kernel may still be
+// reading; it lets the next kernel (the GEMV) launch at once, so the GEMV's weight prefetch
+// overlaps the copy.  Reading the host copy before that wait is what the entry point's contract
+// allows: x_host must not be written by device work queued before the call (a host-side caller
+// fills it before making the call).
 // ------------------------------------------------------------------------------------------------
 __global__ void host_x_copy_kernel(const uint16_t *src, uint16_t *dst, int64_t n)
 {

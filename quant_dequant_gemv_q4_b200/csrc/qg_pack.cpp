@@ -14,6 +14,9 @@
 // ql[64h + 32(t % 2) + l] (bits 0-3 for t < 2, bits 4-7 for t >= 2) and its high two bits at bits
 // 2t, 2t + 1 of qh[32h + l].
 // Q8_0 block {fp16 d; i8 qs[32]}.
+// IQ4_XS superblock {fp16 d; u16 scales_h; u8 scales_l[4]; u8 qs[128]}: the 6-bit scale of
+// sub-block j keeps bits 0-3 in nibble j % 2 of scales_l[j / 2] and bits 4-5 at bits 2j, 2j + 1 of
+// scales_h; qs[16j + l] = idx[32j + l] | idx[32j + 16 + l] << 4.
 #include <cstdint>
 #include <cstring>
 
@@ -63,13 +66,14 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K)
     if (fmt == QG_FMT_Q5_K) return (K % 256) ? 0 : (size_t)N * (size_t)(K / 256) * 176u;
     if (fmt == QG_FMT_Q6_K) return (K % 256) ? 0 : (size_t)N * (size_t)(K / 256) * 210u;
     if (fmt == QG_FMT_Q8_0) return (K % 32) ? 0 : (size_t)N * (size_t)(K / 32) * 34u;
+    if (fmt == QG_FMT_IQ4_XS) return (K % 256) ? 0 : (size_t)N * (size_t)(K / 256) * 136u;
     return 0;
 }
 
 int qg_pack_reference(int fmt, int64_t N, int64_t K, const uint16_t *d, const uint16_t *dmin,
                       const uint8_t *sc, const uint8_t *m, const void *q, void *out)
 {
-    if (!is_kquant(fmt) && fmt != QG_FMT_Q8_0) return QG_ERR_FMT;
+    if (!is_kquant(fmt) && fmt != QG_FMT_Q8_0 && fmt != QG_FMT_IQ4_XS) return QG_ERR_FMT;
     if (qg_weight_bytes(fmt, N, K) == 0 && N != 0) return QG_ERR_SHAPE;
     if (N < 0) return QG_ERR_SHAPE;
     if (N == 0) return QG_OK;
@@ -118,6 +122,29 @@ int qg_pack_reference(int fmt, int64_t N, int64_t K, const uint16_t *d, const ui
             }
             std::memcpy(blk + 192, sc + 16 * s, 16);
             put_half(blk + 208, d[s]);
+        }
+    } else if (fmt == QG_FMT_IQ4_XS) {
+        if (!sc) return QG_ERR_NULL;
+        const uint8_t *qq = static_cast<const uint8_t *>(q);
+        const int64_t nsb = N * (K / 256);
+        for (int64_t s = 0; s < nsb; ++s) {
+            uint8_t *blk = o + s * 136;
+            const uint8_t *Q = qq + 256 * s;
+            const uint8_t *L = sc + 8 * s;
+            for (int i = 0; i < 256; ++i)
+                if (Q[i] > 15) return QG_ERR_RANGE;
+            uint16_t scales_h = 0;
+            std::memset(blk + 4, 0, 4);
+            for (int j = 0; j < 8; ++j) {
+                if (L[j] > 63) return QG_ERR_RANGE;
+                blk[4 + j / 2] |= (uint8_t)((L[j] & 15) << (4 * (j % 2)));
+                scales_h |= (uint16_t)((L[j] >> 4) << (2 * j));
+            }
+            put_half(blk, d[s]);
+            put_half(blk + 2, scales_h);
+            for (int j = 0; j < 8; ++j)
+                for (int l = 0; l < 16; ++l)
+                    blk[8 + 16 * j + l] = (uint8_t)(Q[32 * j + l] | (Q[32 * j + 16 + l] << 4));
         }
     } else {
         const int8_t *qq = static_cast<const int8_t *>(q);

@@ -39,36 +39,54 @@ namespace qg {
 //   kGroups     x-sum groups per unit (sub-blocks of 32 weights; Q6_K: scale groups of 16)
 //   kHiOff      the weights of a byte's high nibble sit kHiOff after those of its low nibble
 //   kPerLane    false: one 2-D tensor copy per step; true: one bulk copy per lane
+//   kWinBytes   per-lane copies: bytes of the 16-byte aligned window copied around a unit
 template <int FMT> struct RowsFmt;
 template <> struct RowsFmt<kFmtQ4_K> {
     static constexpr int kUnitBytes = 144, kLaneBytes = 144, kGroups = 8, kHiOff = 32;
     static constexpr bool kPerLane = false;
+    static constexpr int kWinBytes = 0;
 };
 template <> struct RowsFmt<kFmtQ8_0> {
     static constexpr int kUnitBytes = 272, kLaneBytes = 272, kGroups = 8, kHiOff = 32;
     static constexpr bool kPerLane = false;
+    static constexpr int kWinBytes = 0;
 };
 template <> struct RowsFmt<kFmtQ5_K> {
     static constexpr int kUnitBytes = 176, kLaneBytes = 176, kGroups = 8, kHiOff = 32;
     static constexpr bool kPerLane = false;
+    static constexpr int kWinBytes = 0;
 };
+// Q6_K: a 210-byte unit starts 0..14 bytes (even) past a 16-byte boundary: a 224-byte window,
+// in a 240-byte slot (the consumer's funnel shifts read one word past the window)
 template <> struct RowsFmt<kFmtQ6_K> {
     static constexpr int kUnitBytes = 210, kLaneBytes = 240, kGroups = 16, kHiOff = 64;
     static constexpr bool kPerLane = true;
+    static constexpr int kWinBytes = 224;
+};
+// IQ4_XS: a 136-byte unit starts 0 or 8 bytes past a 16-byte boundary: a 144-byte window.  A
+// byte of qs holds weights r and r + 16 of its 32-weight sub-block.
+template <> struct RowsFmt<kFmtIQ4_XS> {
+    static constexpr int kUnitBytes = 136, kLaneBytes = 144, kGroups = 8, kHiOff = 16;
+    static constexpr bool kPerLane = true;
+    static constexpr int kWinBytes = 144;
 };
 
 // First of the four weights whose x the staging stores at chunk c, word i of a unit: the weights
 // of the low nibbles of qs word i of chunk c (Q4_K, Q5_K, Q8_0: 64c + 4i; Q6_K, whose chunk
-// c = 2h + p is ql[64h + 32p .. 64h + 32p + 31]: 128h + 32p + 4i).
+// c = 2h + p is ql[64h + 32p .. 64h + 32p + 31]: 128h + 32p + 4i; IQ4_XS, whose chunk c is the
+// 32 qs bytes of sub-blocks 2c and 2c + 1: 32 (2c + i / 4) + 4 (i % 4)).
 template <int FMT>
 __device__ __forceinline__ int rows_x_lo(int c, int i)
 {
-    return (FMT == kFmtQ6_K) ? 128 * (c >> 1) + 32 * (c & 1) + 4 * i : 64 * c + 4 * i;
+    return (FMT == kFmtQ6_K)     ? 128 * (c >> 1) + 32 * (c & 1) + 4 * i
+           : (FMT == kFmtIQ4_XS) ? 64 * c + 32 * (i >> 2) + 4 * (i & 3)
+                                 : 64 * c + 4 * i;
 }
 
 // warps per CTA: as many as the shared-memory budget allows next to x
 template <int FMT, int BP> struct RowsWarps {
-    static constexpr int value = (FMT == kFmtQ4_K || FMT == kFmtQ5_K) ? (BP >= 8 ? 12 : 16)
+    static constexpr int value = (FMT == kFmtQ4_K || FMT == kFmtQ5_K || FMT == kFmtIQ4_XS)
+                                     ? (BP >= 8 ? 12 : 16)
                                  : (FMT == kFmtQ6_K)                  ? (BP >= 4 ? 8 : 12)
                                                                       : (BP >= 4 ? 6 : 8);
 };
@@ -189,11 +207,18 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
         const int b = jcb % BP;
         const int jc = jcb / BP;
         const int c = jc & 3, j = jc >> 2;
-        uint4 v;  // group order (e, e+2, e+1, e+3)
-        v.x = h[0] | (h[2] << 16);
-        v.y = h[1] | (h[3] << 16);
-        v.z = h[4] | (h[6] << 16);
-        v.w = h[5] | (h[7] << 16);
+        uint4 v;
+        if (FMT == kFmtIQ4_XS) {  // pair order (e, e+16), (e+1, e+17), (e+2, e+18), (e+3, e+19)
+            v.x = h[0] | (h[4] << 16);
+            v.y = h[1] | (h[5] << 16);
+            v.z = h[2] | (h[6] << 16);
+            v.w = h[3] | (h[7] << 16);
+        } else {  // group order (e, e+2, e+1, e+3)
+            v.x = h[0] | (h[2] << 16);
+            v.y = h[1] | (h[3] << 16);
+            v.z = h[4] | (h[6] << 16);
+            v.w = h[5] | (h[7] << 16);
+        }
         *reinterpret_cast<uint4 *>(xs + rows_x_off<BP>(US, j, c, i, b)) = v;
         // sub-block sums of the chunk: low half (sub-block 2c) and high half (2c+1), fp32, the
         // same xor-butterfly order on every lane
@@ -205,7 +230,13 @@ __device__ __forceinline__ void rows_stage_x(const RowsArgs &a, int s, int US_s,
                     __half2float(__ushort_as_half((unsigned short)h[5]))) +
                    (__half2float(__ushort_as_half((unsigned short)h[6])) +
                     __half2float(__ushort_as_half((unsigned short)h[7])));
-        if (G == 8) {
+        if (FMT == kFmtIQ4_XS) {
+            // all eight halves lie in sub-block 2c + i / 4: the four words of each sub-block
+            float t = lo + hi;
+#pragma unroll
+            for (int off = 1; off < 4; off <<= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+            if ((i & 3) == 0) xsum[rows_xsum_off<BP, G>(US, j, 2 * c + (i >> 2), b)] = t;
+        } else if (G == 8) {
             // 32-weight sub-blocks 2c (low nibbles) and 2c + 1: all 8 words of the chunk
 #pragma unroll
             for (int off = 1; off < 8; off <<= 1) {
@@ -530,6 +561,86 @@ __device__ __forceinline__ void rows_q6k(const uint32_t *win, int o, bool tail, 
     }
 }
 
+// IQ4_XS codebook lookup of the eight 4-bit indices of a qs word: lo = the biased levels
+// (level + 128, one byte each) of nibbles 0..3, hi = of nibbles 4..7, in nibble order.  A nibble's
+// low three bits pick one of the eight bytes of (kIq4Lut0, kIq4Lut1) and of (kIq4Lut2, kIq4Lut3);
+// its bit 3 then picks which of the two results to keep.
+__device__ __forceinline__ void iq4_lookup(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t s = w & 0x77777777u;
+    const uint32_t pick = ((w >> 1) & 0x44444444u) | 0x32103210u;  // nibble k: k % 4 + 4 * bit 3
+    lo = __byte_perm(__byte_perm(kIq4Lut0, kIq4Lut1, s), __byte_perm(kIq4Lut2, kIq4Lut3, s), pick);
+    hi = __byte_perm(__byte_perm(kIq4Lut0, kIq4Lut1, s >> 16), __byte_perm(kIq4Lut2, kIq4Lut3, s >> 16),
+                     pick >> 16);
+}
+
+// One IQ4_XS superblock against x (unit j of the slice), from the lane's ring window: the
+// superblock starts `o` bytes (0 or 8) into the 16-byte aligned window `win`, so its word k is
+// window word o/4 + k.  When `tail` is set (the tensor's last superblock, whose window was cut at
+// the tensor's last 16-byte boundary) its last two words are read from `gblk` in global memory.
+// Arithmetic: each biased level u = level + 128 (1..241) becomes the fp16 subnormal u * 2^-24
+// (the byte under a zero byte), fma.rn.f32.f16 forms u * x exactly, and per sub-block
+//   sum level * x = 2^24 * sum (u * 2^-24) x - 128 X_j,
+// scaled by d * (ls_j - 32) (exact in fp32).
+template <int BP>
+__device__ __forceinline__ void rows_iq4xs(const uint32_t *win, int o, bool tail, const uint8_t *gblk,
+                                           const __half *xs, const float *xsum, int US, int j,
+                                           float (&v)[BP])
+{
+    const uint32_t *wp = win + (o >> 2);
+    const uint32_t w0 = wp[0];   // d (bits 0-15), scales_h (bits 16-31)
+    const uint32_t sl = wp[1];   // scales_l[0..3]
+    const uint32_t sh = w0 >> 16;
+    const float ds = __half2float(__ushort_as_half((unsigned short)(w0 & 0xFFFFu))) * 16777216.0f;
+    auto word = [&](int k) {
+        return (tail && k >= 32) ? *reinterpret_cast<const uint32_t *>(gblk + 4 * k) : wp[k];
+    };
+#pragma unroll
+    for (int b = 0; b < BP; ++b) v[b] = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        // sub-blocks 2c and 2c + 1: scales_l byte c (both nibbles), scales_h bits 4c .. 4c+3
+        const int lsA = (int)(((sl >> (8 * c)) & 15u) | (((sh >> (4 * c)) & 3u) << 4));
+        const int lsB = (int)(((sl >> (8 * c + 4)) & 15u) | (((sh >> (4 * c + 2)) & 3u) << 4));
+        const float DA = ds * (float)(lsA - 32), DB = ds * (float)(lsB - 32);
+        float a0[BP], a1[BP], b0[BP], b1[BP];
+#pragma unroll
+        for (int b = 0; b < BP; ++b) a0[b] = a1[b] = b0[b] = b1[b] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t lo, hi;
+            iq4_lookup(word(2 + 8 * c + i), lo, hi);
+            const uint32_t p0 = __byte_perm(lo, 0u, 0x4140), p1 = __byte_perm(lo, 0u, 0x4342);
+            const uint32_t p2 = __byte_perm(hi, 0u, 0x4140), p3 = __byte_perm(hi, 0u, 0x4342);
+#pragma unroll
+            for (int b = 0; b < BP; ++b) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xs + rows_x_off<BP>(US, j, c, i, b));
+                if (i < 4) {
+                    mfma2(a0[b], p0, xv.x);
+                    mfma2(a1[b], p1, xv.y);
+                    mfma2(a0[b], p2, xv.z);
+                    mfma2(a1[b], p3, xv.w);
+                } else {
+                    mfma2(b0[b], p0, xv.x);
+                    mfma2(b1[b], p1, xv.y);
+                    mfma2(b0[b], p2, xv.z);
+                    mfma2(b1[b], p3, xv.w);
+                }
+            }
+        }
+        // the u x sums carry 2^-24, so 128 X is scaled by 2^-17 to match
+#pragma unroll
+        for (int b = 0; b < BP; ++b) {
+            const float XA = xsum[rows_xsum_off<BP>(US, j, 2 * c, b)];
+            const float XB = xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)];
+            float t = v[b];
+            t = fmaf(DA, fmaf(-7.62939453125e-06f, XA, a0[b] + a1[b]), t);
+            t = fmaf(DB, fmaf(-7.62939453125e-06f, XB, b0[b] + b1[b]), t);
+            v[b] = t;
+        }
+    }
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar)
 {
@@ -717,9 +828,9 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         tma_load_2d(smem_u32(myring + islot * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER, ig_row, bar);
         advance();
     };
-    // per-lane copies (all 32 lanes): rows whose unit is not 16-byte aligned in W (Q6_K) cannot be
-    // described by a tensor map, so each lane copies the 16-byte aligned window [off & ~15,
-    // (off & ~15) + LB - 16) around its row's unit at byte off; windows never reach past the
+    // per-lane copies (all 32 lanes): rows whose unit is not 16-byte aligned in W (Q6_K, IQ4_XS)
+    // cannot be described by a tensor map, so each lane copies the 16-byte aligned window
+    // [off & ~15, (off & ~15) + kWinBytes) around its row's unit at byte off; windows never reach past the
     // tensor's last 16-byte boundary (the last unit of the tensor may come up short: its tail is
     // read from global memory by the consumer).  Lanes past the last row copy nothing.
     auto issue_lanes = [&]() {
@@ -730,7 +841,8 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
         if (row < a.N) {
             const int64_t ad = ((row * a.UPR + ucol0 + iu) * UB) & ~(int64_t)15;
             const int64_t room = a.wend - ad;
-            nb = (uint32_t)(room < (LB - 16) ? room : (LB - 16));
+            constexpr int WIN = RowsFmt<FMT>::kWinBytes;
+            nb = (uint32_t)(room < WIN ? room : WIN);
             src = a.w[ig_map] + ad;
         }
         const uint32_t tot = __reduce_add_sync(0xffffffffu, nb);
@@ -802,7 +914,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
                 rows_q4k<BP>(u, xs, xsum, a.US, j, v);
             } else if (FMT == kFmtQ5_K) {
                 rows_q5k<BP>(u, xs, xsum, a.US, j, v);
-            } else if (FMT == kFmtQ6_K) {
+            } else if (FMT == kFmtQ6_K || FMT == kFmtIQ4_XS) {
                 // this lane's row and unit: where its superblock sits in the window
                 const int g = q / bs.P;
                 const bool second = (MATS > 1) && g >= bs.Gm;
@@ -810,8 +922,11 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
                 const int64_t m = row * a.UPR + ucol0 + j;  // superblock index in the tensor
                 const int o = (int)((m * UB) & 15);
                 const bool tail = a.wtail && row == a.N - 1 && ucol0 + j == a.UPR - 1;
-                rows_q6k<BP>(reinterpret_cast<const uint32_t *>(u), o, tail,
-                             a.w[second ? MATS - 1 : 0] + m * UB, xs, xsum, a.US, j, v);
+                const uint8_t *gblk = a.w[second ? MATS - 1 : 0] + m * UB;
+                if (FMT == kFmtQ6_K)
+                    rows_q6k<BP>(reinterpret_cast<const uint32_t *>(u), o, tail, gblk, xs, xsum, a.US, j, v);
+                else
+                    rows_iq4xs<BP>(reinterpret_cast<const uint32_t *>(u), o, tail, gblk, xs, xsum, a.US, j, v);
             } else {
                 rows_q8_0<BP>(u, xs, a.US, j, v);
             }

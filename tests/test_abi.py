@@ -44,7 +44,8 @@ def test_weight_bytes(L, orc):
     for fmt, N, K in [(12, 17408, 5120), (12, 5120, 17408), (8, 12288, 5120), (12, 1024, 5120),
                       (8, 3, 96), (12, 0, 256), (12, 1, 300), (8, 1, 33), (7, 1, 256),
                       (12, -1, 256), (12, 1, 0), (13, 17408, 5120), (14, 5120, 17408),
-                      (13, 3, 768), (14, 3, 768), (13, 1, 300), (14, 1, 32), (14, 0, 256)]:
+                      (13, 3, 768), (14, 3, 768), (13, 1, 300), (14, 1, 32), (14, 0, 256),
+                      (23, 17408, 5120), (23, 3, 768), (23, 1, 300), (23, 0, 256)]:
         assert qg.qg_weight_bytes(fmt, N, K) == max(orc.weight_bytes(fmt, N, K), 0), (fmt, N, K)
 
 
@@ -131,6 +132,26 @@ def test_pack_kquant_bytes_roundtrip(L, orc, fmt):
     assert np.array_equal(W, W2)
 
 
+def test_pack_iq4xs_roundtrips_through_oracle_unpack(L, orc):
+    """Random fields -> product packer -> oracle field view == the same fields, and random bytes
+    -> oracle fields -> packer == the same bytes (every bit of the superblock is a field bit)."""
+    rng = np.random.default_rng(23)
+    N, K = 3, 768
+    nsb = N * K // 256
+    d = rng.integers(0, 65536, nsb, dtype=np.uint16)
+    ls = rng.integers(0, 64, N * K // 32, dtype=np.uint8)
+    idx = rng.integers(0, 16, N * K, dtype=np.uint8)
+    W = qg.qg_pack_reference(23, N, K, d, None, ls, None, idx)
+    f = orc.unpack_iq4xs(W, nsb)
+    assert np.array_equal(f["d"], d)
+    assert np.array_equal(f["ls"].reshape(-1), ls) and np.array_equal(f["idx"].reshape(-1), idx)
+    W = synth.iq4xs_weights(2, 512, seed=9)
+    f = orc.unpack_iq4xs(W, 4)
+    W2 = qg.qg_pack_reference(23, 2, 512, f["d"], None, f["ls"].reshape(-1), None,
+                              f["idx"].reshape(-1))
+    assert np.array_equal(W, W2)
+
+
 def test_pack_range_checks(L):
     N, K = 1, 256
     ok = dict(d=np.zeros(1, np.uint16), dmin=np.zeros(1, np.uint16), sc=np.zeros(8, np.uint8),
@@ -152,6 +173,14 @@ def test_pack_range_checks(L):
             qg.qg_pack_reference(fmt, N, K, ok["d"], ok["dmin"], ok["sc"] if fmt == 13 else
                                  np.zeros(16, np.int8), ok["m"], q)
         assert e.value.status == qg.QG_ERR_RANGE
+    ls, idx = np.zeros(8, np.uint8), np.zeros(256, np.uint8)
+    qg.qg_pack_reference(23, N, K, ok["d"], None, ls, None, idx)
+    for arr, bad in [(ls, 64), (idx, 16)]:
+        arr[3] = bad
+        with pytest.raises(qg.QgError) as e:
+            qg.qg_pack_reference(23, N, K, ok["d"], None, ls, None, idx)
+        assert e.value.status == qg.QG_ERR_RANGE
+        arr[3] = 0
     q8 = np.zeros(32, np.int8)
     q8[5] = -128
     with pytest.raises(qg.QgError) as e:
