@@ -1,0 +1,77 @@
+"""The default kernels' accuracy on weights shaped like a min-offset quantizer's output.
+
+A Q4_K/Q5_K quantizer that stores a per-sub-block minimum places dmin*m_j near the middle of
+d*sc_j*[0, qmax], so each weight d*sc_j*q - dmin*m_j is a difference of two terms several times
+larger than itself.  The default (factored) kernels sum d*sc_j*sum(q*x) and dmin*m_j*sum(x)
+separately, so their rounding scales with sum(|d*sc*q*x| + |dmin*m*x|), not sum|w*x|.  These tests
+hold AUTO to the strict bar |y - y_ref| <= 1e-5 * sum|w*x| + 1e-6 on such weights at full size
+(the yardstick of "DP4A Q4K/Q6K GEMV profile is catastrophic through the Gated DeltaNet recurrence
+... #3513", Description: the exact f64 dequantized dot) and report how large the factored
+magnitude gets relative to sum|w*x|.
+"""
+import numpy as np
+import pytest
+
+from quant_dequant_gemv_q4_b200 import synth
+from test_gpu_kquants import _sample_rows, gpu_gemv
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quant_dequant_gemv_q4_b200 import build
+    build.build()
+    return torch.device("cuda:0")
+
+
+def min_offset_fields(N, K, qmax, seed):
+    """(d, dmin, sc, m, q) with dmin*m_j = d*sc_j*u_j, u_j ~ U(4, 11) (to the 6-bit grid): the
+    sub-block's minimum sits 4..11 quantization steps below zero."""
+    rng = np.random.default_rng(seed)
+    nsb, nsub = N * K // 256, N * K // 32
+    d = rng.uniform(1e-4, 2e-3, nsb).astype(np.float16)
+    sc = rng.integers(1, 64, nsub).astype(np.int64)
+    u = rng.uniform(4.0, 11.0, nsub) * qmax / 15.0
+    ds = d.astype(np.float64).repeat(8) * sc                  # d * sc_j
+    want = ds * u                                            # the wanted dmin * m_j
+    dmin = (want.reshape(nsb, 8).max(axis=1) / 63.0).astype(np.float16)
+    dmin = np.maximum(dmin, np.float16(2.0 ** -24))
+    m = np.clip(np.rint(want / dmin.astype(np.float64).repeat(8)), 0, 63).astype(np.uint8)
+    q = rng.integers(0, qmax + 1, N * K).astype(np.uint8)
+    return d.view(np.uint16), dmin.view(np.uint16), sc.astype(np.uint8), m, q
+
+
+@pytest.mark.parametrize("fmt,qmax", [(12, 15), (13, 31)])
+@pytest.mark.parametrize("B", [1, 8])
+def test_min_offset_weights_strict_bound(dev, orc, fmt, qmax, B):
+    import quant_dequant_gemv_q4_b200 as qg
+    N, K = 17408, 5120
+    d, dmin, sc, m, q = min_offset_fields(N, K, qmax, seed=fmt * 10 + B)
+    W = qg.qg_pack_reference(fmt, N, K, d, dmin, sc, m, q)
+    x = synth.activations(K, B, seed=B + 90, massive_frac=1e-3)
+    y = gpu_gemv(dev, W, fmt, N, K, x, 0)
+    rows = _sample_rows(N, np.random.default_rng(B + fmt), k=200)
+    yref, A = orc.gemv(W, fmt, N, K, x, B, rows=rows)
+    # the factored magnitude of the sampled rows
+    dd = np.array([orc.half_to_double(int(v)) for v in d]).repeat(8)
+    dm = np.array([orc.half_to_double(int(v)) for v in dmin]).repeat(8)
+    nsub_row = K // 32
+    Af = np.empty_like(A)
+    xa = np.abs(x.astype(np.float64))
+    for i, r in enumerate(rows):
+        s = slice(r * nsub_row, (r + 1) * nsub_row)
+        qs = q[r * K:(r + 1) * K].astype(np.float64)
+        a = (dd[s] * sc[s]).repeat(32) * qs + (dm[s] * m[s]).repeat(32)
+        Af[i] = a @ xa
+    ratio = float(np.median(Af / A))
+    err = np.abs(y[rows].astype(np.float64) - yref)
+    bound = 1e-5 * A + 1e-6
+    worst = float((err / bound).max())
+    print(f"fmt={fmt} B={B}: factored/strict magnitude median {ratio:.2f}, "
+          f"max err / bound {worst:.3f}")
+    assert ratio > 2.0  # the case is what it claims to be
+    assert np.all(err <= bound), worst
