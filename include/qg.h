@@ -115,7 +115,13 @@ enum {
      * tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the
      * instruction are the B columns of x), so B = 1..8 cost the same (Q4_K: up to 16 columns as
      * two 8-column tiles).  Same error bound as FACTORED.  Requires K % 256 == 0. */
-    QG_VARIANT_TENSOR = 4
+    QG_VARIANT_TENSOR = 4,
+    /* Q4_K and Q5_K: the FACTORED arithmetic with the q*x sums on the fifth-generation tensor
+     * cores (tcgen05.mma kind::f16: the unpacked codes as the A operand in tensor memory, x as the
+     * B operand in shared memory, fp32 accumulators in tensor memory, one accumulator column per
+     * 32-weight sub-block), B = 1..16 for both formats.  Same error bound as FACTORED.  Requires
+     * K % 256 == 0. */
+    QG_VARIANT_TCGEN05 = 5
 };
 
 /* Bytes of an N x K tensor in format fmt; 0 if fmt is unknown, N < 0, K < 1 or K is not a

@@ -26,6 +26,7 @@ QG_VARIANT_DIRECT = 1
 QG_VARIANT_FACTORED = 2
 QG_VARIANT_GENERIC = 3
 QG_VARIANT_TENSOR = 4
+QG_VARIANT_TCGEN05 = 5
 
 QG_OK = 0
 QG_ERR_NULL = 1

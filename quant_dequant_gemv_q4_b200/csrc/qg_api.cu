@@ -15,6 +15,7 @@
 #include "qg_device.cuh"
 #include "qg_rows.cuh"
 #include "qg_mma.cuh"
+#include "qg_umma.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -221,6 +222,7 @@ struct RowsPlan {
     int BP, NW, S, US, Gs, G, red_floats;
     size_t smem;
     bool tensor;  // mma_gemv_kernel instead of rows_gemv_kernel
+    bool umma;    // umma_gemv_kernel (tcgen05) instead of either
 };
 
 RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di, bool tensor,
@@ -310,6 +312,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
         p.red_floats = red;
         p.smem = smem;
         p.tensor = tensor;
+        p.umma = false;
         if (util > best_util) {
             best_util = util;
             util_best = p;
@@ -328,6 +331,84 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     }
     if (best.smem == 0) best = util_best;
     return best;  // smem == 0 if nothing fits
+}
+
+// Plan of the tcgen05 kernel: the same bands and K slices as the row-band kernels, with warpgroups
+// of four warps taking (128-row tile, K part) pairs.  Among the slicings whose shared memory fits
+// (and, past one slice, keep at least 5 units of a row per slice), the least
+//   cost = max(32-row steps of a CTA, warps x steps of its busiest warp) + [S > 1] * 16 * 144 / UB,
+// the row-band kernels' model with a warp's step being its quarter of a warpgroup step.
+RowsPlan make_umma_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di, int mats = 1)
+{
+    RowsPlan best{};
+    const int BP = padded_cols(B);
+    const int NW = BP >= 16 ? UmmaWarps<16>::value : BP >= 8 ? UmmaWarps<8>::value : UmmaWarps<1>::value;
+    const int NWG = NW / 4;
+    const int UB = (fmt == kFmtQ5_K) ? UmmaFmt<kFmtQ5_K>::kUnitBytes : UmmaFmt<kFmtQ4_K>::kUnitBytes;
+    const int U = 16 / BP;
+    const size_t ring = (size_t)NW * kRowsStages * 32 * UB;
+    const size_t bars = (size_t)(NW * kRowsStages + NWG * 4) * 8 + 16;
+    const int64_t UPR = K / 256;
+    const int64_t max_slices = std::min<int64_t>(std::min<int64_t>(UPR, 64), std::max(di.sms, 1));
+    double best_cost = 1e300;
+    int64_t best_steps = INT64_MAX;
+    for (int64_t S0 = 1; S0 <= max_slices; ++S0) {
+        const int64_t US = (UPR + S0 - 1) / S0;
+        const int64_t S = (UPR + US - 1) / US;
+        if (S != S0) continue;
+        if (S > 1 && US < 5) continue;
+        const int64_t Gs = std::max<int64_t>(1, std::min<int64_t>(di.sms / S, N));
+        const int64_t band_rows = (N + Gs - 1) / Gs;
+        const int64_t T = (band_rows + 127) / 128;
+        const int64_t P = std::max<int64_t>(1, std::min<int64_t>(NWG / std::max<int64_t>(mats * T, 1), US));
+        const int64_t pairs = mats * T * P;
+        const int64_t USP = ((US + U - 1) / U) * U;
+        // partial rows of every (32-row group, K part); a CTA with fewer rows than band_rows may
+        // have fewer tiles and more parts, so take the largest tiles x parts over T' <= T
+        int64_t tp = 0;
+        for (int64_t T1 = 1; T1 <= T; ++T1)
+            tp = std::max<int64_t>(tp, T1 * std::max<int64_t>(1, std::min<int64_t>(NWG / std::max<int64_t>(mats * T1, 1), US)));
+        const int64_t red = mats * 4 * tp * 32 * BP;
+        const size_t smem = ring + (size_t)USP * 512 * BP + (size_t)US * 8 * BP * 4 + (size_t)red * 4 + bars;
+        if (smem > (size_t)di.smem_optin) continue;
+        const int64_t warp_steps = ((pairs + NWG - 1) / NWG) * ((US + P - 1) / P);
+        const int64_t steps = mats * 4 * T * US;
+        const double cost = (double)std::max<int64_t>(steps, NW * warp_steps) + (S > 1 ? 16.0 * 144.0 / UB : 0.0);
+        if (cost < best_cost || (cost == best_cost && steps < best_steps)) {
+            best_cost = cost;
+            best_steps = steps;
+            best.BP = BP;
+            best.NW = NW;
+            best.S = (int)S;
+            best.US = (int)US;
+            best.Gs = (int)Gs;
+            best.G = (int)(Gs * S);
+            best.red_floats = (int)red;
+            best.smem = smem;
+            best.tensor = true;
+            best.umma = true;
+        }
+    }
+    return best;  // smem == 0 if nothing fits
+}
+
+const void *umma_kernel_ptr(int fmt, int BP, int mats)
+{
+#define QG_UMMA_SWITCH(F, M)                                                              \
+    switch (BP) {                                                                         \
+    case 1: return reinterpret_cast<const void *>(&umma_gemv_kernel<F, 1, M>);          \
+    case 2: return reinterpret_cast<const void *>(&umma_gemv_kernel<F, 2, M>);          \
+    case 4: return reinterpret_cast<const void *>(&umma_gemv_kernel<F, 4, M>);          \
+    case 8: return reinterpret_cast<const void *>(&umma_gemv_kernel<F, 8, M>);          \
+    default: return reinterpret_cast<const void *>(&umma_gemv_kernel<F, 16, M>);        \
+    }
+    if (fmt == kFmtQ5_K) {
+        if (mats == 2) { QG_UMMA_SWITCH(kFmtQ5_K, 2) }
+        QG_UMMA_SWITCH(kFmtQ5_K, 1)
+    }
+    if (mats == 2) { QG_UMMA_SWITCH(kFmtQ4_K, 2) }
+    QG_UMMA_SWITCH(kFmtQ4_K, 1)
+#undef QG_UMMA_SWITCH
 }
 
 const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
@@ -454,7 +535,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
                 unsigned *cnt, float *part, bool pdl, const void *W2 = nullptr, int act = 0,
                 const float *res = nullptr)
 {
-    const void *fn = rows_kernel_ptr(fmt, p.BP, p.tensor, W2 ? 2 : 1);
+    const void *fn = p.umma ? umma_kernel_ptr(fmt, p.BP, W2 ? 2 : 1) : rows_kernel_ptr(fmt, p.BP, p.tensor, W2 ? 2 : 1);
     int rc = ensure_smem_attr(dev, fn, di.smem_optin);
     if (rc != QG_OK) return rc;
     WeightMaps<2> maps;  // the first map alone is the WeightMaps<1> of a single matrix
@@ -552,9 +633,11 @@ int resolve_variant(int fmt, int64_t K, int B, int variant, int *var_out)
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
     if (var == QG_VARIANT_TENSOR && (fmt == QG_FMT_Q8_0 || fmt == QG_FMT_IQ4_XS)) return QG_ERR_VARIANT;
-    if (B > 8 && fmt != QG_FMT_Q4_K) return QG_ERR_BATCH;  // 9..16 columns: the Q4_K kernel only
+    // 9..16 columns: the Q4_K tensor-core kernels, and the tcgen05 kernel for Q5_K too
+    if (B > 8 && fmt != QG_FMT_Q4_K && !(fmt == QG_FMT_Q5_K && var == QG_VARIANT_TCGEN05)) return QG_ERR_BATCH;
     if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16 columns: tensor cores only
+    if (var == QG_VARIANT_TCGEN05 && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K) return QG_ERR_VARIANT;
+    if (B > 8 && var != QG_VARIANT_TENSOR && var != QG_VARIANT_TCGEN05) return QG_ERR_BATCH;
     *var_out = var;
     return QG_OK;
 }
@@ -565,7 +648,7 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
     if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
-    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TENSOR) return QG_ERR_VARIANT;
+    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TCGEN05) return QG_ERR_VARIANT;
     if (N == 0) return QG_OK;
     if (!x || !y) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
@@ -586,8 +669,9 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
         return rc;
     }
 
-    if (var == QG_VARIANT_FACTORED || var == QG_VARIANT_TENSOR) {
-        const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
+    if (var == QG_VARIANT_FACTORED || var == QG_VARIANT_TENSOR || var == QG_VARIANT_TCGEN05) {
+        const RowsPlan p = (var == QG_VARIANT_TCGEN05) ? make_umma_plan(fmt, N, K, B, di)
+                                                       : make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
         if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
         WsView ws;
         const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
@@ -895,7 +979,7 @@ int qg_plan(int fmt, int64_t N, int64_t K, int B, int variant, int mats, int sms
     const int64_t bw = (fmt == QG_FMT_Q8_0) ? 32 : 256;
     if (N < 1 || K < 1 || K % bw != 0 || (mats != 1 && mats != 2)) return QG_ERR_SHAPE;
     if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
-    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TENSOR) return QG_ERR_VARIANT;
+    if (variant < QG_VARIANT_AUTO || variant > QG_VARIANT_TCGEN05) return QG_ERR_VARIANT;
     int var = 0, rc = QG_OK;
     if (mats == 2) {
         // the gate/up pair: the variant qg_gemv would take, rows of whole units
@@ -927,7 +1011,8 @@ int qg_plan(int fmt, int64_t N, int64_t K, int B, int variant, int mats, int sms
         std::memcpy(out, o, sizeof(o));
         return QG_OK;
     }
-    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR, mats);
+    const RowsPlan p = (var == QG_VARIANT_TCGEN05) ? make_umma_plan(fmt, N, K, B, di, mats)
+                                                   : make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR, mats);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     const int64_t o[6] = {var, p.S, p.US, p.G, p.NW, (int64_t)p.smem};
     std::memcpy(out, o, sizeof(o));

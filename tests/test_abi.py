@@ -219,7 +219,12 @@ def test_variant_checks(L):
     # unknown variants are rejected; the streaming variants need rows of whole 256-weight units
     assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 7) == qg.QG_ERR_VARIANT
     assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, -1) == qg.QG_ERR_VARIANT
-    assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 5) == qg.QG_ERR_VARIANT
+    assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 1, FAKE, None, 6) == qg.QG_ERR_VARIANT
+    # the tcgen05 variant takes Q4_K and Q5_K (1..16 columns) only
+    for fmt in (8, 14, 23):
+        assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TCGEN05) == qg.QG_ERR_VARIANT
+    assert L.qg_gemv_variant(FAKE, 13, 4, 300, FAKE, 1, FAKE, None, qg.QG_VARIANT_TCGEN05) == qg.QG_ERR_SHAPE
+    assert L.qg_gemv_variant(FAKE, 13, 4, 256, FAKE, 17, FAKE, None, qg.QG_VARIANT_TCGEN05) == qg.QG_ERR_BATCH
     # the tensor-core variant takes Q4_K only; every streaming variant needs K % 256 == 0
     assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
     for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_TENSOR):

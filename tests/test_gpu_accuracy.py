@@ -75,3 +75,26 @@ def test_min_offset_weights_strict_bound(dev, orc, fmt, qmax, B):
           f"max err / bound {worst:.3f}")
     assert ratio > 2.0  # the case is what it claims to be
     assert np.all(err <= bound), worst
+
+
+@pytest.mark.parametrize("fmt,B", [(12, 2), (12, 8), (12, 16), (13, 2), (13, 8), (14, 4), (14, 8)])
+@pytest.mark.parametrize("variant", [0, 5])
+def test_tensor_core_margin_with_massive_activations(dev, orc, fmt, B, variant):
+    """The tensor-core kernels with 1% of x scaled x100: the error stays well inside the strict
+    bound (at most half of it).  The codes enter the MMA as normal fp16 numbers; carried as fp16
+    subnormals, the tensor core's sums kept only about 12 bits below their largest product and the
+    same cases reached 0.95 of the bound."""
+    import quant_dequant_gemv_q4_b200 as qg
+    if variant == 5 and fmt == 14:
+        pytest.skip("the tcgen05 kernel takes Q4_K and Q5_K")
+    worst = 0.0
+    for N, K in [(300, 768), (129, 2560), (64, 17408)]:
+        W = synth.weights(fmt, N, K, seed=N + K + B)
+        x = synth.activations(K, B, seed=B + 7, massive_frac=1e-2)
+        y = gpu_gemv(dev, W, fmt, N, K, x, variant)
+        if variant == 0:
+            assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
+        yref, A = orc.gemv(W, fmt, N, K, x, B)
+        worst = max(worst, float((np.abs(y.astype(np.float64) - yref) / (1e-5 * A + 1e-6)).max()))
+    print(f"fmt={fmt} B={B} variant={variant}: max err / bound {worst:.3f}")
+    assert worst <= 0.5
