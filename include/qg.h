@@ -77,7 +77,7 @@ enum {
     QG_ERR_NULL = 1,    /* a required pointer is NULL */
     QG_ERR_FMT = 2,     /* unknown format flag */
     QG_ERR_SHAPE = 3,   /* N < 0, K < 1, or K not a multiple of the block size */
-    QG_ERR_BATCH = 4,   /* B outside 1..8 (1..16 for Q4_K with K % 256 == 0) */
+    QG_ERR_BATCH = 4,   /* B outside 1..8 (1..16 for Q4_K, Q5_K, Q6_K with K % 256 == 0) */
     QG_ERR_ALIGN = 5,   /* W not 16-byte aligned, x not 2-byte aligned or y not 4-byte aligned */
     QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
     QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
@@ -113,8 +113,9 @@ enum {
     QG_VARIANT_GENERIC = 3,
     /* The K-quants (Q4_K, Q5_K, Q6_K): the FACTORED arithmetic with the q*x products on the
      * tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the
-     * instruction are the B columns of x), so B = 1..8 cost the same (Q4_K: up to 16 columns as
-     * two 8-column tiles).  Same error bound as FACTORED.  Requires K % 256 == 0. */
+     * instruction are the B columns of x), so B = 1..8 cost the same (up to 16 columns as two
+     * 8-column tiles).  The codes enter the MMA as normal fp16 numbers O + q (the offset removed
+     * with the x sums).  Same error bound as FACTORED.  Requires K % 256 == 0. */
     QG_VARIANT_TENSOR = 4,
     /* Q4_K and Q5_K: the FACTORED arithmetic with the q*x sums on the fifth-generation tensor
      * cores (tcgen05.mma kind::f16: the unpacked codes as the A operand in tensor memory, x as the
@@ -133,8 +134,8 @@ size_t qg_weight_bytes(int fmt, int64_t N, int64_t K);
  *   fmt    QG_FMT_Q4_K, QG_FMT_Q5_K, QG_FMT_Q6_K, QG_FMT_IQ4_XS or QG_FMT_Q8_0
  *   N, K   rows and reduction length; N >= 0 (N == 0 does nothing); K >= 1, K % block == 0
  *   x      device, fp16 bits [K][B], 2-byte aligned, read only
- *   B      number of columns: 1..8; 1..16 for Q4_K with K % 256 == 0 (9..16 columns run on the
- *          tensor-core kernel, every weight still read once)
+ *   B      number of columns: 1..8; 1..16 for Q4_K, Q5_K and Q6_K with K % 256 == 0 (9..16 columns
+ *          run on the tensor-core kernel, every weight still read once)
  *   y      device, fp32 [N][B], 4-byte aligned, fully overwritten (not accumulated)
  *   stream a cudaStream_t (NULL = the legacy default stream); the call is asynchronous
  * Returns QG_OK once the work is enqueued. */
@@ -173,7 +174,7 @@ int qg_gemv_host(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x
  *   x, B     as for qg_gemv; h: device, fp32 [N][B], 4-byte aligned, fully overwritten
  * The products and sums are those of qg_gemv's default kernels for (fmt, B); silu is evaluated in
  * fp32 with expf.  Errors as qg_gemv, plus QG_ERR_SHAPE when K % 256 != 0 (the fused path needs rows
- * of whole 256-weight units). */
+ * of whole 256-weight units); B = 9..16 for Q4_K and Q5_K only (QG_ERR_BATCH for Q6_K). */
 int qg_gemv_gate_up_silu(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K,
                          const uint16_t *x, int B, float *h, void *stream);
 

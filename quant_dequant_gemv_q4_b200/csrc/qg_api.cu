@@ -445,12 +445,12 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_ROWS_IQ41(bp) rows_gemv_kernel<kFmtIQ4_XS, bp, 1>
 #define QG_ROWS_IQ42(bp) rows_gemv_kernel<kFmtIQ4_XS, bp, 2>
     if (tensor && fmt == kFmtQ5_K) {
-        if (mats == 2) { QG_BP_SWITCH(QG_MMA5K2) }
-        QG_BP_SWITCH(QG_MMA5K1)
+        if (mats == 2) { QG_BP_SWITCH16(QG_MMA5K2) }
+        QG_BP_SWITCH16(QG_MMA5K1)
     }
     if (tensor && fmt == kFmtQ6_K) {
-        if (mats == 2) { QG_BP_SWITCH(QG_MMA6K2) }
-        QG_BP_SWITCH(QG_MMA6K1)
+        if (mats == 2) { QG_BP_SWITCH16(QG_MMA6K2) }
+        QG_BP_SWITCH16(QG_MMA6K1)
     }
     if (tensor) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
@@ -633,8 +633,8 @@ int resolve_variant(int fmt, int64_t K, int B, int variant, int *var_out)
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
     if (var == QG_VARIANT_TENSOR && (fmt == QG_FMT_Q8_0 || fmt == QG_FMT_IQ4_XS)) return QG_ERR_VARIANT;
-    // 9..16 columns: the Q4_K tensor-core kernels, and the tcgen05 kernel for Q5_K too
-    if (B > 8 && fmt != QG_FMT_Q4_K && !(fmt == QG_FMT_Q5_K && var == QG_VARIANT_TCGEN05)) return QG_ERR_BATCH;
+    // 9..16 columns: the K-quants' tensor-core kernels only
+    if (B > 8 && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K) return QG_ERR_BATCH;
     if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (var == QG_VARIANT_TCGEN05 && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K) return QG_ERR_VARIANT;
     if (B > 8 && var != QG_VARIANT_TENSOR && var != QG_VARIANT_TCGEN05) return QG_ERR_BATCH;
@@ -751,7 +751,9 @@ int gate_up_impl(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K, 
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
+    // 9..16 columns: the tensor-core kernel; the Q6_K pair's partial rows and copy windows leave
+    // no room for them
+    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt == QG_FMT_Q6_K)) return QG_ERR_BATCH;
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -783,7 +785,7 @@ int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16: the K-quants' tensor-core kernel
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -865,8 +867,9 @@ int qg_gemv_host(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
     if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
-    // 9..16 columns run on the Q4_K tensor-core kernel only (rows of whole 256-weight units)
-    if (B > 8 && (fmt != QG_FMT_Q4_K || K % 256 != 0)) return QG_ERR_BATCH;
+    // 9..16 columns run on the K-quants' tensor-core kernel only (rows of whole 256-weight units)
+    if (B > 8 && ((fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K) || K % 256 != 0))
+        return QG_ERR_BATCH;
     if (N == 0) return QG_OK;
     if (!x_host || !y_host) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x_host) % 2 != 0 || reinterpret_cast<uintptr_t>(y_host) % 4 != 0)
@@ -986,7 +989,7 @@ int qg_plan(int fmt, int64_t N, int64_t K, int B, int variant, int mats, int sms
         if (variant != QG_VARIANT_AUTO) return QG_ERR_VARIANT;
         if (K % 256 != 0) return QG_ERR_SHAPE;
         var = auto_variant(fmt, K, B);
-        if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
+        if (B > 8 && (var != QG_VARIANT_TENSOR || fmt == QG_FMT_Q6_K)) return QG_ERR_BATCH;
     } else if ((rc = resolve_variant(fmt, K, B, variant, &var)) != QG_OK) {
         return rc;
     }
@@ -1079,7 +1082,7 @@ const char *qg_status_string(int status)
     case QG_ERR_NULL: return "a required pointer is NULL";
     case QG_ERR_FMT: return "unknown format flag";
     case QG_ERR_SHAPE: return "invalid shape (N < 0, K < 1 or K not a multiple of the block size)";
-    case QG_ERR_BATCH: return "B must be in 1..8 (1..16 for Q4_K with K % 256 == 0)";
+    case QG_ERR_BATCH: return "B must be in 1..8 (1..16 for Q4_K, Q5_K, Q6_K with K % 256 == 0)";
     case QG_ERR_ALIGN: return "misaligned pointer (W 16 B, x 2 B, y 4 B)";
     case QG_ERR_CUDA: return "CUDA runtime error";
     case QG_ERR_NOMEM: return "workspace allocation failed";
@@ -1142,7 +1145,7 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
         return QG_ERR_ALIGN;
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && (var != QG_VARIANT_TENSOR || fmt != QG_FMT_Q4_K)) return QG_ERR_BATCH;
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16: the K-quants' tensor-core kernel
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;

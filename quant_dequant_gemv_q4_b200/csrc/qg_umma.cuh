@@ -278,13 +278,13 @@ __global__ void __launch_bounds__(UmmaWarps<BP>::value * 32, 1)
     static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
     static_assert(NW % 4 == 0 && NWG <= 4, "warpgroups of four warps, at most four per CTA");
 
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int s = blockIdx.x / a.Gs;
     const int cta = blockIdx.x % a.Gs;
     const int US_s = min(a.US, a.UPR - s * a.US);
     const int USP = ((a.US + U - 1) / U) * U;  // staged units, a whole number of B groups
     uint8_t *ring = smem;
-    uint8_t *xs = smem + NW * NS * BOX;  // B groups, 1024-byte aligned (NW * NS * BOX is)
+    uint8_t *xs = smem + NW * NS * BOX;  // B groups: 128-byte aligned core matrices (BOX is a 128 multiple)
     float *xsum = reinterpret_cast<float *>(xs + (size_t)USP * 512 * BP);
     float *red = xsum + a.US * 8 * BP;
     uint64_t *bars = reinterpret_cast<uint64_t *>(red + a.red_floats);  // ring bars, then MMA bars

@@ -229,11 +229,14 @@ def test_variant_checks(L):
     assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
     for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_TENSOR):
         assert L.qg_gemv_variant(FAKE, 8, 4, 96, FAKE, 1, FAKE, None, v) == qg.QG_ERR_VARIANT
-    # Q5_K / Q6_K: no four-lanes-per-unit kernel; 1..8 columns on every kernel
+    # Q5_K / Q6_K: no four-lanes-per-unit kernel; 9..16 columns on the tensor-core kernel only
     for fmt in (13, 14):
         assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_DIRECT) == qg.QG_ERR_VARIANT
-        assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None, qg.QG_VARIANT_TENSOR) in (
-            qg.QG_ERR_BATCH, qg.QG_ERR_VARIANT)
+        for v in (qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC):
+            assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
+        assert L.qg_gemv(FAKE, fmt, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
+    # IQ4_XS and Q8_0: 1..8 columns
+    for fmt in (8, 23):
         assert L.qg_gemv(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
         assert L.qg_gemv(FAKE, fmt, 4, 300, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
 
@@ -290,6 +293,7 @@ def test_batch_width_limits(L):
         assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
     assert L.qg_gemv_noalloc(FAKE, 8, 4, 256, FAKE, 16, FAKE, None) == qg.QG_ERR_BATCH
     assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 8, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 14, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
     assert L.qg_gemv_residual(FAKE, 8, 4, 256, FAKE, 12, FAKE, FAKE, None) == qg.QG_ERR_BATCH
 
 
@@ -299,8 +303,9 @@ def test_gemv_host_rejects_bad_arguments(L):
     assert f(FAKE, 99, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_FMT
     assert f(FAKE, 12, 4, 300, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
     assert f(FAKE, 12, 4, 256, FAKE, 0, FAKE, None) == qg.QG_ERR_BATCH
-    assert f(FAKE, 8, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # 9..16: Q4_K only
-    assert f(FAKE, 14, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, 8, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # 9..16: the K-quants only
+    assert f(FAKE, 23, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+    assert f(FAKE, 14, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
     assert f(FAKE, 12, 4, 256, 0, 1, FAKE, None) == qg.QG_ERR_NULL
     assert f(FAKE, 12, 4, 256, FAKE, 1, 0, None) == qg.QG_ERR_NULL
     assert f(FAKE, 12, 4, 256, FAKE + 1, 1, FAKE, None) == qg.QG_ERR_ALIGN

@@ -307,14 +307,69 @@ def test_x_not_16_byte_aligned(dev, orc, fmt, B):
 
 
 @pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
-def test_wide_b_rejected(dev, fmt):
+def test_wide_b_only_on_tensor_cores(dev, fmt):
+    """9..16 columns: the CUDA-core and per-row kernels refuse them; the default (tensor cores)
+    takes them."""
     import quant_dequant_gemv_q4_b200 as qg
     W = synth.weights(fmt, 8, 256, seed=1)
     x = synth.activations(256, 9, seed=1)
-    for v in (0, 2, 3):
+    for v in (2, 3):
         with pytest.raises(qg.QgError) as e:
             gpu_gemv(dev, W, fmt, 8, 256, x, v)
         assert e.value.status == qg.QG_ERR_BATCH
+    gpu_gemv(dev, W, fmt, 8, 256, x, 0)
+    assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
+
+
+# ------------------------------------------------------------------------------------------------
+# Verify widths 9..16 (two 8-column tiles on the tensor cores)
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
+@pytest.mark.parametrize("N,K", [(1, 256), (7, 1280), (33, 5120), (300, 768), (129, 2560)])
+@pytest.mark.parametrize("B", [9, 12, 16])
+def test_gemv_wide_small(dev, orc, fmt, N, K, B):
+    W = synth.weights(fmt, N, K, seed=N * 5 + K + fmt)
+    x = synth.activations(K, B, seed=B + fmt, massive_frac=1e-3)
+    y = gpu_gemv(dev, W, fmt, N, K, x, 0)
+    yref, A = orc.gemv(W, fmt, N, K, x, B)
+    assert_within(y, yref, A, f"fmt={fmt} N={N} K={K} B={B}")
+
+
+@pytest.mark.parametrize("fmt", [Q5_K, Q6_K])
+@pytest.mark.parametrize("N,K", [(17408, 5120), (5120, 17408)])
+@pytest.mark.parametrize("B", [12, 16])
+def test_full_size_sampled_wide(dev, orc, fmt, N, K, B):
+    import quant_dequant_gemv_q4_b200 as qg
+    W = synth.weights(fmt, N, K, seed=N + B + fmt)
+    x = synth.activations(K, B, seed=B + 5)
+    y = gpu_gemv(dev, W, fmt, N, K, x, 0)
+    assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
+    assert np.isfinite(y).all()
+    rows = _sample_rows(N, np.random.default_rng(fmt + B))
+    yref, A = orc.gemv(W, fmt, N, K, x, B, rows=rows)
+    assert_within(y[rows], yref, A, f"fmt={fmt} {N}x{K} B={B}")
+    y2 = gpu_gemv(dev, W, fmt, N, K, x, 0)
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32)), "not deterministic"
+
+
+def test_q5k_gate_up_wide(dev, orc):
+    """The fused pair at 12 columns in Q5_K (Q6_K's pair stops at 8: QG_ERR_BATCH)."""
+    import torch
+    import quant_dequant_gemv_q4_b200 as qg
+    from test_gate_up import assert_h_within
+    N, K, B = 129, 2560, 12
+    Wg = synth.q5k_weights(N, K, seed=51)
+    Wu = synth.q5k_weights(N, K, seed=52)
+    x = synth.activations(K, B, seed=53)
+    h = torch.full((N, B), float("nan"), dtype=torch.float32, device=dev)
+    qg.qg_gemv_gate_up_silu(_t(Wg, dev), _t(Wu, dev), Q5_K, N, K, _t(x.view(np.uint16), dev), B, h)
+    torch.cuda.synchronize()
+    assert_h_within(h.cpu().numpy(), orc.gate_up_silu(Wg, Wu, Q5_K, N, K, x, B), "q5k pair B=12")
+    W6 = synth.q6k_weights(N, K, seed=54)
+    with pytest.raises(qg.QgError) as e:
+        qg.qg_gemv_gate_up_silu(_t(W6, dev), _t(W6, dev), Q6_K, N, K, _t(x.view(np.uint16), dev), B, h)
+    assert e.value.status == qg.QG_ERR_BATCH
 
 
 def test_q6k_tail_window_every_misalignment(dev, orc):

@@ -9,6 +9,7 @@ import quant_dequant_gemv_q4_b200 as qg
 from quant_dequant_gemv_q4_b200 import synth
 
 Q4_K, Q5_K, Q6_K, Q8_0 = synth.Q4_K, synth.Q5_K, synth.Q6_K, synth.Q8_0
+IQ4_XS = synth.IQ4_XS
 B200 = dict(sms=148, smem_optin=232448)
 FACTORED, GENERIC, TENSOR, DIRECT = (qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC,
                                      qg.QG_VARIANT_TENSOR, qg.QG_VARIANT_DIRECT)
@@ -61,7 +62,7 @@ SHAPES = [(1, 256), (17, 256), (33, 512), (100, 768), (1000, 2560), (4096, 4096)
 
 
 @pytest.mark.parametrize("sms,smem", [(148, 232448), (132, 232448), (8, 232448), (148, 180000)])
-@pytest.mark.parametrize("fmt", [Q4_K, Q5_K, Q6_K, Q8_0])
+@pytest.mark.parametrize("fmt", [Q4_K, Q5_K, Q6_K, Q8_0, IQ4_XS])
 def test_plan_invariants(sms, smem, fmt):
     """Every plan fits the device, covers K exactly once with its slices, launches at most one CTA
     per SM, and takes the variant qg_gemv's default rule names."""
@@ -73,8 +74,10 @@ def test_plan_invariants(sms, smem, fmt):
                 try:
                     p = qg.qg_plan(fmt, N, K, B, 0, mats, sms, smem)
                 except qg.QgError as e:
-                    # B > 8 is the Q4_K tensor-core kernel's only; a small device may fit no plan
-                    assert (B > 8 and fmt != Q4_K and e.status == qg.QG_ERR_BATCH) or \
+                    # B > 8 is the K-quants' tensor-core kernel's only (and not the Q6_K pair's);
+                    # a small device may fit no plan
+                    wide_ok = fmt in (Q4_K, Q5_K) or (fmt == Q6_K and mats == 1)
+                    assert (B > 8 and not wide_ok and e.status == qg.QG_ERR_BATCH) or \
                         e.status == qg.QG_ERR_SHAPE, (N, K, B, mats, e)
                     continue
                 n += 1
@@ -83,7 +86,7 @@ def test_plan_invariants(sms, smem, fmt):
                 assert S * US >= UPR > (S - 1) * US
                 assert 1 <= p["ctas"] <= sms
                 assert p["warps"] in (6, 8, 12, 16)
-                assert p["variant"] == (TENSOR if fmt != Q8_0 and B >= 2 else FACTORED)
+                assert p["variant"] == (TENSOR if fmt in (Q4_K, Q5_K, Q6_K) and B >= 2 else FACTORED)
     assert n > 0
 
 
