@@ -510,17 +510,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 2-D view of W for the TMA: N rows of K/256 units in u32 elements; a box is 32 rows x one unit.
+// 2-D view of W for the TMA: N rows of K/256 units in u32 elements; a box is 32 rows x one unit
+// (IQ4_XS: x 144 bytes, the 16-byte aligned window around a 136-byte unit; its rows must be
+// 16-byte multiples, an even number of units).
 int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *map)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return QG_ERR_CUDA;
-    const int UB = (fmt == kFmtQ4_K)   ? RowsFmt<kFmtQ4_K>::kUnitBytes
-                   : (fmt == kFmtQ5_K) ? RowsFmt<kFmtQ5_K>::kUnitBytes
-                                       : RowsFmt<kFmtQ8_0>::kUnitBytes;
-    const cuuint64_t dims[2] = {(cuuint64_t)(K / 256) * (UB / 4), (cuuint64_t)N};
+    const int UB = (fmt == kFmtQ4_K)     ? RowsFmt<kFmtQ4_K>::kUnitBytes
+                   : (fmt == kFmtQ5_K)   ? RowsFmt<kFmtQ5_K>::kUnitBytes
+                   : (fmt == kFmtIQ4_XS) ? RowsFmt<kFmtIQ4_XS>::kUnitBytes
+                                         : RowsFmt<kFmtQ8_0>::kUnitBytes;
+    const int BB = (fmt == kFmtIQ4_XS) ? RowsFmt<kFmtIQ4_XS>::kWinBytes : UB;  // box bytes of a row
+    if (((K / 256) * UB) % 16 != 0) return QG_ERR_SHAPE;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 256) * UB / 4, (cuuint64_t)N};
     const cuuint64_t strides[1] = {(cuuint64_t)(K / 256) * UB};
-    const cuuint32_t box[2] = {(cuuint32_t)(UB / 4), 32};
+    const cuuint32_t box[2] = {(cuuint32_t)(BB / 4), 32};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(W), dims, strides,
                            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -542,7 +547,9 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     static_assert(offsetof(WeightMaps<2>, m) == 0 && sizeof(WeightMaps<1>) == sizeof(CUtensorMap),
                   "WeightMaps<1> is a prefix of WeightMaps<2>");
     std::memset(&maps, 0, sizeof(maps));
-    const bool per_lane = (fmt == kFmtQ6_K || fmt == kFmtIQ4_XS);  // units not 16-byte aligned: no tensor map
+    // units not 16-byte aligned: no tensor map for Q6_K; IQ4_XS rows of an even number of units
+    // are 16-byte multiples, and a 144-byte box around each unit is a legal copy
+    const bool per_lane = (fmt == kFmtQ6_K) || (fmt == kFmtIQ4_XS && (K / 256) % 2 != 0);
     if (!per_lane) {
         if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
         if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
@@ -553,6 +560,7 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     a.w[1] = static_cast<const uint8_t *>(W2 ? W2 : W);
     a.wend = wbytes & ~(int64_t)15;
     a.wtail = (wbytes & 15) ? 1 : 0;
+    a.tmap = (fmt == kFmtIQ4_XS && !per_lane) ? 1 : 0;
     a.x = x;
     a.out = (p.S > 1) ? part : y;
     a.y = y;

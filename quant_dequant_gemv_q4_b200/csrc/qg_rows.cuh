@@ -116,6 +116,9 @@ struct RowsArgs {
     const uint8_t *w[2];  // per-lane copies (Q6_K): the weight tensors (16-byte aligned)
     int64_t wend;         // per-lane copies: the tensor's byte size rounded down to 16
     int wtail;            // per-lane copies: 1 if the byte size is not a multiple of 16
+    int tmap;             // a per-lane format whose rows are 16-byte multiples (IQ4_XS with an even
+                          // number of superblocks per row): the weight maps are valid, one 2-D copy
+                          // per step as for the other formats
 };
 
 // silu(v) * u, the FFN activation of the gate/up pair (silu(v) = v / (1 + e^-v))
@@ -763,8 +766,9 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     constexpr int UB = RowsFmt<FMT>::kUnitBytes;
     constexpr int LB = RowsFmt<FMT>::kLaneBytes;
     constexpr bool PER_LANE = RowsFmt<FMT>::kPerLane;
-    constexpr int BOX = 32 * LB;  // ring bytes of one step: 32 rows x one unit
-    constexpr int INNER = UB / 4; // u32 elements of one unit
+    constexpr int BOX = 32 * LB;  // ring bytes of one step: 32 rows x one unit (or its window)
+    // one bulk copy per lane, or (a per-lane format whose rows are 16-byte multiples) 2-D copies
+    const bool lane_copy = PER_LANE && !a.tmap;
     static_assert(BOX % 128 == 0, "tensor-copy destinations in shared memory must be 128-byte aligned");
     static_assert(LB % 16 == 0, "bulk-copy destinations must be 16-byte aligned");
 
@@ -821,11 +825,14 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
             if (iq < npairs) cursor_pair();
         }
     };
-    // one 2-D tensor copy of the step's 32 rows x one unit (lane 0 alone)
+    // one 2-D tensor copy of the step's 32 rows x one unit (lane 0 alone).  The box starts at the
+    // unit's first byte rounded down to 16 (the unit itself for the formats whose units are
+    // 16-byte multiples; IQ4_XS units sit 0 or 8 bytes past it, inside a 144-byte box).
     auto issue = [&]() {
         const uint32_t bar = bar0 + 8 * islot;
         mbar_arrive_expect_tx(bar, BOX);
-        tma_load_2d(smem_u32(myring + islot * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER, ig_row, bar);
+        const int xw = (int)((((int64_t)(ucol0 + iu) * UB) & ~(int64_t)15) >> 2);
+        tma_load_2d(smem_u32(myring + islot * BOX), &maps.m[ig_map], xw, ig_row, bar);
         advance();
     };
     // per-lane copies (all 32 lanes): rows whose unit is not 16-byte aligned in W (Q6_K, IQ4_XS)
@@ -855,17 +862,17 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     // 1. weight prefetch (independent of the previous kernel on the stream): the first steps
     //    into the ring
     if (nsteps > 0 && lane == 0) {
-        if (!PER_LANE) {
+        if (!lane_copy) {
 #pragma unroll
             for (int m = 0; m < MATS; ++m)
                 asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[m])) : "memory");
         }
         for (int i = 0; i < NS; ++i) mbar_init(bar0 + 8 * i, 1);
         mbar_init_fence();
-        if (!PER_LANE)
+        if (!lane_copy)
             for (int i = 0; i < kPreStages && i < nsteps; ++i) issue();
     }
-    if (PER_LANE && nsteps > 0) {
+    if (lane_copy && nsteps > 0) {
         __syncwarp();
         for (int i = 0; i < kPreStages && i < nsteps; ++i) issue_lanes();
     }
@@ -876,7 +883,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     // 3. x for this slice -> shared memory (fp16 in consumer order) and per-sub-block sums,
     //    then the rest of the ring (this warp's x loads have returned by now)
     rows_stage_x<BP, FMT>(a, s, US_s, xs, xsum);
-    if (PER_LANE) {
+    if (lane_copy) {
         for (int i = kPreStages; i < NS && i < nsteps; ++i) issue_lanes();
     } else if (lane == 0) {
         for (int i = kPreStages; i < NS && i < nsteps; ++i) issue();
@@ -934,7 +941,7 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
             for (int b = 0; b < BP; ++b) acc[b] += v[b];
             __syncwarp();
             if (step + NS < nsteps) {
-                if (PER_LANE) {
+                if (lane_copy) {
                     fence_proxy_async_smem();
                     issue_lanes();
                 } else if (lane == 0) {
