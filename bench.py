@@ -441,6 +441,49 @@ def oracle_sample_rate(call: synth.Gemv, seed: int, seconds: float):
     return nbytes / t_total / 1e9, done_rows, t_total, nbytes
 
 
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# The workload calls the oracle is timed on per config (whole calls: median of 3 runs, 5 for the
+# small attention call), on the same seeded inputs as the GPU table.
+ORACLE_CONFIG_CALLS = (
+    ("q4k_attn_kv_1024x5120", 5),
+    ("q4k_ssm_qkv_10240x5120", 3),
+    ("q4k_ffn_pair_b1", 3),
+    ("mixed_q8_0_q4k_b1", 3),
+    ("q4k_ffn_gate_verify", 3),
+)
+
+
+def oracle_config_table() -> dict:
+    """The oracle per call of every workload config: median wall time of whole calls (single
+    thread), us/call and GB/s on the call's algorithmic bytes."""
+    import oracle
+    oracle.build()
+    out = {}
+    for name, runs in ORACLE_CONFIG_CALLS:
+        wl = synth.WORKLOADS[name]
+        for c in wl.calls:
+            W, x = wl.inputs(c)
+            ts = []
+            for _ in range(runs):
+                t0 = time.perf_counter()
+                oracle.gemv(W, c.fmt, c.N, c.K, x, c.B)
+                ts.append(time.perf_counter() - t0)
+            t = statistics.median(ts)
+            out[f"{name}/{c.name}"] = {"us_per_call": round(t * 1e6, 1),
+                                       "gbs": round(c.algorithmic_bytes / t / 1e9, 4), "runs": runs}
+    return out
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if world > 1:
@@ -554,6 +597,8 @@ def main(argv=None):
     ap.add_argument("--table-steps", type=int, default=4000)
     ap.add_argument("--no-table", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-cpu-configs", action="store_true",
+                    help="skip the oracle's per-config table (whole calls of every config)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: CPU seconds the whole warm-up + timed run takes")
@@ -639,6 +684,20 @@ def main(argv=None):
            "splits": qg.qg_last_splits(), "steps": steps8}
     del cs16
 
+    # the same tensor on the tcgen05 kernel (an explicit variant; the default kernels are the
+    # CUDA-core one at B = 1 and the mma.sync one at B >= 2)
+    tcgen05 = []
+    for Bt, call in ((1, HEADLINE), (8, HEADLINE_B8), (16, HEADLINE_B16)):
+        cst = CallSet([call], HEADLINE_SEED, device, l2)
+        st_t = max(200, min(args.steps // 8, 4000))
+        s_t, _ = time_callset(cst, st_t, args.warmup, qg.QG_VARIANT_TCGEN05, None)
+        s_t = dist_max(s_t, device)
+        tcgen05.append({"B": Bt, "us_per_call": round(s_t * 1e6 / st_t, 3),
+                        "frac_of_hbm": round(cst.bytes_per_step * st_t / s_t / 1e9 / hbm, 4),
+                        "splits": qg.qg_last_splits(), "steps": st_t})
+        del cst
+    torch.cuda.empty_cache()
+
     # the fused FFN gate/up pair (one launch, two weight streams, h = silu(g) * u)
     gate_up = []
     for Bg in (1, 8):
@@ -695,7 +754,9 @@ def main(argv=None):
                "sample": f"{rows} rows ({rows / HEADLINE.N:.2f} passes, {nb / 1e6:.1f} MB) of the "
                          f"N=17408 K=5120 B=1 call in {t:.1f} s, single-threaded C oracle "
                          f"(dequant + fp64 dot)",
-               "host_cores": os.cpu_count()}
+               "host_cores": os.cpu_count(), "host_cpu": host_cpu_model()}
+        if not args.no_cpu_configs:
+            cpu["per_config"] = oracle_config_table()
 
     if world > 1:
         barrier()
@@ -719,6 +780,7 @@ def main(argv=None):
         "roofline": roofline,
         "b8": b8,
         "b16": b16,
+        "tcgen05": tcgen05,
         "gate_up_silu": gate_up,
         "clocks": clocks,
         "e2e": e2e,

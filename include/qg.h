@@ -215,7 +215,7 @@ int qg_pack_reference(int fmt, int64_t N, int64_t K, const uint16_t *d, const ui
                       const uint8_t *sc, const uint8_t *m, const void *q, void *out);
 
 /* Kernel variant launched by the last successful qg_gemv / qg_gemv_variant of the calling host
- * thread (a launch witness: QG_VARIANT_DIRECT, _FACTORED, _GENERIC or _TENSOR), 0 if none yet. */
+ * thread (a launch witness: QG_VARIANT_DIRECT, _FACTORED, _GENERIC, _TENSOR or _TCGEN05), 0 if none yet. */
 int qg_last_variant(void);
 
 /* Number of K slices the last GEMV of the calling thread used (1 = no split-K second pass). */
@@ -268,7 +268,7 @@ int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
  *     last CTA of a band resets its counter); the partial rows are written before they are read.
  *     So nothing is cleared between calls.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- *     that device current) and caches it; make that first call before any stream capture.
+ *     that device current) and caches it; later calls reuse it.
  *   - Every call on every stream shares the one array: calls that overlap on the GPU race and give
  *     wrong results.  Serialize them (one stream, or events between streams).
  *   - QG_ERR_SCRATCH if the call needs more scratch than the array holds (this happens only when

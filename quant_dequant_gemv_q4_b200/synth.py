@@ -208,5 +208,14 @@ WORKLOADS = {
     "kquant_ffn_gate_b8": Workload("kquant_ffn_gate_b8", 7, (
         Gemv("q5k_ffn_gate_b8", Q5_K, 17408, 5120, 8, 0),
         Gemv("q6k_ffn_gate_b8", Q6_K, 17408, 5120, 8, 1))),
+    # the IQ4_XS row of the same FFN tensors (the T4 dossier's GEMV prompt names it next to Q4_K)
+    "iq4xs_ffn_pair_b1": Workload("iq4xs_ffn_pair_b1", 8, (
+        Gemv("ffn_gate", IQ4_XS, 17408, 5120, 1, 0, 1e-3),
+        Gemv("ffn_down", IQ4_XS, 5120, 17408, 1, 1, 1e-3))),
+    # verify widths beyond 8 (up to 16 draft tokens) on the FFN gate in every K-quant
+    "kquant_ffn_gate_b16": Workload("kquant_ffn_gate_b16", 9, (
+        Gemv("q4k_ffn_gate_b16", Q4_K, 17408, 5120, 16, 0),
+        Gemv("q5k_ffn_gate_b16", Q5_K, 17408, 5120, 16, 1),
+        Gemv("q6k_ffn_gate_b16", Q6_K, 17408, 5120, 16, 2))),
 }
 FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q6_K: "Q6_K", Q8_0: "Q8_0", IQ4_XS: "IQ4_XS"}
