@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 # device code and the host planner/launcher.  The tensor-core kernel's file (qg_mma.cuh) and the
 # host packer are not among them, so a change there leaves the headline's DRAM capture valid.
 ROWS_KERNEL_FILES = ("qg_api.cu", "qg_device.cuh", "qg_rows.cuh")
-MMA_KERNEL_FILES = ROWS_KERNEL_FILES + ("qg_mma.cuh",)  # the B >= 2 tensor-core kernel
+MMA_KERNEL_FILES = ROWS_KERNEL_FILES + ("qg_codes.cuh", "qg_mma.cuh")  # the B >= 2 tensor-core kernel
 
 
 def kernel_source_hash(files=None) -> str:
@@ -238,7 +238,11 @@ def time_callset(cs: CallSet, steps: int, warmup: int, variant: int, clocks: Clo
     event (event-record nodes, cudaEventRecordExternal), so the timed region opens while the GPU
     is already streaming: neither the graph's launch nor its upload (done by the warm-up replays,
     which run the whole graph) falls inside it, and every timed call is a steady-state call on a
-    fresh weight copy."""
+    fresh weight copy.  The start event sits on a side branch forked after the last untimed call:
+    it fires when that call completes, while the first timed call keeps its programmatic edge to
+    it (its prologue may overlap the untimed call's tail, as every call's does in the chain).  The
+    region is thus `steps` completion-to-completion intervals of the chain; the end event follows
+    the last timed call's full completion."""
     import torch
     stream = torch.cuda.Stream(device=cs.device)
     R = cs.copies
@@ -250,12 +254,15 @@ def time_callset(cs: CallSet, steps: int, warmup: int, variant: int, clocks: Clo
     start = torch.cuda.Event(enable_timing=True, external=True)
     end = torch.cuda.Event(enable_timing=True, external=True)
     graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=cs.device)
     with torch.cuda.graph(graph, stream=stream):
         for i in range(lead):
             cs.launch(i % R, stream, variant)
-        start.record(stream)
+        side.wait_stream(stream)
+        start.record(side)
         for i in range(steps):
             cs.launch((lead + i) % R, stream, variant)
+        stream.wait_stream(side)
         end.record(stream)
     # warm-up: whole-graph replays until at least `warmup` steps have run (at least one replay,
     # which uploads the graph)

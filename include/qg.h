@@ -114,8 +114,8 @@ enum {
     /* The K-quants (Q4_K, Q5_K, Q6_K): the FACTORED arithmetic with the q*x products on the
      * tensor cores (mma.sync m16n8k16, f16 operands, fp32 accumulation; the 8 columns of the
      * instruction are the B columns of x), so B = 1..8 cost the same (up to 16 columns as two
-     * 8-column tiles).  The codes enter the MMA as normal fp16 numbers O + q (the offset removed
-     * with the x sums).  Same error bound as FACTORED.  Requires K % 256 == 0. */
+     * 8-column tiles).  The codes enter the MMA as the fp16 integers q (normal or zero), so
+     * every product is exact.  Same error bound as FACTORED.  Requires K % 256 == 0. */
     QG_VARIANT_TENSOR = 4,
     /* Q4_K and Q5_K: the FACTORED arithmetic with the q*x sums on the fifth-generation tensor
      * cores (tcgen05.mma kind::f16: the unpacked codes as the A operand in tensor memory, x as the

@@ -12,20 +12,23 @@
 // same tensor work, and the weights are unpacked once for all columns.  Products are exact
 // (integers up to 15 times fp16 x) and the sums are fp32, so the arithmetic is the factored form
 // of the CUDA-core kernel:
-//   sum_i w_i x_i = sum_j [ D_j * sum_{i in j} (O + q_i) x_i  -  (O D_j + M_j) * sum_{i in j} x_i ],
-//   D_j = d*sc_j, M_j = dmin*m_j (exact in fp32), j = 32-weight sub-block, O the code offset.
+//   sum_i w_i x_i = sum_j [ D_j * sum_{i in j} q_i x_i  -  M_j * sum_{i in j} x_i ],
+//   D_j = d*sc_j, M_j = dmin*m_j (exact in fp32), j = 32-weight sub-block.
 //
 // Mapping.  The grid, row bands, (row group, K part) pairs and the per-warp ring of 2-D TMA
 // boxes (32 rows x one 144-byte superblock) are those of the CUDA-core kernel (qg_rows.cuh).  Per
 // step a warp multiplies its 32 rows as two 16-row tiles:
 //   A fragment (rows g and g+8 of a tile, lane = 4g + t): word 2t+h of the 32-byte chunk c of the
-//     row; its low nibbles of bytes 0 and 2 (sub-block 2c) are shifted into the mantissa of two
-//     normal fp16 numbers 16 + q (exponent 4, q in mantissa bits 6-9), its high nibbles likewise
-//     (sub-block 2c+1), and the same on word >> 8 gives bytes 1 and 3.  So one 32-bit word feeds
-//     four A registers.  Normal operands keep the tensor core's full accumulation precision (with
-//     codes as fp16 subnormals its sums keep only about 12 bits below the largest product, which
-//     measured up to 0.95 of the error bound with massive activations; 0.05 with 16 + q); the
-//     offset is removed with the x sums: sum (16 + q) x = 16 X_j + sum q x.
+//     row; its low nibbles of bytes 0 and 2 (sub-block 2c) are masked under the exponent of 1024
+//     (one LOP3: the fp16 pair 1024 + q, q in mantissa bits 0-3) and one packed fp16 FMA takes
+//     the 1024 back out, leaving the fp16 integers q exactly; its high nibbles (sub-block 2c+1)
+//     give 1024 + 16 q the same way, and the FMA scales by 1/16 as it subtracts 64; word >> 8
+//     gives bytes 1 and 3.  So one 32-bit word feeds four A registers through four LOP3 (ALU
+//     pipe), one multiply-high (the shift) and four f16x2 FMAs (FMA pipe).  Normal operands keep
+//     the tensor core's full accumulation precision (with codes as fp16 subnormals its sums keep
+//     only about 12 bits below the largest product, which measured up to 0.95 of the error bound
+//     with massive activations), and codes without an offset keep every product as small as the
+//     weight itself.
 //   B fragment: x in the matching order, staged once per CTA (mma_stage_x).
 //   C fragment: rows g, g+8 x columns 2t, 2t+1, fresh per (chunk, tile, nibble half), then scaled
 //     by D_j of its row and added to the warp's accumulators.
@@ -35,6 +38,7 @@
 // (q5k_a_regs, mma_q6k_step), and Q6_K scales each 16-weight k-tile by its own group's D_t.
 #pragma once
 
+#include "qg_codes.cuh"
 #include "qg_rows.cuh"
 
 namespace qg {
@@ -45,24 +49,19 @@ template <int BP> struct MmaWarps {
     static constexpr int value = BP >= 16 ? 8 : BP >= 8 ? 12 : 16;
 };
 
-// Formats of the tensor-core kernel: Q4_K, and Q5_K (the Q4_K superblock with a fifth-bit plane
-// qh[32] before qs).  kQs: offset of qs in the superblock; kOff: the offset O of the A operand's
-// normal fp16 codes O + q (Q4_K 16, Q5_K 32, Q6_K 64: the smallest power of two above the codes,
-// so O + q has O's exponent and q fits its mantissa; a smaller offset keeps more of the sum's
-// precision for q x).
+// Formats of the tensor-core kernel: Q4_K, Q5_K (the Q4_K superblock with a fifth-bit plane
+// qh[32] before qs) and Q6_K.  kQs: offset of qs in the superblock.
 template <int FMT> struct MmaFmt;
 template <> struct MmaFmt<kFmtQ4_K> {
     static constexpr int kUnitBytes = 144, kQs = 16;
-    static constexpr float kOff = 16.0f;
 };
 template <> struct MmaFmt<kFmtQ5_K> {
     static constexpr int kUnitBytes = 176, kQs = 48;
-    static constexpr float kOff = 32.0f;
 };
 template <> struct MmaFmt<kFmtQ6_K> {  // rows arrive in 240-byte per-lane windows (qg_rows.cuh)
     static constexpr int kUnitBytes = 240, kQs = 0;
-    static constexpr float kOff = 64.0f;
 };
+
 // n-tiles of 8 columns per mma (16 columns: two, sharing the unpacked A fragment)
 template <int BP> struct MmaNT {
     static constexpr int value = BP > 8 ? 2 : 1;
@@ -182,13 +181,12 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
 
 // One step: 32 rows (two 16-row tiles) x one superblock (unit j of the slice) at u0 (row stride
 // 144 B).  acc: C-fragment accumulators of the warp's rows; accM: this lane's row (row = lane),
-// the min term.  dtab: the warp's [8][32] table of D_j (scaled by 2^24 / 2^20 for the low /
-// high nibble halves), position (row % 8) * 4 + row / 8 so that rows g, g+8, g+16, g+24 are one
-// float4.
+// the min term.  dtab: the warp's [8][32] table of D_j, position (row % 8) * 4 + row / 8 so that
+// rows g, g+8, g+16, g+24 are one float4.
 // Q5_K: the A registers of one qs word w and its qh word hw (bytes l..l+3 of chunk c): the low
 // nibbles with their fifth bit (bit 2c of each qh byte) and the high nibbles with theirs (bit
-// 2c + 1), each merged into a byte as q = nibble | bit << 4 and read as normal fp16 pairs 32 + q
-// (exponent 5, q in mantissa bits 5-9): lo0 / hi0 = bytes 0 and 2, lo1 / hi1 = bytes 1 and 3.
+// 2c + 1), each merged into a byte as q = nibble | bit << 4 and read as the fp16 integer pairs q
+// (f16x2_code): lo0 / hi0 = bytes 0 and 2, lo1 / hi1 = bytes 1 and 3.
 template <int C>
 __device__ __forceinline__ void q5k_a_regs(uint32_t w, uint32_t hw, uint32_t &lo0, uint32_t &lo1,
                                            uint32_t &hi0, uint32_t &hi1)
@@ -197,10 +195,10 @@ __device__ __forceinline__ void q5k_a_regs(uint32_t w, uint32_t hw, uint32_t &lo
     const uint32_t t2 = (C == 0) ? hw << 3 : (C == 1) ? hw << 1 : (C == 2) ? hw >> 1 : hw >> 3;
     const uint32_t wl = (w & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
     const uint32_t wh = ((w >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
-    lo0 = ((wl << 5) & 0x03E003E0u) | 0x50005000u;
-    lo1 = (__umulhi(wl, 1u << 29) & 0x03E003E0u) | 0x50005000u;  // >> 3 on the FMA pipe
-    hi0 = ((wh << 5) & 0x03E003E0u) | 0x50005000u;
-    hi1 = (__umulhi(wh, 1u << 29) & 0x03E003E0u) | 0x50005000u;
+    lo0 = f16x2_code((wl & 0x001F001Fu) | kE1024);
+    lo1 = f16x2_code((__umulhi(wl, 1u << 24) & 0x001F001Fu) | kE1024);  // >> 8 on the FMA pipe
+    hi0 = f16x2_code((wh & 0x001F001Fu) | kE1024);
+    hi1 = f16x2_code((__umulhi(wh, 1u << 24) & 0x001F001Fu) | kE1024);
 }
 
 // Row of a 16-row tile that fragment row g (lane >> 2) of mma.m16n8k16 stands for, in the Q4_K /
@@ -237,7 +235,6 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
         *reinterpret_cast<uint32_t *>(&dd) = hdr.x;
         const float2 dm = __half22float2(dd);
         const float2 dscale = f2(dm.x, dm.x);
-        constexpr float O = MmaFmt<FMT>::kOff;
         const int pos = (lane & 7) * 4 + (lane >> 3);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -255,12 +252,11 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
             const float2 M = __fmul2_rn(f2(dm.y, dm.y), mm);
             dtab[(2 * c) * 32 + pos] = D.x;
             dtab[(2 * c + 1) * 32 + pos] = D.y;
-            // the min term and the code offset: -(M_j + O D_j) X_j
-            const float Mx = fmaf(O, D.x, M.x), My = fmaf(O, D.y, M.y);
+            // the min term: -M_j X_j
 #pragma unroll
             for (int b = 0; b < BP; ++b) {
-                accM[b] = fmaf(-Mx, xsum[rows_xsum_off<BP>(US, j, 2 * c, b)], accM[b]);
-                accM[b] = fmaf(-My, xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)], accM[b]);
+                accM[b] = fmaf(-M.x, xsum[rows_xsum_off<BP>(US, j, 2 * c, b)], accM[b]);
+                accM[b] = fmaf(-M.y, xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)], accM[b]);
             }
         }
     }
@@ -309,17 +305,17 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
                     default: q5k_a_regs<3>(wa, ha, l0, l2, h0, h2); q5k_a_regs<3>(wb, hb, l1, l3, h1, h3); break;
                     }
                 } else {
-                    // 16 + q: each nibble into mantissa bits 6-9 under exponent 4 (the shifts
-                    // right as multiply-highs on the FMA pipe)
-                    const uint32_t M4 = 0x03C003C0u, E4 = 0x4C004C00u;
-                    l0 = ((wa << 6) & M4) | E4;                      // low nibbles, bytes 0 and 2
-                    l1 = ((wb << 6) & M4) | E4;
-                    l2 = (__umulhi(wa, 1u << 30) & M4) | E4;         // low nibbles, bytes 1 and 3
-                    l3 = (__umulhi(wb, 1u << 30) & M4) | E4;
-                    h0 = ((wa << 2) & M4) | E4;                      // high nibbles, bytes 0 and 2
-                    h1 = ((wb << 2) & M4) | E4;
-                    h2 = (__umulhi(wa, 1u << 26) & M4) | E4;         // high nibbles, bytes 1 and 3
-                    h3 = (__umulhi(wb, 1u << 26) & M4) | E4;
+                    // the fp16 integers q: nibbles under the exponent of 1024, the offset
+                    // removed by one f16x2 FMA (word >> 8 as a multiply-high on the FMA pipe)
+                    const uint32_t va = __umulhi(wa, 1u << 24), vb = __umulhi(wb, 1u << 24);
+                    l0 = f16x2_code((wa & 0x000F000Fu) | kE1024);    // low nibbles, bytes 0 and 2
+                    l1 = f16x2_code((wb & 0x000F000Fu) | kE1024);
+                    l2 = f16x2_code((va & 0x000F000Fu) | kE1024);    // low nibbles, bytes 1 and 3
+                    l3 = f16x2_code((vb & 0x000F000Fu) | kE1024);
+                    h0 = f16x2_code16((wa & 0x00F000F0u) | kE1024);  // high nibbles, bytes 0 and 2
+                    h1 = f16x2_code16((wb & 0x00F000F0u) | kE1024);
+                    h2 = f16x2_code16((va & 0x00F000F0u) | kE1024);  // high nibbles, bytes 1 and 3
+                    h3 = f16x2_code16((vb & 0x00F000F0u) | kE1024);
                 }
 #pragma unroll
                 for (int nt = 0; nt < MmaNT<BP>::value; ++nt) {
@@ -350,8 +346,8 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 // thread (g, t) takes ql word 16hf + 8p + 4kk + t and qh word 32 + 8hf + 4kk + t of rows g and
 // g + 8 of the tile; their two high bits (bits 2p, 2p+1 for the low nibbles, 2p+4, 2p+5 for the
 // high ones) are merged byte-wise next to the nibbles and the 6-bit values q enter the MMA as the
-// normal fp16 numbers 64 + q.  The offsets are applied per group through the x sums:
-// sum (q - 32) x = sum (64 + q) x - 96 X_t.
+// fp16 integers q (f16x2_code).  The offset is applied per group through the x sums:
+// sum (q - 32) x = sum q x - 32 X_t.
 template <int BP>
 __device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
                                              int US, int j, float *dtab,
@@ -388,10 +384,10 @@ __device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf,
         for (int tg = 0; tg < 16; ++tg) {
             const float D = ds * (float)(int8_t)(scw[tg >> 2] >> (8 * (tg & 3)));
             dtab[tg * 32 + pos] = D;
-            // sum (q - 32) x = sum (64 + q) x - 96 X_t: the A codes carry the offset 64
+            // sum (q - 32) x = sum q x - 32 X_t
 #pragma unroll
             for (int b = 0; b < BP; ++b)
-                accM[b] = fmaf(D * -96.0f, xsum[rows_xsum_off<BP, 16>(US, j, tg, b)], accM[b]);
+                accM[b] = fmaf(D * -32.0f, xsum[rows_xsum_off<BP, 16>(US, j, tg, b)], accM[b]);
         }
     }
     __syncwarp();
@@ -431,12 +427,15 @@ __device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf,
                 const uint32_t wha = ((wa >> 4) & 0x0F0F0F0Fu) | (t2a & 0xF0F0F0F0u);
                 const uint32_t wlb = (wb & 0x0F0F0F0Fu) | (t1b & 0xF0F0F0F0u);
                 const uint32_t whb = ((wb >> 4) & 0x0F0F0F0Fu) | (t2b & 0xF0F0F0F0u);
-                // 64 + q: the 6-bit code into mantissa bits 4-9 under exponent 6
-                const uint32_t M6 = 0x03F003F0u, E6 = 0x54005400u;
-                const uint32_t l0 = ((wla * 16u) & M6) | E6, l1 = ((wlb * 16u) & M6) | E6;
-                const uint32_t l2 = (__umulhi(wla, 1u << 28) & M6) | E6, l3 = (__umulhi(wlb, 1u << 28) & M6) | E6;
-                const uint32_t h0 = ((wha * 16u) & M6) | E6, h1 = ((whb * 16u) & M6) | E6;
-                const uint32_t h2 = (__umulhi(wha, 1u << 28) & M6) | E6, h3 = (__umulhi(whb, 1u << 28) & M6) | E6;
+                // the fp16 integers q: the 6-bit codes under the exponent of 1024, the offset
+                // removed by one f16x2 FMA (bytes 1 and 3 through a multiply-high by 2^24)
+                constexpr uint32_t M6 = 0x003F003Fu;
+                const uint32_t l0 = f16x2_code((wla & M6) | kE1024), l1 = f16x2_code((wlb & M6) | kE1024);
+                const uint32_t l2 = f16x2_code((__umulhi(wla, 1u << 24) & M6) | kE1024);
+                const uint32_t l3 = f16x2_code((__umulhi(wlb, 1u << 24) & M6) | kE1024);
+                const uint32_t h0 = f16x2_code((wha & M6) | kE1024), h1 = f16x2_code((whb & M6) | kE1024);
+                const uint32_t h2 = f16x2_code((__umulhi(wha, 1u << 24) & M6) | kE1024);
+                const uint32_t h3 = f16x2_code((__umulhi(whb, 1u << 24) & M6) | kE1024);
                 const int tlo = 8 * hf + 2 * p + kk;
                 const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + tlo * 32 + 4 * g);
                 const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (tlo + 4) * 32 + 4 * g);

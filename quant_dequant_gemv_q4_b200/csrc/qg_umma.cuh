@@ -6,12 +6,11 @@
 //
 // The arithmetic is the factored form of the CUDA-core kernel,
 //   sum_i w_i x_i = sum_j [ d*sc_j * sum_{i in j} q_i x_i  -  dmin*m_j * sum_{i in j} x_i ],
-// with the inner sums on the tensor cores.  Each code q enters the MMA as the normal fp16 number
-// O + q (Q4_K: O = 16, Q5_K: O = 32; the code is masked into the mantissa under a fixed exponent),
-// so every product with x is exact, and sum (O + q) x = D_j is corrected by O * X_j afterwards.
-// (Codes carried as fp16 subnormals, as the CUDA-core kernels do, lose accumulation precision in
-// the tensor core: measured, the sums keep about 12 bits below the largest product then, 22 or more
-// with normal operands.)
+// with the inner sums on the tensor cores.  Each code q enters the MMA as the fp16 integer q
+// (qg_codes.cuh: one LOP3 under the exponent of 1024, one f16x2 FMA to take the 1024 out), so
+// every product with x is exact.  (Codes carried as fp16 subnormals, as the CUDA-core kernels do,
+// lose accumulation precision in the tensor core: measured, the sums keep about 12 bits below the
+// largest product then, 22 or more with normal operands.)
 //
 // Mapping.  A CTA owns a band of rows of one K slice, as in the CUDA-core kernel.  Its warps form
 // warpgroups of four; a warpgroup takes (row tile, K part) pairs, a row tile being 128 rows: warp
@@ -27,8 +26,8 @@
 //      memory): the two K-steps of sub-block 2c into one N = 16 accumulator tile, those of
 //      sub-block 2c + 1 into a second, and commits them to the slot's "done" mbarrier;
 //   3. before it writes the slot again, each warp waits for "done", reads its rows' accumulators
-//      back (tcgen05.ld) and adds d*sc_j * D_j; the terms (O*d*sc_j + dmin*m_j) * X_j (X_j from
-//      the staged x sums) are applied at unpack time.
+//      back (tcgen05.ld) and adds d*sc_j * D_j; the terms dmin*m_j * X_j (X_j from the staged x
+//      sums) are applied at unpack time.
 // No warp waits for the others of its group: only the issuing thread waits for the slot's four
 // arrivals, and a warp waits only for MMAs issued a chunk before it needs their slot.
 //
@@ -42,6 +41,7 @@
 
 #include <cuda.h>
 
+#include "qg_codes.cuh"
 #include "qg_device.cuh"
 #include "qg_rows.cuh"
 
@@ -485,26 +485,25 @@ __global__ void __launch_bounds__(UmmaWarps<BP>::value * 32, 1)
                 uint32_t r[32];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    // codes as normal fp16 O + q (Q4_K: 16 + q, exponent 4, q in mantissa bits 6-9;
-                    // Q5_K: 32 + q, exponent 5, q in bits 5-9): every product with x is exact and
-                    // the tensor core keeps its full accumulation precision on normal operands
+                    // codes as the fp16 integers q (qg_codes.cuh): every product with x is exact
+                    // and the tensor core keeps its full accumulation precision
                     uint32_t a0, a1, a2, a3;
                     if (FMT == kFmtQ4_K) {
-                        const uint32_t w = qw[i];
-                        a0 = ((w << 6) & 0x03C003C0u) | 0x4C004C00u;  // low nibbles of bytes 0, 2
-                        a1 = ((w >> 2) & 0x03C003C0u) | 0x4C004C00u;  // low nibbles of bytes 1, 3
-                        a2 = ((w << 2) & 0x03C003C0u) | 0x4C004C00u;  // high nibbles of bytes 0, 2
-                        a3 = ((w >> 6) & 0x03C003C0u) | 0x4C004C00u;  // high nibbles of bytes 1, 3
+                        const uint32_t w = qw[i], v = __umulhi(w, 1u << 24);  // v = w >> 8
+                        a0 = f16x2_code((w & 0x000F000Fu) | kE1024);    // low nibbles of bytes 0, 2
+                        a1 = f16x2_code((v & 0x000F000Fu) | kE1024);    // low nibbles of bytes 1, 3
+                        a2 = f16x2_code16((w & 0x00F000F0u) | kE1024);  // high nibbles of bytes 0, 2
+                        a3 = f16x2_code16((v & 0x00F000F0u) | kE1024);  // high nibbles of bytes 1, 3
                     } else {
                         const uint32_t hw = hq[i];
                         const uint32_t t1 = (c == 0) ? hw << 4 : (c == 1) ? hw << 2 : (c == 2) ? hw : hw >> 2;
                         const uint32_t t2 = (c == 0) ? hw << 3 : (c == 1) ? hw << 1 : (c == 2) ? hw >> 1 : hw >> 3;
                         const uint32_t wl = (qw[i] & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
                         const uint32_t wh = ((qw[i] >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
-                        a0 = ((wl << 5) & 0x03E003E0u) | 0x50005000u;
-                        a1 = ((wl >> 3) & 0x03E003E0u) | 0x50005000u;
-                        a2 = ((wh << 5) & 0x03E003E0u) | 0x50005000u;
-                        a3 = ((wh >> 3) & 0x03E003E0u) | 0x50005000u;
+                        a0 = f16x2_code((wl & 0x001F001Fu) | kE1024);
+                        a1 = f16x2_code((__umulhi(wl, 1u << 24) & 0x001F001Fu) | kE1024);
+                        a2 = f16x2_code((wh & 0x001F001Fu) | kE1024);
+                        a3 = f16x2_code((__umulhi(wh, 1u << 24) & 0x001F001Fu) | kE1024);
                     }
                     // K-step (s, h) with h = i / 4 holds columns 8 (2s + h) + 2 (i % 4) + {0, 1}: the
                     // weights (e, e+2) then (e+1, e+3) of the word
@@ -514,13 +513,12 @@ __global__ void __launch_bounds__(UmmaWarps<BP>::value * 32, 1)
                     r[16 + cl] = live ? a2 : 0u;
                     r[16 + cl + 1] = live ? a3 : 0u;
                 }
-                // the offset and min terms now: sum w x = d sc (D - O X) - dmin m X per sub-block
-                constexpr float O = (FMT == kFmtQ4_K) ? 16.0f : 32.0f;
+                // the min terms now: sum w x = d sc D - dmin m X per sub-block
 #pragma unroll
                 for (int b = 0; b < BP; ++b) {
                     const float X0 = xsum[(j * 8 + 2 * c) * BP + b];
                     const float X1 = xsum[(j * 8 + 2 * c + 1) * BP + b];
-                    acc[b] = fmaf(-fmaf(O, dsc1, dmm1), X1, fmaf(-fmaf(O, dsc0, dmm0), X0, acc[b]));
+                    acc[b] = fmaf(-dmm1, X1, fmaf(-dmm0, X0, acc[b]));
                 }
                 if (sl) { e10 = dsc0; e11 = dsc1; col1 = (j % U) * BP; }
                 else    { e00 = dsc0; e01 = dsc1; col0 = (j % U) * BP; }

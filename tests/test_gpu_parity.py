@@ -237,6 +237,8 @@ def test_full_size_workloads_sampled(dev, orc, wl, variant):
             continue  # the variants beyond the default are Q4_K's
         W, x = w.inputs(call)
         v = variant if call.fmt == Q4_K else 0
+        if call.B > 8 and v in (1, 2):
+            continue  # DIRECT and FACTORED take B <= 8
         y = gpu_gemv(dev, W, call.fmt, call.N, call.K, x, v)
         assert np.isfinite(y).all()
         rows = _sample_rows(call.N, rng)
