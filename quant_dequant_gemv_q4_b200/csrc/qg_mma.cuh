@@ -12,30 +12,31 @@
 // same tensor work, and the weights are unpacked once for all columns.  Products are exact
 // (integers up to 15 times fp16 x) and the sums are fp32, so the arithmetic is the factored form
 // of the CUDA-core kernel:
-//   sum_i w_i x_i = sum_j [ D_j * sum_{i in j} q_i x_i  -  M_j * sum_{i in j} x_i ],
-//   D_j = d*sc_j, M_j = dmin*m_j (exact in fp32), j = 32-weight sub-block.
+//   sum_i w_i x_i = d * sum_j sc_j sum_{i in j} q_i x_i  -  sum_j M_j * sum_{i in j} x_i,
+//   M_j = dmin*m_j (exact in fp32), j = 32-weight sub-block.
 //
 // Mapping.  The grid, row bands, (row group, K part) pairs and the per-warp ring of 2-D TMA
 // boxes (32 rows x one 144-byte superblock) are those of the CUDA-core kernel (qg_rows.cuh).  Per
 // step a warp multiplies its 32 rows as two 16-row tiles:
 //   A fragment (rows g and g+8 of a tile, lane = 4g + t): word 2t+h of the 32-byte chunk c of the
-//     row; its low nibbles of bytes 0 and 2 (sub-block 2c) are masked under the exponent of 1024
-//     (one LOP3: the fp16 pair 1024 + q, q in mantissa bits 0-3) and one packed fp16 FMA takes
-//     the 1024 back out, leaving the fp16 integers q exactly; its high nibbles (sub-block 2c+1)
-//     give 1024 + 16 q the same way, and the FMA scales by 1/16 as it subtracts 64; word >> 8
-//     gives bytes 1 and 3.  So one 32-bit word feeds four A registers through four LOP3 (ALU
-//     pipe), one multiply-high (the shift) and four f16x2 FMAs (FMA pipe).  Normal operands keep
-//     the tensor core's full accumulation precision (with codes as fp16 subnormals its sums keep
-//     only about 12 bits below the largest product, which measured up to 0.95 of the error bound
-//     with massive activations), and codes without an offset keep every product as small as the
-//     weight itself.
+//     row; its low nibbles of bytes 0 and 2 (sub-block 2c) are masked as the fp16 subnormal pair
+//     q 2^-24 and multiplied (one f16x2 multiply) into normal fp16 numbers; its high nibbles
+//     (sub-block 2c+1) stay in place as q 2^-20 and are multiplied likewise; word >> 8 gives
+//     bytes 1 and 3.  So one 32-bit word feeds four A registers through four LOP3 (ALU pipe), one
+//     multiply-high (the shift) and four f16x2 multiplies (FMA pipe).  Normal operands keep the
+//     tensor core's full accumulation precision (on subnormal codes its sums keep only about 12
+//     bits below the largest product, which measured up to 0.95 of the error bound with massive
+//     activations).  The multiplier is a power of two (Q4_K, Q6_K) or the sub-block scale times
+//     a power of two (Q5_K), see mma_q4k_step / mma_q5k_step.
 //   B fragment: x in the matching order, staged once per CTA (mma_stage_x).
-//   C fragment: rows g, g+8 x columns 2t, 2t+1, fresh per (chunk, tile, nibble half), then scaled
-//     by D_j of its row and added to the warp's accumulators.
+//   C fragment: rows g, g+8 x columns 2t, 2t+1, scaled by the sub-block's d sc_j (Q4_K), or the
+//     superblock's d (Q5_K), of its row and added to the warp's accumulators.
 // The scales come from a per-warp table: lane l decodes row l's header (as in the CUDA-core
-// kernel), writes D_j for its row, and folds -M_j * sum(x over j) into its own per-row sum.
-// Q5_K and Q6_K keep this skeleton; their high-bit planes are merged into the A words byte-wise
-// (q5k_a_regs, mma_q6k_step), and Q6_K scales each 16-weight k-tile by its own group's D_t.
+// kernel), writes its row's entries, and folds -M_j * sum(x over j) into its own per-row sum.
+// Q5_K keeps this skeleton; its fifth-bit plane is merged into the A words byte-wise
+// (q5k_a_codes).  Q6_K (mma_q6k_step) has signed 8-bit scales whose products with the 6-bit codes
+// do not fit fp16 exactly: its codes enter as q 2^-10 and each 16-weight k-tile's C fragments are
+// scaled by its own group's d sc_t 2^10.
 #pragma once
 
 #include "qg_codes.cuh"
@@ -180,25 +181,40 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
 }
 
 // One step: 32 rows (two 16-row tiles) x one superblock (unit j of the slice) at u0 (row stride
-// 144 B).  acc: C-fragment accumulators of the warp's rows; accM: this lane's row (row = lane),
-// the min term.  dtab: the warp's [8][32] table of D_j, position (row % 8) * 4 + row / 8 so that
-// rows g, g+8, g+16, g+24 are one float4.
-// Q5_K: the A registers of one qs word w and its qh word hw (bytes l..l+3 of chunk c): the low
-// nibbles with their fifth bit (bit 2c of each qh byte) and the high nibbles with theirs (bit
-// 2c + 1), each merged into a byte as q = nibble | bit << 4 and read as the fp16 integer pairs q
-// (f16x2_code): lo0 / hi0 = bytes 0 and 2, lo1 / hi1 = bytes 1 and 3.
+// 144 B; Q5_K 176 B).  acc: C-fragment accumulators of the warp's rows; accM: this lane's row
+// (row = lane), the min term.  Rows are placed in the warp's table dtab at position
+// (row % 8) * 4 + row / 8, so that rows g, g+8, g+16, g+24 are one run.
+//
+// Q4_K (mma_q4k_step): the codes enter the MMA as the normal fp16 numbers q * 2^-10 (low nibbles
+// masked as q * 2^-24 and multiplied by 2^14, high nibbles left in place as q * 2^-20 and
+// multiplied by 2^10).  A C fragment sums one sub-block's half of a chunk for one tile (two MMAs)
+// and is scaled by d * sc_j * 2^10 of its row (dtab: [8 sub-blocks][32 positions] floats).
+//
+// Q5_K (mma_q5k_step): the sub-block scales are folded into the A operand.  A code q of sub-block
+// j enters as q * sc_j * 2^-14 (the masked subnormal q * 2^-24 times the fp16 pair sc_j * 2^10;
+// dtab holds those pairs, [4 chunks][32 positions] x (low, high)); q * sc_j <= 31 * 63 < 2^11, so
+// the product is exact and normal (or zero).  The C fragments then sum a whole superblock and are
+// scaled once per step by d * 2^14 of their row:
+//   sum_i w_i x_i = d * 2^14 * sum_i (q_i sc_j(i) 2^-14) x_i  -  sum_j dmin m_j X_j.
+// Measured on B200: folding saves Q5_K about 1.5 us per 17408 x 5120 call at B = 8 (its A words
+// cost more instructions, which folding offsets), while for Q4_K the longer MMA accumulation
+// chains cost more than the saved scaling instructions (0.5 us slower at B = 8).
+// Q5_K: the A codes of one qs word w and its qh word hw (bytes l..l+3 of chunk c): the low nibbles
+// with their fifth bit (bit 2c of each qh byte) and the high nibbles with theirs (bit 2c + 1), each
+// merged into a byte as q = nibble | bit << 4, masked as subnormals q * 2^-24: lo0 / hi0 = bytes 0
+// and 2, lo1 / hi1 = bytes 1 and 3.
 template <int C>
-__device__ __forceinline__ void q5k_a_regs(uint32_t w, uint32_t hw, uint32_t &lo0, uint32_t &lo1,
-                                           uint32_t &hi0, uint32_t &hi1)
+__device__ __forceinline__ void q5k_a_codes(uint32_t w, uint32_t hw, uint32_t &lo0, uint32_t &lo1,
+                                            uint32_t &hi0, uint32_t &hi1)
 {
     const uint32_t t1 = (C == 0) ? hw << 4 : (C == 1) ? hw << 2 : (C == 2) ? hw : hw >> 2;
     const uint32_t t2 = (C == 0) ? hw << 3 : (C == 1) ? hw << 1 : (C == 2) ? hw >> 1 : hw >> 3;
     const uint32_t wl = (w & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
     const uint32_t wh = ((w >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
-    lo0 = f16x2_code((wl & 0x001F001Fu) | kE1024);
-    lo1 = f16x2_code((__umulhi(wl, 1u << 24) & 0x001F001Fu) | kE1024);  // >> 8 on the FMA pipe
-    hi0 = f16x2_code((wh & 0x001F001Fu) | kE1024);
-    hi1 = f16x2_code((__umulhi(wh, 1u << 24) & 0x001F001Fu) | kE1024);
+    lo0 = wl & 0x001F001Fu;
+    lo1 = __umulhi(wl, 1u << 24) & 0x001F001Fu;  // >> 8 on the FMA pipe
+    hi0 = wh & 0x001F001Fu;
+    hi1 = __umulhi(wh, 1u << 24) & 0x001F001Fu;
 }
 
 // Row of a 16-row tile that fragment row g (lane >> 2) of mma.m16n8k16 stands for, in the Q4_K /
@@ -213,12 +229,13 @@ __device__ __forceinline__ int mma_frag_row(int g)
     return (FMT == kFmtQ6_K) ? g : 2 * (g & 3) + (g >> 2);
 }
 
-template <int BP, int FMT = kFmtQ4_K>
+template <int BP>
 __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
                                              int US, int j, float *dtab,
                                              float (&acc)[2][MmaNT<BP>::value][4], float (&accM)[BP],
                                              int lane)
 {
+    constexpr int FMT = kFmtQ4_K;
     constexpr int UB = MmaFmt<FMT>::kUnitBytes;
     constexpr int QS = MmaFmt<FMT>::kQs;
     const int g = lane >> 2, t = lane & 3;
@@ -250,8 +267,8 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
                                          f2(-8388608.0f, -8388608.0f));
             const float2 D = __fmul2_rn(dscale, sc);
             const float2 M = __fmul2_rn(f2(dm.y, dm.y), mm);
-            dtab[(2 * c) * 32 + pos] = D.x;
-            dtab[(2 * c + 1) * 32 + pos] = D.y;
+            dtab[(2 * c) * 32 + pos] = D.x * 1024.0f;  // the codes are q 2^-10
+            dtab[(2 * c + 1) * 32 + pos] = D.y * 1024.0f;
             // the min term: -M_j X_j
 #pragma unroll
             for (int b = 0; b < BP; ++b) {
@@ -281,12 +298,6 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
             const uint8_t *rowA = u0 + (tile * 16 + pr) * UB + QS + 32 * c + 8 * t;
             const uint2 wA = *reinterpret_cast<const uint2 *>(rowA);           // row tile*16 + pr
             const uint2 wB = *reinterpret_cast<const uint2 *>(rowA + 8 * UB);  // row tile*16 + pr + 8
-            uint2 qhA = make_uint2(0u, 0u), qhB = make_uint2(0u, 0u);  // Q5_K: qh words 2t, 2t+1
-            if (FMT == kFmtQ5_K) {
-                const uint8_t *qhp = u0 + (tile * 16 + pr) * UB + 16 + 8 * t;
-                qhA = *reinterpret_cast<const uint2 *>(qhp);
-                qhB = *reinterpret_cast<const uint2 *>(qhp + 8 * UB);
-            }
             float cl[MmaNT<BP>::value][4], ch[MmaNT<BP>::value][4];
 #pragma unroll
             for (int nt = 0; nt < MmaNT<BP>::value; ++nt)
@@ -296,26 +307,19 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
             for (int h = 0; h < 2; ++h) {
                 const uint32_t wa = h ? wA.y : wA.x, wb = h ? wB.y : wB.x;
                 uint32_t l0, l1, l2, l3, h0, h1, h2, h3;
-                if (FMT == kFmtQ5_K) {
-                    const uint32_t ha = h ? qhA.y : qhA.x, hb = h ? qhB.y : qhB.x;
-                    switch (c) {  // c is a compile-time constant after unrolling
-                    case 0: q5k_a_regs<0>(wa, ha, l0, l2, h0, h2); q5k_a_regs<0>(wb, hb, l1, l3, h1, h3); break;
-                    case 1: q5k_a_regs<1>(wa, ha, l0, l2, h0, h2); q5k_a_regs<1>(wb, hb, l1, l3, h1, h3); break;
-                    case 2: q5k_a_regs<2>(wa, ha, l0, l2, h0, h2); q5k_a_regs<2>(wb, hb, l1, l3, h1, h3); break;
-                    default: q5k_a_regs<3>(wa, ha, l0, l2, h0, h2); q5k_a_regs<3>(wb, hb, l1, l3, h1, h3); break;
-                    }
-                } else {
-                    // the fp16 integers q: nibbles under the exponent of 1024, the offset
-                    // removed by one f16x2 FMA (word >> 8 as a multiply-high on the FMA pipe)
+                {
+                    // low nibbles masked as q 2^-24, high nibbles left in place as q 2^-20, then
+                    // made the normal fp16 numbers q 2^-10 (word >> 8 as a multiply-high on the
+                    // FMA pipe for bytes 1 and 3)
                     const uint32_t va = __umulhi(wa, 1u << 24), vb = __umulhi(wb, 1u << 24);
-                    l0 = f16x2_code((wa & 0x000F000Fu) | kE1024);    // low nibbles, bytes 0 and 2
-                    l1 = f16x2_code((wb & 0x000F000Fu) | kE1024);
-                    l2 = f16x2_code((va & 0x000F000Fu) | kE1024);    // low nibbles, bytes 1 and 3
-                    l3 = f16x2_code((vb & 0x000F000Fu) | kE1024);
-                    h0 = f16x2_code16((wa & 0x00F000F0u) | kE1024);  // high nibbles, bytes 0 and 2
-                    h1 = f16x2_code16((wb & 0x00F000F0u) | kE1024);
-                    h2 = f16x2_code16((va & 0x00F000F0u) | kE1024);  // high nibbles, bytes 1 and 3
-                    h3 = f16x2_code16((vb & 0x00F000F0u) | kE1024);
+                    l0 = f16x2_mul(wa & 0x000F000Fu, kF16x2_2p14);  // low nibbles, bytes 0 and 2
+                    l1 = f16x2_mul(wb & 0x000F000Fu, kF16x2_2p14);
+                    l2 = f16x2_mul(va & 0x000F000Fu, kF16x2_2p14);  // low nibbles, bytes 1 and 3
+                    l3 = f16x2_mul(vb & 0x000F000Fu, kF16x2_2p14);
+                    h0 = f16x2_mul(wa & 0x00F000F0u, kF16x2_2p10);  // high nibbles, bytes 0 and 2
+                    h1 = f16x2_mul(wb & 0x00F000F0u, kF16x2_2p10);
+                    h2 = f16x2_mul(va & 0x00F000F0u, kF16x2_2p10);  // high nibbles, bytes 1 and 3
+                    h3 = f16x2_mul(vb & 0x00F000F0u, kF16x2_2p10);
                 }
 #pragma unroll
                 for (int nt = 0; nt < MmaNT<BP>::value; ++nt) {
@@ -338,6 +342,160 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
     }
 }
 
+template <int BP>
+__device__ __forceinline__ void mma_q5k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
+                                             int US, int j, float *dtab,
+                                             float (&acc)[2][MmaNT<BP>::value][4], float (&accM)[BP],
+                                             int lane)
+{
+    constexpr int FMT = kFmtQ5_K;
+    constexpr int UB = MmaFmt<FMT>::kUnitBytes;
+    constexpr int QS = MmaFmt<FMT>::kQs;
+    constexpr int NT = MmaNT<BP>::value;
+    constexpr int SPLIT = (NT == 1) ? 2 : 1;  // C fragments per (tile, n-tile): low / high codes
+    const int g = lane >> 2, t = lane & 3;
+    const int pr = mma_frag_row<FMT>(g);  // the tile row of fragment row g
+    uint2 *mtab = reinterpret_cast<uint2 *>(dtab);
+    float dsh;  // d * 2^14 of row `lane`
+    {
+        // header of row `lane`: the GGML get_scale_min_k4 table decoded with 32-bit masks (byte k
+        // of each word = sub-block k or k+4), d and dmin exact in fp32
+        const uint4 hdr = *reinterpret_cast<const uint4 *>(u0 + lane * UB);
+        const uint32_t SC_lo = hdr.y & 0x3F3F3F3Fu;
+        const uint32_t MM_lo = hdr.z & 0x3F3F3F3Fu;
+        const uint32_t SC_hi = (hdr.w & 0x0F0F0F0Fu) | ((hdr.y >> 2) & 0x30303030u);
+        const uint32_t MM_hi = ((hdr.w >> 4) & 0x0F0F0F0Fu) | ((hdr.z >> 2) & 0x30303030u);
+        __half2 dd;
+        *reinterpret_cast<uint32_t *>(&dd) = hdr.x;
+        const float2 dm = __half22float2(dd);
+        dsh = dm.x * 16384.0f;
+        const int pos = (lane & 7) * 4 + (lane >> 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t scw = c < 2 ? SC_lo : SC_hi;
+            const uint32_t mmw = c < 2 ? MM_lo : MM_hi;
+            const uint32_t sel = 0x7650u + 2u * (c & 1);
+            // 6-bit integers to float through the 2^23 mantissa: (2^23 + v) - 2^23
+            const float2 sc = __fadd2_rn(f2(__uint_as_float(__byte_perm(scw, 0x4B000000u, sel)),
+                                            __uint_as_float(__byte_perm(scw, 0x4B000000u, sel + 1))),
+                                         f2(-8388608.0f, -8388608.0f));
+            const float2 mm = __fadd2_rn(f2(__uint_as_float(__byte_perm(mmw, 0x4B000000u, sel)),
+                                            __uint_as_float(__byte_perm(mmw, 0x4B000000u, sel + 1))),
+                                         f2(-8388608.0f, -8388608.0f));
+            mtab[c * 32 + pos] = make_uint2(f16x2_dup(sc.x * 1024.0f), f16x2_dup(sc.y * 1024.0f));
+            const float2 M = __fmul2_rn(f2(dm.y, dm.y), mm);
+            // the min term: -M_j X_j
+#pragma unroll
+            for (int b = 0; b < BP; ++b) {
+                accM[b] = fmaf(-M.x, xsum[rows_xsum_off<BP>(US, j, 2 * c, b)], accM[b]);
+                accM[b] = fmaf(-M.y, xsum[rows_xsum_off<BP>(US, j, 2 * c + 1, b)], accM[b]);
+            }
+        }
+    }
+    __syncwarp();
+    // the superblock's sums times d * 2^14 of their rows (rows pr and pr + 8 of each tile)
+    float C[2][NT][SPLIT][4];
+    auto zero_c = [&]() {
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int sp = 0; sp < SPLIT; ++sp)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) C[tile][nt][sp][k] = 0.0f;
+    };
+    auto fold_c = [&]() {
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const float dA = __shfl_sync(0xffffffffu, dsh, tile * 16 + pr);
+            const float dB = __shfl_sync(0xffffffffu, dsh, tile * 16 + pr + 8);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int sp = 0; sp < SPLIT; ++sp) {
+                    acc[tile][nt][0] = fmaf(dA, C[tile][nt][sp][0], acc[tile][nt][0]);
+                    acc[tile][nt][2] = fmaf(dB, C[tile][nt][sp][2], acc[tile][nt][2]);
+                    if (BP > 1) {
+                        acc[tile][nt][1] = fmaf(dA, C[tile][nt][sp][1], acc[tile][nt][1]);
+                        acc[tile][nt][3] = fmaf(dB, C[tile][nt][sp][3], acc[tile][nt][3]);
+                    }
+                }
+        }
+    };
+    // at 16 columns (two n-tiles sharing the A registers) the C fragments are folded per chunk,
+    // which keeps them out of the registers live across the step
+    constexpr bool kFoldPerChunk = (NT == 2);
+    zero_c();
+    // n-tile nt covers columns 8nt .. 8nt+7 (one tile for BP <= 8); lane g supplies column 8nt + g
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (kFoldPerChunk && c > 0) zero_c();
+        uint2 xb[NT][2][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = (BP > 8) ? 8 * nt + g : g % BP;
+                    xb[nt][lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
+                }
+        // multipliers of rows pr, pr + 8 (tile 0) and pr + 16, pr + 24 (tile 1): (low, high) pairs
+        const uint4 m0 = *reinterpret_cast<const uint4 *>(mtab + c * 32 + 4 * pr);
+        const uint4 m1 = *reinterpret_cast<const uint4 *>(mtab + c * 32 + 4 * pr + 2);
+        // the A words of both tiles: rows tile*16 + pr and tile*16 + pr + 8
+        uint2 wA[2], wB[2], qhA[2], qhB[2];
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const uint8_t *rowA = u0 + (tile * 16 + pr) * UB + QS + 32 * c + 8 * t;
+            wA[tile] = *reinterpret_cast<const uint2 *>(rowA);
+            wB[tile] = *reinterpret_cast<const uint2 *>(rowA + 8 * UB);
+            const uint8_t *qhp = u0 + (tile * 16 + pr) * UB + 16 + 8 * t;  // qh words 2t, 2t+1
+            qhA[tile] = *reinterpret_cast<const uint2 *>(qhp);
+            qhB[tile] = *reinterpret_cast<const uint2 *>(qhp + 8 * UB);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            // A registers of both tiles, then their MMAs interleaved so that no MMA waits on the
+            // one just issued
+            uint32_t A[2][2][4];  // [tile][low / high codes][register]
+#pragma unroll
+            for (int tile = 0; tile < 2; ++tile) {
+                const uint4 m = tile ? m1 : m0;
+                const uint32_t wa = h ? wA[tile].y : wA[tile].x, wb = h ? wB[tile].y : wB[tile].x;
+                uint32_t l0, l1, l2, l3, h0, h1, h2, h3;  // masked codes (subnormal fp16 pairs)
+                const uint32_t ha = h ? qhA[tile].y : qhA[tile].x, hb = h ? qhB[tile].y : qhB[tile].x;
+                switch (c) {  // c is a compile-time constant after unrolling
+                case 0: q5k_a_codes<0>(wa, ha, l0, l2, h0, h2); q5k_a_codes<0>(wb, hb, l1, l3, h1, h3); break;
+                case 1: q5k_a_codes<1>(wa, ha, l0, l2, h0, h2); q5k_a_codes<1>(wb, hb, l1, l3, h1, h3); break;
+                case 2: q5k_a_codes<2>(wa, ha, l0, l2, h0, h2); q5k_a_codes<2>(wb, hb, l1, l3, h1, h3); break;
+                default: q5k_a_codes<3>(wa, ha, l0, l2, h0, h2); q5k_a_codes<3>(wb, hb, l1, l3, h1, h3); break;
+                }
+                // times sc * 2^10: q sc 2^-14, exact and normal
+                A[tile][0][0] = f16x2_mul(l0, m.x);
+                A[tile][0][2] = f16x2_mul(l2, m.x);
+                A[tile][0][1] = f16x2_mul(l1, m.z);
+                A[tile][0][3] = f16x2_mul(l3, m.z);
+                A[tile][1][0] = f16x2_mul(h0, m.y);
+                A[tile][1][2] = f16x2_mul(h2, m.y);
+                A[tile][1][1] = f16x2_mul(h1, m.w);
+                A[tile][1][3] = f16x2_mul(h3, m.w);
+            }
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int tile = 0; tile < 2; ++tile)
+                        mma_16816(C[tile][nt][lh * (SPLIT - 1)], A[tile][lh][0], A[tile][lh][1], A[tile][lh][2],
+                                  A[tile][lh][3], xb[nt][lh][h].x, xb[nt][lh][h].y);
+        }
+        if (kFoldPerChunk) fold_c();
+    }
+    if (!kFoldPerChunk) fold_c();
+}
+
 // One Q6_K step: 32 rows x one superblock from the warp's per-lane windows at u0 (window of row
 // r at u0 + 240 r; its superblock starts o_r = (m_r * 210) mod 16 bytes in, m_r its superblock
 // index in the tensor).  Chunk c = 2hf + p is ql[64hf + 32p ..]; its k-tile kk (words 4kk .. 4kk+3)
@@ -346,8 +504,8 @@ __device__ __forceinline__ void mma_q4k_step(const uint8_t *u0, const uint2 *xf,
 // thread (g, t) takes ql word 16hf + 8p + 4kk + t and qh word 32 + 8hf + 4kk + t of rows g and
 // g + 8 of the tile; their two high bits (bits 2p, 2p+1 for the low nibbles, 2p+4, 2p+5 for the
 // high ones) are merged byte-wise next to the nibbles and the 6-bit values q enter the MMA as the
-// fp16 integers q (f16x2_code).  The offset is applied per group through the x sums:
-// sum (q - 32) x = sum q x - 32 X_t.
+// normal fp16 numbers q 2^-10 (the D_t table holds d sc_t 2^10).  The offset is applied per group
+// through the x sums: sum (q - 32) x = sum q x - 32 X_t.
 template <int BP>
 __device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf, const float *xsum,
                                              int US, int j, float *dtab,
@@ -383,7 +541,7 @@ __device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf,
 #pragma unroll
         for (int tg = 0; tg < 16; ++tg) {
             const float D = ds * (float)(int8_t)(scw[tg >> 2] >> (8 * (tg & 3)));
-            dtab[tg * 32 + pos] = D;
+            dtab[tg * 32 + pos] = D * 1024.0f;  // the codes are q 2^-10
             // sum (q - 32) x = sum q x - 32 X_t
 #pragma unroll
             for (int b = 0; b < BP; ++b)
@@ -427,15 +585,15 @@ __device__ __forceinline__ void mma_q6k_step(const uint8_t *u0, const uint2 *xf,
                 const uint32_t wha = ((wa >> 4) & 0x0F0F0F0Fu) | (t2a & 0xF0F0F0F0u);
                 const uint32_t wlb = (wb & 0x0F0F0F0Fu) | (t1b & 0xF0F0F0F0u);
                 const uint32_t whb = ((wb >> 4) & 0x0F0F0F0Fu) | (t2b & 0xF0F0F0F0u);
-                // the fp16 integers q: the 6-bit codes under the exponent of 1024, the offset
-                // removed by one f16x2 FMA (bytes 1 and 3 through a multiply-high by 2^24)
+                // the 6-bit codes masked as subnormals q 2^-24 (bytes 1 and 3 through a
+                // multiply-high by 2^24), then made the normal fp16 numbers q 2^-10 (qg_codes.cuh)
                 constexpr uint32_t M6 = 0x003F003Fu;
-                const uint32_t l0 = f16x2_code((wla & M6) | kE1024), l1 = f16x2_code((wlb & M6) | kE1024);
-                const uint32_t l2 = f16x2_code((__umulhi(wla, 1u << 24) & M6) | kE1024);
-                const uint32_t l3 = f16x2_code((__umulhi(wlb, 1u << 24) & M6) | kE1024);
-                const uint32_t h0 = f16x2_code((wha & M6) | kE1024), h1 = f16x2_code((whb & M6) | kE1024);
-                const uint32_t h2 = f16x2_code((__umulhi(wha, 1u << 24) & M6) | kE1024);
-                const uint32_t h3 = f16x2_code((__umulhi(whb, 1u << 24) & M6) | kE1024);
+                const uint32_t l0 = f16x2_mul(wla & M6, kF16x2_2p14), l1 = f16x2_mul(wlb & M6, kF16x2_2p14);
+                const uint32_t l2 = f16x2_mul(__umulhi(wla, 1u << 24) & M6, kF16x2_2p14);
+                const uint32_t l3 = f16x2_mul(__umulhi(wlb, 1u << 24) & M6, kF16x2_2p14);
+                const uint32_t h0 = f16x2_mul(wha & M6, kF16x2_2p14), h1 = f16x2_mul(whb & M6, kF16x2_2p14);
+                const uint32_t h2 = f16x2_mul(__umulhi(wha, 1u << 24) & M6, kF16x2_2p14);
+                const uint32_t h3 = f16x2_mul(__umulhi(whb, 1u << 24) & M6, kF16x2_2p14);
                 const int tlo = 8 * hf + 2 * p + kk;
                 const float4 Dlo = *reinterpret_cast<const float4 *>(dtab + tlo * 32 + 4 * g);
                 const float4 Dhi = *reinterpret_cast<const float4 *>(dtab + (tlo + 4) * 32 + 4 * g);
@@ -616,8 +774,10 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
                 mma_q6k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
                                  lane, a, row0, ucol0 + j, a.w[second ? MATS - 1 : 0]);
             } else {
-                mma_q4k_step<BP, FMT>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc,
-                                      accM, lane);
+                if (FMT == kFmtQ5_K)
+                    mma_q5k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM, lane);
+                else
+                    mma_q4k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM, lane);
             }
             __syncwarp();
             if (step + kRowsStages < nsteps) {

@@ -6,9 +6,9 @@
 //
 // The arithmetic is the factored form of the CUDA-core kernel,
 //   sum_i w_i x_i = sum_j [ d*sc_j * sum_{i in j} q_i x_i  -  dmin*m_j * sum_{i in j} x_i ],
-// with the inner sums on the tensor cores.  Each code q enters the MMA as the fp16 integer q
-// (qg_codes.cuh: one LOP3 under the exponent of 1024, one f16x2 FMA to take the 1024 out), so
-// every product with x is exact.  (Codes carried as fp16 subnormals, as the CUDA-core kernels do,
+// with the inner sums on the tensor cores.  Each code q enters the MMA as the normal fp16 number
+// q 2^-10 (qg_codes.cuh: one LOP3 leaves the subnormal q 2^-24, one f16x2 multiply by a power of two
+// normalises it), so every product with x is exact.  (Codes carried as fp16 subnormals, as the CUDA-core kernels do,
 // lose accumulation precision in the tensor core: measured, the sums keep about 12 bits below the
 // largest product then, 22 or more with normal operands.)
 //
@@ -485,25 +485,25 @@ __global__ void __launch_bounds__(UmmaWarps<BP>::value * 32, 1)
                 uint32_t r[32];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    // codes as the fp16 integers q (qg_codes.cuh): every product with x is exact
-                    // and the tensor core keeps its full accumulation precision
+                    // codes as the normal fp16 numbers q 2^-10 (qg_codes.cuh): every product with
+                    // x is exact and the tensor core keeps its full accumulation precision
                     uint32_t a0, a1, a2, a3;
                     if (FMT == kFmtQ4_K) {
                         const uint32_t w = qw[i], v = __umulhi(w, 1u << 24);  // v = w >> 8
-                        a0 = f16x2_code((w & 0x000F000Fu) | kE1024);    // low nibbles of bytes 0, 2
-                        a1 = f16x2_code((v & 0x000F000Fu) | kE1024);    // low nibbles of bytes 1, 3
-                        a2 = f16x2_code16((w & 0x00F000F0u) | kE1024);  // high nibbles of bytes 0, 2
-                        a3 = f16x2_code16((v & 0x00F000F0u) | kE1024);  // high nibbles of bytes 1, 3
+                        a0 = f16x2_mul(w & 0x000F000Fu, kF16x2_2p14);  // low nibbles of bytes 0, 2
+                        a1 = f16x2_mul(v & 0x000F000Fu, kF16x2_2p14);  // low nibbles of bytes 1, 3
+                        a2 = f16x2_mul(w & 0x00F000F0u, kF16x2_2p10);  // high nibbles of bytes 0, 2
+                        a3 = f16x2_mul(v & 0x00F000F0u, kF16x2_2p10);  // high nibbles of bytes 1, 3
                     } else {
                         const uint32_t hw = hq[i];
                         const uint32_t t1 = (c == 0) ? hw << 4 : (c == 1) ? hw << 2 : (c == 2) ? hw : hw >> 2;
                         const uint32_t t2 = (c == 0) ? hw << 3 : (c == 1) ? hw << 1 : (c == 2) ? hw >> 1 : hw >> 3;
                         const uint32_t wl = (qw[i] & 0x0F0F0F0Fu) | (t1 & 0xF0F0F0F0u);
                         const uint32_t wh = ((qw[i] >> 4) & 0x0F0F0F0Fu) | (t2 & 0xF0F0F0F0u);
-                        a0 = f16x2_code((wl & 0x001F001Fu) | kE1024);
-                        a1 = f16x2_code((__umulhi(wl, 1u << 24) & 0x001F001Fu) | kE1024);
-                        a2 = f16x2_code((wh & 0x001F001Fu) | kE1024);
-                        a3 = f16x2_code((__umulhi(wh, 1u << 24) & 0x001F001Fu) | kE1024);
+                        a0 = f16x2_mul(wl & 0x001F001Fu, kF16x2_2p14);
+                        a1 = f16x2_mul(__umulhi(wl, 1u << 24) & 0x001F001Fu, kF16x2_2p14);
+                        a2 = f16x2_mul(wh & 0x001F001Fu, kF16x2_2p14);
+                        a3 = f16x2_mul(__umulhi(wh, 1u << 24) & 0x001F001Fu, kF16x2_2p14);
                     }
                     // K-step (s, h) with h = i / 4 holds columns 8 (2s + h) + 2 (i % 4) + {0, 1}: the
                     // weights (e, e+2) then (e+1, e+3) of the word
@@ -520,8 +520,9 @@ __global__ void __launch_bounds__(UmmaWarps<BP>::value * 32, 1)
                     const float X1 = xsum[(j * 8 + 2 * c + 1) * BP + b];
                     acc[b] = fmaf(-dmm1, X1, fmaf(-dmm0, X0, acc[b]));
                 }
-                if (sl) { e10 = dsc0; e11 = dsc1; col1 = (j % U) * BP; }
-                else    { e00 = dsc0; e01 = dsc1; col0 = (j % U) * BP; }
+                // the accumulators hold sums of (q 2^-10) x
+                if (sl) { e10 = dsc0 * 1024.0f; e11 = dsc1 * 1024.0f; col1 = (j % U) * BP; }
+                else    { e00 = dsc0 * 1024.0f; e01 = dsc1 * 1024.0f; col0 = (j % U) * BP; }
                 tmem_st32(lane_off + wg_col + 32u * sl, r);
                 tmem_wait_st();
                 tc_fence_before();
