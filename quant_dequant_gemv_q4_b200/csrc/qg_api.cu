@@ -262,7 +262,9 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
             NW = MmaWarpsF<kFmtQ6_K, 1>::value;
             tab_floats = std::max(512, 32 * BP);
         } else {
-            LB = (fmt == kFmtQ5_K) ? MmaFmt<kFmtQ5_K>::kUnitBytes : MmaFmt<kFmtQ4_K>::kUnitBytes;
+            LB = (fmt == kFmtQ5_K)     ? MmaFmt<kFmtQ5_K>::kUnitBytes
+                 : (fmt == kFmtIQ4_XS) ? MmaFmt<kFmtIQ4_XS>::kUnitBytes
+                                       : MmaFmt<kFmtQ4_K>::kUnitBytes;
             NW = BP >= 16 ? MmaWarps<16>::value : BP >= 8 ? MmaWarps<8>::value : MmaWarps<1>::value;
             tab_floats = std::max(256, 32 * BP);
         }
@@ -281,7 +283,7 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     // group, K part) pairs to keep every warp streaming).  Ties: fewer steps, then fewer slices.
     // The tensor-core kernel only takes slicings with at most one pair per warp.  If no slicing
     // qualifies, the one with the most busy lanes.
-    const int UB = tensor ? (fmt == kFmtQ5_K ? 176 : fmt == kFmtQ6_K ? 210 : 144)
+    const int UB = tensor ? (fmt == kFmtQ5_K ? 176 : fmt == kFmtQ6_K ? 210 : fmt == kFmtIQ4_XS ? 136 : 144)
                           : (fmt == kFmtQ6_K ? 210 : fmt == kFmtIQ4_XS ? 136 : LB);
     double best_cost = 1e300;
     int64_t best_steps = INT64_MAX;
@@ -434,6 +436,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_MMA5K2(bp) mma_gemv_kernel<bp, 2, kFmtQ5_K>
 #define QG_MMA6K1(bp) mma_gemv_kernel<bp, 1, kFmtQ6_K>
 #define QG_MMA6K2(bp) mma_gemv_kernel<bp, 2, kFmtQ6_K>
+#define QG_MMAIQ1(bp) mma_gemv_kernel<bp, 1, kFmtIQ4_XS>
+#define QG_MMAIQ2(bp) mma_gemv_kernel<bp, 2, kFmtIQ4_XS>
 #define QG_ROWS_Q4K1(bp) rows_gemv_kernel<kFmtQ4_K, bp, 1>
 #define QG_ROWS_Q4K2(bp) rows_gemv_kernel<kFmtQ4_K, bp, 2>
 #define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
@@ -451,6 +455,10 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
     if (tensor && fmt == kFmtQ6_K) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA6K2) }
         QG_BP_SWITCH16(QG_MMA6K1)
+    }
+    if (tensor && fmt == kFmtIQ4_XS) {
+        if (mats == 2) { QG_BP_SWITCH16(QG_MMAIQ2) }
+        QG_BP_SWITCH16(QG_MMAIQ1)
     }
     if (tensor) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
@@ -484,6 +492,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #undef QG_ROWS_Q801
 #undef QG_ROWS_Q4K2
 #undef QG_ROWS_Q4K1
+#undef QG_MMAIQ2
+#undef QG_MMAIQ1
 #undef QG_MMA6K2
 #undef QG_MMA6K1
 #undef QG_MMA5K2
@@ -620,15 +630,22 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
     return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
-// The variant qg_gemv takes: the tensor-core kernel for Q4_K with B >= 2 (the CUDA-core kernel
-// spends one FMA per weight and column, so its cost grows with B while the tensor-core kernel's
-// does not; at B = 1 the CUDA-core kernel is faster), the CUDA-core row kernel otherwise, and the
-// generic kernel for rows that are not whole 256-weight units.
+// Formats with a tensor-core kernel: the K-quants, and IQ4_XS with an even number of units per row
+// (its rows are then 16-byte multiples, copied in tensor boxes).
+bool has_tensor_kernel(int fmt, int64_t K)
+{
+    return fmt == QG_FMT_Q4_K || fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K ||
+           (fmt == QG_FMT_IQ4_XS && (K / 256) % 2 == 0);
+}
+
+// The variant qg_gemv takes: the tensor-core kernel with B >= 2 where the format has one (the
+// CUDA-core kernel spends one FMA per weight and column, so its cost grows with B while the
+// tensor-core kernel's does not; at B = 1 the CUDA-core kernel is faster), the CUDA-core row kernel
+// otherwise, and the generic kernel for rows that are not whole 256-weight units.
 int auto_variant(int fmt, int64_t K, int B)
 {
     if (K % 256 != 0) return QG_VARIANT_GENERIC;
-    const bool has_tensor = (fmt == QG_FMT_Q4_K || fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K);
-    return (has_tensor && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
+    return (has_tensor_kernel(fmt, K) && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
 }
 
 // The kernel variant a GEMV call runs (QG_VARIANT_AUTO resolved), or the argument error.
@@ -640,9 +657,9 @@ int resolve_variant(int fmt, int64_t K, int B, int variant, int *var_out)
     int var = variant;
     if (var == QG_VARIANT_AUTO) var = auto_variant(fmt, K, B);
     if (var != QG_VARIANT_GENERIC && !streamable) return QG_ERR_VARIANT;
-    if (var == QG_VARIANT_TENSOR && (fmt == QG_FMT_Q8_0 || fmt == QG_FMT_IQ4_XS)) return QG_ERR_VARIANT;
-    // 9..16 columns: the K-quants' tensor-core kernels only
-    if (B > 8 && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K) return QG_ERR_BATCH;
+    if (var == QG_VARIANT_TENSOR && !has_tensor_kernel(fmt, K)) return QG_ERR_VARIANT;
+    // 9..16 columns: the tensor-core kernels only
+    if (B > 8 && !has_tensor_kernel(fmt, K)) return QG_ERR_BATCH;
     if (var == QG_VARIANT_DIRECT && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q8_0) return QG_ERR_VARIANT;
     if (var == QG_VARIANT_TCGEN05 && fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K) return QG_ERR_VARIANT;
     if (B > 8 && var != QG_VARIANT_TENSOR && var != QG_VARIANT_TCGEN05) return QG_ERR_BATCH;
@@ -875,9 +892,8 @@ int qg_gemv_host(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x
     int rc = check_common(W, fmt, N, K);
     if (rc != QG_OK) return rc;
     if (B < 1 || B > kMaxB) return QG_ERR_BATCH;
-    // 9..16 columns run on the K-quants' tensor-core kernel only (rows of whole 256-weight units)
-    if (B > 8 && ((fmt != QG_FMT_Q4_K && fmt != QG_FMT_Q5_K && fmt != QG_FMT_Q6_K) || K % 256 != 0))
-        return QG_ERR_BATCH;
+    // 9..16 columns run on the tensor-core kernels only (rows of whole 256-weight units)
+    if (B > 8 && (!has_tensor_kernel(fmt, K) || K % 256 != 0)) return QG_ERR_BATCH;
     if (N == 0) return QG_OK;
     if (!x_host || !y_host) return QG_ERR_NULL;
     if (reinterpret_cast<uintptr_t>(x_host) % 2 != 0 || reinterpret_cast<uintptr_t>(y_host) % 4 != 0)

@@ -62,6 +62,12 @@ template <> struct MmaFmt<kFmtQ5_K> {
 template <> struct MmaFmt<kFmtQ6_K> {  // rows arrive in 240-byte per-lane windows (qg_rows.cuh)
     static constexpr int kUnitBytes = 240, kQs = 0;
 };
+// IQ4_XS with an even number of 136-byte units per row: a 144-byte box per row, the 16-byte
+// aligned window around the unit, which starts 0 or 8 bytes into it (the same for every row of a
+// step); qs at byte 8 of the unit
+template <> struct MmaFmt<kFmtIQ4_XS> {
+    static constexpr int kUnitBytes = 144, kQs = 8;
+};
 
 // n-tiles of 8 columns per mma (16 columns: two, sharing the unpacked A fragment)
 template <int BP> struct MmaNT {
@@ -113,7 +119,11 @@ __device__ __forceinline__ int mma_xf_swz(int c, int lh, int h, int BP)
 // Q6_K keeps the same fragment slots with its own weight order: chunk c = 2hf + p is
 // ql[64hf + 32p ..], k-tile h covers its words 4h .. 4h+3 (one 16-weight scale group), so
 //   e = 256j + 128(c >> 1) + 32(c & 1) + 64lh + 16h + 4t,
-// and the x sums are per 16-weight group 8(c >> 1) + 2(c & 1) + h + 4lh.
+// and the x sums are per 16-weight group 8(c >> 1) + 2(c & 1) + h + 4lh.  IQ4_XS: k-tile h of chunk
+// c is sub-block 2c + h (qs words 4h .. 4h+3 of the chunk; a qs byte holds weights r and r + 16 of
+// its sub-block; k-half lh takes qs bytes 2lh, 2lh + 1 of the thread's word, whose weights pair
+// as (r, r + 16)), so the four x rows are e, e + 1, e + 16, e + 17 with e = 256j + 32(2c + h) +
+// 4t + 2lh, and it needs no x sums (its codes are the signed levels themselves).
 template <int BP, int FMT = kFmtQ4_K>
 __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, uint2 *xf,
                                             float *xsum)
@@ -130,10 +140,18 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
         if (j < US_s) {
             const int e = (FMT == kFmtQ6_K)
                               ? j * 256 + 128 * (c >> 1) + 32 * (c & 1) + 64 * lh + 16 * h + 4 * t
-                              : j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
+                          : (FMT == kFmtIQ4_XS) ? j * 256 + 32 * (2 * c + h) + 4 * t + 2 * lh
+                                                : j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
             const uint16_t *src = xsl + (int64_t)e * B;  // 4 * B contiguous halves
             const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
-            if (B == BP && (8 * BP) % 16 == 0 && (addr & 15) == 0) {
+            if (FMT == kFmtIQ4_XS) {
+                // rows e, e + 1, e + 16, e + 17 (two runs of 2 * B halves)
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int col = 0; col < BP; ++col)
+                        if (col < B) xv[r * BP + col] = src[((r & 1) + 16 * (r >> 1)) * B + col];
+            } else if (B == BP && (8 * BP) % 16 == 0 && (addr & 15) == 0) {
 #pragma unroll
                 for (int q = 0; q < (8 * BP) / 16; ++q) {
                     const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
@@ -154,7 +172,7 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
             }
         }
 #pragma unroll
-        for (int col = 0; col < BP; ++col) {
+        for (int col = 0; col < BP && FMT != kFmtIQ4_XS; ++col) {  // IQ4_XS needs no x sums
             float sum = (__half2float(__ushort_as_half((unsigned short)xv[0 * BP + col])) +
                          __half2float(__ushort_as_half((unsigned short)xv[1 * BP + col]))) +
                         (__half2float(__ushort_as_half((unsigned short)xv[2 * BP + col])) +
@@ -496,6 +514,109 @@ __device__ __forceinline__ void mma_q5k_step(const uint8_t *u0, const uint2 *xf,
     if (!kFoldPerChunk) fold_c();
 }
 
+// One IQ4_XS step: 32 rows (two 16-row tiles) x one superblock at u0 (row stride 144 B; the unit
+// starts `o` = 0 or 8 bytes into each row's window).  Thread (g, t) takes qs word t + 4h of chunk c
+// of rows g and g + 8 of a tile (sub-block 2c + h, weights 4t .. 4t+3 and 16 + 4t .. 16 + 4t+3),
+// looks its eight indices up in the codebook (iq4_lookup: biased levels u = level + 128, a byte
+// each, in nibble order), spreads two bytes under the exponent of 1024 (one byte permute per
+// register: the fp16 pair 1024 + u) and takes 1152 out with one f16x2 add, leaving the levels as
+// exact fp16 integers (-127..113, all normal).  The MMA of k-half lh takes qs bytes 2lh, 2lh + 1
+// of the word, so a register holds the weights (r, r + 16) of one byte; x is staged in that order
+// (mma_stage_x).  Both MMAs of (c, h) sum into one C fragment of sub-block 2c + h, scaled by
+// d (ls - 32) of its row (dtab: [8 sub-blocks][32 positions]).
+template <int BP>
+__device__ __forceinline__ void mma_iq4xs_step(const uint8_t *u0, int o, const uint2 *xf, int j,
+                                               float *dtab, float (&acc)[2][MmaNT<BP>::value][4],
+                                               int lane)
+{
+    constexpr int FMT = kFmtIQ4_XS;
+    constexpr int LB = MmaFmt<FMT>::kUnitBytes;
+    constexpr int NT = MmaNT<BP>::value;
+    const int g = lane >> 2, t = lane & 3;
+    const int pr = mma_frag_row<FMT>(g);
+    const uint8_t *unit = u0 + o;
+    {
+        // header of row `lane`: d (bytes 0-1), scales_h (2-3), scales_l (4-7)
+        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(unit + lane * LB);
+        const uint32_t sl = *reinterpret_cast<const uint32_t *>(unit + lane * LB + 4);
+        const uint32_t sh = w0 >> 16;
+        const float d = __half2float(__ushort_as_half((unsigned short)(w0 & 0xFFFFu)));
+        const int pos = (lane & 7) * 4 + (lane >> 3);
+#pragma unroll
+        for (int sb = 0; sb < 8; ++sb) {
+            const int ls = (int)(((sl >> (4 * sb)) & 15u) | (((sh >> (2 * sb)) & 3u) << 4));
+            dtab[sb * 32 + pos] = d * (float)(ls - 32);  // exact: an fp16 times a 6-bit integer
+        }
+    }
+    __syncwarp();
+    // two biased bytes of v (selector: bytes 0 and 2, or 1 and 3) -> the fp16 levels u - 128
+    auto levels = [](uint32_t v, uint32_t sel) {  // sel 0x4140: bytes 0, 1; 0x4342: bytes 2, 3
+        const uint32_t p = __byte_perm(v, 0x64646464u, sel);  // (1024 + u, 1024 + u')
+        uint32_t r;
+        asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(p), "r"(0xE480E480u));  // - (1152, 1152)
+        return r;
+    };
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint2 xb[NT][2][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = (BP > 8) ? 8 * nt + g : g % BP;
+                    xb[nt][lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
+                }
+        const float4 D0 = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * pr);
+        const float4 D1 = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * pr);
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const uint8_t *rowA = unit + (tile * 16 + pr) * LB + MmaFmt<FMT>::kQs + 32 * c + 4 * t;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t wa = *reinterpret_cast<const uint32_t *>(rowA + 16 * h);
+                const uint32_t wb = *reinterpret_cast<const uint32_t *>(rowA + 16 * h + 8 * LB);
+                uint32_t loA, hiA, loB, hiB;
+                iq4_lookup(wa, loA, hiA);
+                iq4_lookup(wb, loB, hiB);
+                float cs[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) cs[nt][k] = 0.0f;
+                // lo = levels of qs bytes 0, 1 (low, high nibble each), hi = of bytes 2, 3: the
+                // pairs (byte b low, byte b high) are weights (4t + b, 4t + b + 16)
+                {
+                    const uint32_t a0 = levels(loA, 0x4140u), a1 = levels(loB, 0x4140u);
+                    const uint32_t a2 = levels(loA, 0x4342u), a3 = levels(loB, 0x4342u);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816(cs[nt], a0, a1, a2, a3, xb[nt][0][h].x, xb[nt][0][h].y);
+                }
+                {
+                    const uint32_t a0 = levels(hiA, 0x4140u), a1 = levels(hiB, 0x4140u);
+                    const uint32_t a2 = levels(hiA, 0x4342u), a3 = levels(hiB, 0x4342u);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816(cs[nt], a0, a1, a2, a3, xb[nt][1][h].x, xb[nt][1][h].y);
+                }
+                const float4 D = h ? D1 : D0;
+                const float da = tile ? D.z : D.x, db = tile ? D.w : D.y;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[tile][nt][0] = fmaf(da, cs[nt][0], acc[tile][nt][0]);
+                    acc[tile][nt][2] = fmaf(db, cs[nt][2], acc[tile][nt][2]);
+                    if (BP > 1) {
+                        acc[tile][nt][1] = fmaf(da, cs[nt][1], acc[tile][nt][1]);
+                        acc[tile][nt][3] = fmaf(db, cs[nt][3], acc[tile][nt][3]);
+                    }
+                }
+            }
+        }
+    }
+}
+
 // One Q6_K step: 32 rows x one superblock from the warp's per-lane windows at u0 (window of row
 // r at u0 + 240 r; its superblock starts o_r = (m_r * 210) mod 16 bytes in, m_r its superblock
 // index in the tensor).  Chunk c = 2hf + p is ql[64hf + 32p ..]; its k-tile kk (words 4kk .. 4kk+3)
@@ -626,7 +747,7 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
     constexpr int NW = MmaWarpsF<FMT, BP>::value;
     constexpr int TAB = MmaTabF<FMT, BP>::value;
     constexpr bool PER_LANE = (FMT == kFmtQ6_K);    // per-lane copy windows (rows kernel, Q6_K)
-    constexpr int UB = PER_LANE ? 210 : MmaFmt<FMT>::kUnitBytes;  // unit bytes in W
+    constexpr int UB = PER_LANE ? 210 : (FMT == kFmtIQ4_XS) ? 136 : MmaFmt<FMT>::kUnitBytes;  // in W
     constexpr int LB = MmaFmt<FMT>::kUnitBytes;     // ring bytes per row
     constexpr int GR = PER_LANE ? 16 : 8;           // x-sum groups per unit
     constexpr int BOX = 32 * LB;
@@ -686,8 +807,10 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
     auto issue = [&](int i) {
         const uint32_t bar = bar0 + 8 * (i % kRowsStages);
         mbar_arrive_expect_tx(bar, BOX);
-        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], (ucol0 + iu) * INNER,
-                    ig_row, bar);
+        // IQ4_XS: the box starts at the unit's byte offset rounded down to 16 bytes
+        const int bx = (FMT == kFmtIQ4_XS) ? (int)(((int64_t)(ucol0 + iu) * UB & ~(int64_t)15) >> 2)
+                                           : (ucol0 + iu) * INNER;
+        tma_load_2d(smem_u32(myring + (i % kRowsStages) * BOX), &maps.m[ig_map], bx, ig_row, bar);
         advance();
     };
     // Q6_K: per-lane bulk copies of the 16-byte aligned window around each row's unit (all 32
@@ -774,7 +897,10 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
                 mma_q6k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
                                  lane, a, row0, ucol0 + j, a.w[second ? MATS - 1 : 0]);
             } else {
-                if (FMT == kFmtQ5_K)
+                if (FMT == kFmtIQ4_XS)
+                    mma_iq4xs_step<BP>(myring + (step % kRowsStages) * BOX, (int)(((int64_t)(ucol0 + j) * UB) & 15),
+                                       xf, j, dtab, acc, lane);
+                else if (FMT == kFmtQ5_K)
                     mma_q5k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM, lane);
                 else
                     mma_q4k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM, lane);

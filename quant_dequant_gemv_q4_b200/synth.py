@@ -217,5 +217,10 @@ WORKLOADS = {
         Gemv("q4k_ffn_gate_b16", Q4_K, 17408, 5120, 16, 0),
         Gemv("q5k_ffn_gate_b16", Q5_K, 17408, 5120, 16, 1),
         Gemv("q6k_ffn_gate_b16", Q6_K, 17408, 5120, 16, 2))),
+    # IQ4_XS on the batched-verify widths (the tensor-core kernel at B >= 2)
+    "iq4xs_ffn_gate_verify": Workload("iq4xs_ffn_gate_verify", 10, (
+        Gemv("ffn_gate_b2", IQ4_XS, 17408, 5120, 2, 0, 1e-3),
+        Gemv("ffn_gate_b8", IQ4_XS, 17408, 5120, 8, 1, 1e-3),
+        Gemv("ffn_gate_b16", IQ4_XS, 17408, 5120, 16, 2, 1e-3))),
 }
 FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q6_K: "Q6_K", Q8_0: "Q8_0", IQ4_XS: "IQ4_XS"}

@@ -5,6 +5,8 @@ Bars as for the other formats: the dump is bit-exact (every IQ4_XS weight is exa
 GEMV meets |y - y_ref| <= 1e-5 * sum|w*x| + 1e-6 per output on the synthetic workloads; repeated
 calls are bitwise identical; the exact special case matches exactly.  The factored kernel's own
 bound (relative to sum |d*(ls-32)| * (|level| + 128) * |x|) is checked on near-cancelling weights.
+The tensor-core kernel (QG_VARIANT_TENSOR, the default at B >= 2 when K / 256 is even) multiplies
+the levels themselves, exactly, so it is held to the strict bound everywhere, at B = 2..16.
 """
 import numpy as np
 import pytest
@@ -62,17 +64,44 @@ def test_dump_golden_superblock(dev):
 
 
 SMALL_SHAPES = [(1, 256), (2, 512), (7, 1280), (33, 5120), (300, 768), (129, 2560)]
+TENSOR = 4
 
 
-@pytest.mark.parametrize("variant", [0, 2, 3])
+def even_units(K):
+    return (K // 256) % 2 == 0
+
+
+@pytest.mark.parametrize("variant", [0, 2, 3, TENSOR])
 @pytest.mark.parametrize("N,K", SMALL_SHAPES)
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8])
 def test_gemv_small(dev, orc, variant, N, K, B):
+    import quant_dequant_gemv_q4_b200 as qg
     W = synth.iq4xs_weights(N, K, seed=N * 7 + K)
     x = synth.activations(K, B, seed=B + 23, massive_frac=1e-3)
+    if variant == TENSOR and not even_units(K):
+        with pytest.raises(qg.QgError) as e:
+            gpu_gemv(dev, W, IQ4_XS, N, K, x, variant)
+        assert e.value.status == qg.QG_ERR_VARIANT
+        return
     y = gpu_gemv(dev, W, IQ4_XS, N, K, x, variant)
     yref, A = orc.gemv(W, IQ4_XS, N, K, x, B)
     assert_within(y, yref, A, f"v{variant} N={N} K={K} B={B}")
+    if variant == 0:
+        want = qg.QG_VARIANT_TENSOR if (B >= 2 and even_units(K)) else qg.QG_VARIANT_FACTORED
+        assert qg.qg_last_variant() == want
+
+
+@pytest.mark.parametrize("N,K", [(2, 512), (33, 5120), (129, 2560), (300, 1024), (70, 17408)])
+@pytest.mark.parametrize("B", [9, 12, 16])
+def test_gemv_wide_tensor(dev, orc, N, K, B):
+    """B = 9..16 on the tensor-core kernel: two 8-column n-tiles share the looked-up levels."""
+    import quant_dequant_gemv_q4_b200 as qg
+    W = synth.iq4xs_weights(N, K, seed=N + K + B)
+    x = synth.activations(K, B, seed=B + 29, massive_frac=1e-3)
+    y = gpu_gemv(dev, W, IQ4_XS, N, K, x, 0)
+    assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
+    yref, A = orc.gemv(W, IQ4_XS, N, K, x, B)
+    assert_within(y, yref, A, f"N={N} K={K} B={B}")
 
 
 @pytest.mark.parametrize("N,K,B", [(96, 17408, 8), (17, 65536, 2), (40, 65536, 1)])
@@ -97,7 +126,7 @@ def test_exact_integer_case(dev, orc):
     W = W.reshape(-1)
     x = rng.integers(-2, 3, size=(K, B)).astype(np.float16)
     yref, _ = orc.gemv(W, IQ4_XS, N, K, x, B)
-    for variant in (0, 2, 3):
+    for variant in (0, 2, 3, TENSOR):
         y = gpu_gemv(dev, W, IQ4_XS, N, K, x, variant)
         assert np.array_equal(y.astype(np.float64), yref), variant
 
@@ -118,6 +147,7 @@ def test_near_cancelling_levels(dev, orc):
     x = synth.activations(K, B, seed=25)
     yref, A = orc.gemv(W, IQ4_XS, N, K, x, B)
     assert_within(gpu_gemv(dev, W, IQ4_XS, N, K, x, 3), yref, A, "generic")
+    assert_within(gpu_gemv(dev, W, IQ4_XS, N, K, x, TENSOR), yref, A, "tensor")  # exact levels
     s = np.abs(np.repeat(ls.astype(np.float64) - 32.0, 32)) * 2.0 ** -8
     Af = (s * (np.abs(LEVELS[idx]) + 128.0)).reshape(N, K) @ np.abs(x.astype(np.float64))
     assert_within(gpu_gemv(dev, W, IQ4_XS, N, K, x, 2), yref, Af, "factored")
@@ -136,37 +166,43 @@ def test_tail_window(dev, orc):
 
 
 @pytest.mark.parametrize("N,K", [(17408, 5120), (5120, 17408)])
-@pytest.mark.parametrize("B", [1, 8])
-def test_full_size_sampled(dev, orc, N, K, B):
+@pytest.mark.parametrize("B,variant", [(1, 0), (2, 0), (8, 0), (16, 0), (8, 2)])
+def test_full_size_sampled(dev, orc, N, K, B, variant):
     W = synth.iq4xs_weights(N, K, seed=N + B)
     x = synth.activations(K, B, seed=B + 5, massive_frac=1e-3)
-    y = gpu_gemv(dev, W, IQ4_XS, N, K, x, 0)
+    y = gpu_gemv(dev, W, IQ4_XS, N, K, x, variant)
     assert np.isfinite(y).all()
     rows = _sample_rows(N, np.random.default_rng(B))
     yref, A = orc.gemv(W, IQ4_XS, N, K, x, B, rows=rows)
-    assert_within(y[rows], yref, A, f"{N}x{K} B={B}")
-    y2 = gpu_gemv(dev, W, IQ4_XS, N, K, x, 0)
+    assert_within(y[rows], yref, A, f"{N}x{K} B={B} v{variant}")
+    y2 = gpu_gemv(dev, W, IQ4_XS, N, K, x, variant)
     assert np.array_equal(y.view(np.uint32), y2.view(np.uint32)), "not deterministic"
 
 
 def test_launch_witness_and_variant_checks(dev):
+    """AUTO: TENSOR at B >= 2 when K / 256 is even, FACTORED otherwise; TENSOR refused for an odd
+    K / 256 (rows not 16-byte multiples), DIRECT refused always."""
     import torch
     import quant_dequant_gemv_q4_b200 as qg
-    N, K = 64, 1024
-    W = _t(synth.iq4xs_weights(N, K, seed=1), dev)
-    for B in (1, 2, 8):
-        x = _t(synth.activations(K, B, seed=1).view(np.uint16), dev)
-        y = torch.empty((N, B), dtype=torch.float32, device=dev)
-        qg.qg_gemv(W, IQ4_XS, N, K, x, B, y)
-        assert qg.qg_last_variant() == qg.QG_VARIANT_FACTORED
-        for v in (qg.QG_VARIANT_TENSOR, qg.QG_VARIANT_DIRECT):
-            with pytest.raises(qg.QgError) as e:
-                qg.qg_gemv_variant(W, IQ4_XS, N, K, x, B, y, None, v)
-            assert e.value.status == qg.QG_ERR_VARIANT
+    N = 64
+    for K in (1024, 768):
+        W = _t(synth.iq4xs_weights(N, K, seed=1), dev)
+        for B in (1, 2, 8):
+            x = _t(synth.activations(K, B, seed=1).view(np.uint16), dev)
+            y = torch.empty((N, B), dtype=torch.float32, device=dev)
+            qg.qg_gemv(W, IQ4_XS, N, K, x, B, y)
+            tensor = B >= 2 and even_units(K)
+            assert qg.qg_last_variant() == (qg.QG_VARIANT_TENSOR if tensor else qg.QG_VARIANT_FACTORED)
+            bad = [qg.QG_VARIANT_DIRECT] + ([] if even_units(K) else [qg.QG_VARIANT_TENSOR])
+            for v in bad:
+                with pytest.raises(qg.QgError) as e:
+                    qg.qg_gemv_variant(W, IQ4_XS, N, K, x, B, y, None, v)
+                assert e.value.status == qg.QG_ERR_VARIANT
     assert qg.qg_device_error() == 0
 
 
-@pytest.mark.parametrize("N,K,B", [(33, 5120, 1), (300, 768, 3), (129, 2560, 8), (96, 17408, 2)])
+@pytest.mark.parametrize("N,K,B", [(33, 5120, 1), (300, 768, 3), (129, 2560, 8), (96, 17408, 2),
+                                   (200, 5120, 16), (40, 17408, 12)])
 def test_gate_up(dev, orc, N, K, B):
     import torch
     import quant_dequant_gemv_q4_b200 as qg
@@ -199,10 +235,14 @@ def test_output_guards_untouched(dev, orc):
     W = synth.iq4xs_weights(N, K, seed=4)
     x = synth.activations(K, B, seed=4)
     yref, A = orc.gemv(W, IQ4_XS, N, K, x, B)
-    for v in (0, 2, 3):
+    for v in (0, 2, 3, TENSOR):
+        if v == TENSOR:  # K / 256 even for the tensor-core kernel
+            K2 = 2560
+            W, x = synth.iq4xs_weights(N, K2, seed=5), synth.activations(K2, B, seed=5)
+            yref, A = orc.gemv(W, IQ4_XS, N, K2, x, B)
         buf = torch.full((N * B + 128,), 12345.0, dtype=torch.float32, device=dev)
         y = buf[64:64 + N * B]
-        qg.qg_gemv_variant(_t(W, dev), IQ4_XS, N, K, _t(x.view(np.uint16), dev), B, y, None, v)
+        qg.qg_gemv_variant(_t(W, dev), IQ4_XS, N, x.shape[0], _t(x.view(np.uint16), dev), B, y, None, v)
         torch.cuda.synchronize()
         b = buf.cpu().numpy()
         assert np.all(b[:64] == 12345.0) and np.all(b[64 + N * B:] == 12345.0), v
@@ -227,10 +267,18 @@ def test_x_not_16_byte_aligned(dev, orc, B):
 
 
 def test_wide_b_rejected(dev):
+    """B = 9..16 needs the tensor-core kernel: refused for an odd K / 256 and on the CUDA-core
+    variants."""
     import quant_dequant_gemv_q4_b200 as qg
     W = synth.iq4xs_weights(8, 256, seed=1)
     x = synth.activations(256, 9, seed=1)
     for v in (0, 2, 3):
         with pytest.raises(qg.QgError) as e:
             gpu_gemv(dev, W, IQ4_XS, 8, 256, x, v)
+        assert e.value.status == qg.QG_ERR_BATCH
+    W = synth.iq4xs_weights(8, 512, seed=1)
+    x = synth.activations(512, 9, seed=1)
+    for v in (2, 3):
+        with pytest.raises(qg.QgError) as e:
+            gpu_gemv(dev, W, IQ4_XS, 8, 512, x, v)
         assert e.value.status == qg.QG_ERR_BATCH

@@ -74,9 +74,10 @@ def test_plan_invariants(sms, smem, fmt):
                 try:
                     p = qg.qg_plan(fmt, N, K, B, 0, mats, sms, smem)
                 except qg.QgError as e:
-                    # B > 8 is the K-quants' tensor-core kernel's only (and not the Q6_K pair's);
-                    # a small device may fit no plan
-                    wide_ok = fmt in (Q4_K, Q5_K) or (fmt == Q6_K and mats == 1)
+                    # B > 8 is the tensor-core kernels' only (not the Q6_K pair's, and IQ4_XS's
+                    # with an even K / 256); a small device may fit no plan
+                    wide_ok = fmt in (Q4_K, Q5_K) or (fmt == Q6_K and mats == 1) or \
+                        (fmt == IQ4_XS and UPR % 2 == 0)
                     assert (B > 8 and not wide_ok and e.status == qg.QG_ERR_BATCH) or \
                         e.status == qg.QG_ERR_SHAPE, (N, K, B, mats, e)
                     continue
@@ -86,7 +87,8 @@ def test_plan_invariants(sms, smem, fmt):
                 assert S * US >= UPR > (S - 1) * US
                 assert 1 <= p["ctas"] <= sms
                 assert p["warps"] in (6, 8, 12, 16)
-                assert p["variant"] == (TENSOR if fmt in (Q4_K, Q5_K, Q6_K) and B >= 2 else FACTORED)
+                has_tc = fmt in (Q4_K, Q5_K, Q6_K) or (fmt == IQ4_XS and UPR % 2 == 0)
+                assert p["variant"] == (TENSOR if has_tc and B >= 2 else FACTORED)
     assert n > 0
 
 
