@@ -89,8 +89,8 @@ enum {
 };
 
 /* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses: when
- * K % 256 == 0, TENSOR with B >= 2 for the K-quants (Q4_K, Q5_K, Q6_K) and for IQ4_XS with an
- * even K / 256, FACTORED otherwise; GENERIC when K % 256 != 0. */
+ * K % 256 == 0, TENSOR with B >= 2 for Q4_K, Q5_K and IQ4_XS with an even K / 256, and with
+ * B >= 3 for Q6_K, FACTORED otherwise; GENERIC when K % 256 != 0. */
 enum {
     QG_VARIANT_AUTO = 0,
     /* Each weight is dequantized to the correctly rounded fp32 w = RN(d*sc*q - dmin*m) (Q4_K; the

@@ -638,14 +638,18 @@ bool has_tensor_kernel(int fmt, int64_t K)
            (fmt == QG_FMT_IQ4_XS && (K / 256) % 2 == 0);
 }
 
-// The variant qg_gemv takes: the tensor-core kernel with B >= 2 where the format has one (the
-// CUDA-core kernel spends one FMA per weight and column, so its cost grows with B while the
-// tensor-core kernel's does not; at B = 1 the CUDA-core kernel is faster), the CUDA-core row kernel
-// otherwise, and the generic kernel for rows that are not whole 256-weight units.
+// The variant qg_gemv takes: the tensor-core kernel where the format has one and B is past the
+// measured crossover (the CUDA-core kernel spends one FMA per weight and column, so its cost grows
+// with B while the tensor-core kernel's does not), the CUDA-core row kernel otherwise, and the
+// generic kernel for rows that are not whole 256-weight units.  Crossover on B200 (17408 x 5120 and
+// 5120 x 17408): B = 2 for Q4_K, Q5_K and IQ4_XS (the CUDA-core kernels win only at B = 1); B = 3
+// for Q6_K, whose CUDA-core kernel still wins at B = 2 (31.2 vs 34.7 us) and whose tensor-core
+// step pays for the per-lane copy windows.
 int auto_variant(int fmt, int64_t K, int B)
 {
     if (K % 256 != 0) return QG_VARIANT_GENERIC;
-    return (has_tensor_kernel(fmt, K) && B >= 2) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
+    const int tc_min = (fmt == QG_FMT_Q6_K) ? 3 : 2;
+    return (has_tensor_kernel(fmt, K) && B >= tc_min) ? QG_VARIANT_TENSOR : QG_VARIANT_FACTORED;
 }
 
 // The kernel variant a GEMV call runs (QG_VARIANT_AUTO resolved), or the argument error.

@@ -220,8 +220,12 @@ def test_launch_witness(dev):
     for fmt in (Q5_K, Q6_K):
         W = _t(synth.weights(fmt, N, K, seed=1), dev)
         x = _t(synth.activations(K, 2, seed=1).view(np.uint16), dev)
-        y = torch.empty((N, 2), dtype=torch.float32, device=dev)
+        y = torch.empty((N, 3), dtype=torch.float32, device=dev)
         qg.qg_gemv(W, fmt, N, K, x, 2, y)
+        # the tensor cores from B = 2 (Q5_K) or 3 (Q6_K, whose CUDA-core kernel wins at B = 2)
+        assert qg.qg_last_variant() == (qg.QG_VARIANT_TENSOR if fmt == Q5_K else qg.QG_VARIANT_FACTORED)
+        x3 = _t(synth.activations(K, 3, seed=1).view(np.uint16), dev)
+        qg.qg_gemv(W, fmt, N, K, x3, 3, y)
         assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
         x1 = _t(synth.activations(K, 1, seed=1).view(np.uint16), dev)
         qg.qg_gemv(W, fmt, N, K, x1, 1, y)

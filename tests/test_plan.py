@@ -88,7 +88,8 @@ def test_plan_invariants(sms, smem, fmt):
                 assert 1 <= p["ctas"] <= sms
                 assert p["warps"] in (6, 8, 12, 16)
                 has_tc = fmt in (Q4_K, Q5_K, Q6_K) or (fmt == IQ4_XS and UPR % 2 == 0)
-                assert p["variant"] == (TENSOR if has_tc and B >= 2 else FACTORED)
+                tc_min = 3 if fmt == Q6_K else 2  # Q6_K's CUDA-core kernel still wins at B = 2
+                assert p["variant"] == (TENSOR if has_tc and B >= tc_min else FACTORED)
     assert n > 0
 
 
