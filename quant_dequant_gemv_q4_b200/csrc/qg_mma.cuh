@@ -113,9 +113,41 @@ __device__ __forceinline__ int mma_xf_swz(int c, int lh, int h, int BP)
     return BP >= 4 ? ((h + 2 * lh + 4 * (c & 1)) & (BP - 1)) : 0;
 }
 
-// Thread g stages the 4 consecutive x rows e..e+3 of group g = ((j*4 + c)*2 + lh)*8 + 2t + h
-// (all B columns, one contiguous run of 4*B halves, read with the widest aligned loads), writes
-// their BP fragments, and the 8 groups of one sub-block (8 consecutive lanes) add up its x sums.
+// Sums over the 8 lanes of a sub-block group (lanes 8i .. 8i+7 of the warp, th = lane % 8) of
+// the per-column values s[0..BP): a transposing butterfly.  At xor distance 4, 2, 1 each lane keeps
+// half of its columns (the upper half when its bit of th is set), sends the other half to its
+// partner and adds what it receives, so 8 columns take 4 + 2 + 1 shuffles instead of 3 per column.
+// Once a lane holds a single column the remaining levels are plain butterfly adds.  On return lane
+// th holds the sums of columns [c0, c0 + n) with n = max(BP / 8, 1) and
+// c0 = (th * BP / 8) for BP >= 8, th >> (3 - log2 BP) otherwise (then lanes whose low 3 - log2 BP
+// bits of th are zero hold the only copy needed).
+template <int N, int M>
+__device__ __forceinline__ void xsum_butterfly(float *s, int th)
+{
+    if constexpr (M > 0) {
+        if constexpr (N >= 2) {
+            constexpr int H = N / 2;
+            const bool up = (th & M) != 0;
+#pragma unroll
+            for (int i = 0; i < H; ++i) {
+                const float send = up ? s[i] : s[i + H];
+                const float keep = up ? s[i + H] : s[i];
+                s[i] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+            }
+            xsum_butterfly<H, M / 2>(s, th);
+        } else {
+            s[0] += __shfl_xor_sync(0xffffffffu, s[0], M);
+            xsum_butterfly<1, M / 2>(s, th);
+        }
+    }
+}
+
+// Thread g stages the 4 x rows of group g = ((j*4 + c)*2 + lh)*8 + 2t + h (rows e..e+3 for the
+// K-quants, all B columns), writes their BP fragments, and the 8 groups of one sub-block (8
+// consecutive lanes) add up its x sums.  A thread loads the rows of up to NB groups before it
+// processes any, so their L2 round trips overlap.  A row's BP halves are BP / 2 words (word m:
+// columns 2m, 2m + 1), and a fragment register takes two halves of one column from two rows with
+// one byte permute.
 // Q6_K keeps the same fragment slots with its own weight order: chunk c = 2hf + p is
 // ql[64hf + 32p ..], k-tile h covers its words 4h .. 4h+3 (one 16-weight scale group), so
 //   e = 256j + 128(c >> 1) + 32(c & 1) + 64lh + 16h + 4t,
@@ -128,73 +160,112 @@ template <int BP, int FMT = kFmtQ4_K>
 __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, uint2 *xf,
                                             float *xsum)
 {
+    constexpr int W = (BP + 1) / 2;           // words of one x row (BP halves, BP >= 2; BP = 1: 1)
+    constexpr int NB = BP >= 16 ? 2 : 4;      // groups whose loads are in flight together
     const int B = a.B;
     const uint16_t *xsl = a.x + (int64_t)s * a.US * 256 * B;
     const int ngroups = a.US * 64;  // a multiple of 32: every lane of a warp takes part
-    for (int gi = threadIdx.x; gi < ngroups; gi += blockDim.x) {
+    auto first_row = [&](int gi) {
         const int th = gi & 7, t = th >> 1, h = th & 1;
         const int lh = (gi >> 3) & 1, c = (gi >> 4) & 3, j = gi >> 6;
-        uint32_t xv[4 * BP];  // x[e + r][col] at r * BP + col (fp16 bits), zero when absent
+        return (FMT == kFmtQ6_K) ? j * 256 + 128 * (c >> 1) + 32 * (c & 1) + 64 * lh + 16 * h + 4 * t
+               : (FMT == kFmtIQ4_XS) ? j * 256 + 32 * (2 * c + h) + 4 * t + 2 * lh
+                                     : j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
+    };
+    // x row r (0..3) of a group: e + r, or for IQ4_XS e + (r & 1) + 16 (r >> 1)
+    auto row_off = [](int r) { return (FMT == kFmtIQ4_XS) ? (r & 1) + 16 * (r >> 1) : r; };
+    for (int g0 = threadIdx.x; g0 < ngroups; g0 += NB * blockDim.x) {
+        uint32_t rw[NB][4][W];  // raw x rows: [group][row][word], zero when absent
 #pragma unroll
-        for (int q = 0; q < 4 * BP; ++q) xv[q] = 0u;
-        if (j < US_s) {
-            const int e = (FMT == kFmtQ6_K)
-                              ? j * 256 + 128 * (c >> 1) + 32 * (c & 1) + 64 * lh + 16 * h + 4 * t
-                          : (FMT == kFmtIQ4_XS) ? j * 256 + 32 * (2 * c + h) + 4 * t + 2 * lh
-                                                : j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
-            const uint16_t *src = xsl + (int64_t)e * B;  // 4 * B contiguous halves
-            const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
-            if (FMT == kFmtIQ4_XS) {
-                // rows e, e + 1, e + 16, e + 17 (two runs of 2 * B halves)
+        for (int u = 0; u < NB; ++u) {
+            const int gi = g0 + u * blockDim.x;
+            const int j = gi >> 6;
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-                    for (int col = 0; col < BP; ++col)
-                        if (col < B) xv[r * BP + col] = src[((r & 1) + 16 * (r >> 1)) * B + col];
-            } else if (B == BP && (8 * BP) % 16 == 0 && (addr & 15) == 0) {
+                for (int m = 0; m < W; ++m) rw[u][r][m] = 0u;
+            if (gi < ngroups && j < US_s) {
+                const int e = first_row(gi);
+                const uint16_t *src = xsl + (int64_t)e * B;
+                const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
+                if (FMT != kFmtIQ4_XS && B == BP && BP >= 2 && (addr & 15) == 0) {
+                    // 4 rows x BP halves = 2 BP words, contiguous: BP / 2 16-byte loads
 #pragma unroll
-                for (int q = 0; q < (8 * BP) / 16; ++q) {
-                    const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
-                    xv[8 * q + 0] = v.x & 0xFFFFu; xv[8 * q + 1] = v.x >> 16;
-                    xv[8 * q + 2] = v.y & 0xFFFFu; xv[8 * q + 3] = v.y >> 16;
-                    xv[8 * q + 4] = v.z & 0xFFFFu; xv[8 * q + 5] = v.z >> 16;
-                    xv[8 * q + 6] = v.w & 0xFFFFu; xv[8 * q + 7] = v.w >> 16;
+                    for (int q = 0; q < BP / 2; ++q) {
+                        const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
+                        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) rw[u][(4 * q + k) / W][(4 * q + k) % W] = vv[k];
+                    }
+                } else if (FMT != kFmtIQ4_XS && B == 1 && BP == 1 && (addr & 7) == 0) {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(src);
+                    rw[u][0][0] = v.x & 0xFFFFu; rw[u][1][0] = v.x >> 16;
+                    rw[u][2][0] = v.y & 0xFFFFu; rw[u][3][0] = v.y >> 16;
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int col = 0; col < BP; ++col)
+                            if (col < B)
+                                rw[u][r][col >> 1] |= (uint32_t)src[row_off(r) * B + col] << (16 * (col & 1));
                 }
-            } else if (B == BP && BP == 1 && (addr & 7) == 0) {
-                const uint2 v = *reinterpret_cast<const uint2 *>(src);
-                xv[0] = v.x & 0xFFFFu; xv[1] = v.x >> 16; xv[2] = v.y & 0xFFFFu; xv[3] = v.y >> 16;
-            } else {
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-#pragma unroll
-                    for (int col = 0; col < BP; ++col)
-                        if (col < B) xv[r * BP + col] = src[r * B + col];
             }
         }
 #pragma unroll
-        for (int col = 0; col < BP && FMT != kFmtIQ4_XS; ++col) {  // IQ4_XS needs no x sums
-            float sum = (__half2float(__ushort_as_half((unsigned short)xv[0 * BP + col])) +
-                         __half2float(__ushort_as_half((unsigned short)xv[1 * BP + col]))) +
-                        (__half2float(__ushort_as_half((unsigned short)xv[2 * BP + col])) +
-                         __half2float(__ushort_as_half((unsigned short)xv[3 * BP + col])));
-            if (FMT == kFmtQ6_K) {
-                // the 4 lanes t = 0..3 of (c, lh, h) (th = 2t + h): xor over th bits 1 and 2
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-                if (t == 0)
-                    xsum[rows_xsum_off<BP, 16>(a.US, j, 8 * (c >> 1) + 2 * (c & 1) + h + 4 * lh, col)] = sum;
-            } else {
+        for (int u = 0; u < NB; ++u) {
+            const int gi = g0 + u * blockDim.x;
+            if (gi >= ngroups) break;  // uniform across the warp (ngroups and blockDim: multiples of 32)
+            const int th = gi & 7, t = th >> 1, h = th & 1;
+            const int lh = (gi >> 3) & 1, c = (gi >> 4) & 3, j = gi >> 6;
+            if (FMT != kFmtIQ4_XS) {
+                // column sums of the 4 rows in fp32: (x0 + x1) + (x2 + x3)
+                float sc[BP];
 #pragma unroll
-                for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                if (th == 0) xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, col)] = sum;
+                for (int m = 0; m < W; ++m) {
+                    float2 f[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        __half2 hh;
+                        *reinterpret_cast<uint32_t *>(&hh) = rw[u][r][m];
+                        f[r] = __half22float2(hh);
+                    }
+                    const float2 sm = __fadd2_rn(__fadd2_rn(f[0], f[1]), __fadd2_rn(f[2], f[3]));
+                    sc[2 * m] = sm.x;
+                    if (2 * m + 1 < BP) sc[2 * m + 1] = sm.y;
+                }
+                if (FMT == kFmtQ6_K) {
+                    // the 4 lanes t = 0..3 of (c, lh, h) (th = 2t + h): xor over th bits 1 and 2
+#pragma unroll
+                    for (int col = 0; col < BP; ++col) {
+                        float sum = sc[col];
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                        if (t == 0)
+                            xsum[rows_xsum_off<BP, 16>(a.US, j, 8 * (c >> 1) + 2 * (c & 1) + h + 4 * lh, col)] = sum;
+                    }
+                } else {
+                    xsum_butterfly<BP, 4>(sc, th);
+                    if (BP >= 8) {
+#pragma unroll
+                        for (int i = 0; i < (BP >= 8 ? BP / 8 : 1); ++i)
+                            xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, th * (BP / 8) + i)] = sc[i];
+                    } else {
+                        constexpr int SH = BP == 4 ? 1 : BP == 2 ? 2 : 3;  // 3 - log2 BP
+                        if ((th & ((1 << SH) - 1)) == 0)
+                            xsum[rows_xsum_off<BP>(a.US, j, 2 * c + lh, th >> SH)] = sc[0];
+                    }
+                }
+            }
+            // fragments: (x[r0][col], x[r2][col]), (x[r1][col], x[r3][col])
+            const int swz = mma_xf_swz(c, lh, h, BP);
+#pragma unroll
+            for (int col = 0; col < BP; ++col) {
+                const uint32_t sel = (col & 1) ? 0x7632u : 0x5410u;
+                xf[mma_xf_idx(j, c, lh, h, col ^ swz, t, BP)] =
+                    make_uint2(__byte_perm(rw[u][0][col >> 1], rw[u][2][col >> 1], sel),
+                               __byte_perm(rw[u][1][col >> 1], rw[u][3][col >> 1], sel));
             }
         }
-        const int swz = mma_xf_swz(c, lh, h, BP);
-#pragma unroll
-        for (int col = 0; col < BP; ++col)
-            xf[mma_xf_idx(j, c, lh, h, col ^ swz, t, BP)] =
-                make_uint2(xv[0 * BP + col] | (xv[2 * BP + col] << 16),
-                           xv[1 * BP + col] | (xv[3 * BP + col] << 16));
     }
 }
 
