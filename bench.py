@@ -49,6 +49,7 @@ FALLBACK_HBM_GBS = 6650.0
 # host packer are not among them, so a change there leaves the headline's DRAM capture valid.
 ROWS_KERNEL_FILES = ("qg_api.cu", "qg_device.cuh", "qg_rows.cuh")
 MMA_KERNEL_FILES = ROWS_KERNEL_FILES + ("qg_codes.cuh", "qg_mma.cuh")  # the B >= 2 tensor-core kernel
+UMMA_KERNEL_FILES = ROWS_KERNEL_FILES + ("qg_codes.cuh", "qg_umma.cuh")  # the tcgen05 variant
 
 
 def kernel_source_hash(files=None) -> str:
@@ -548,8 +549,9 @@ def run_reference(args):
 
 def run_ncu_case(args):
     """The headline tensor, one copy on the device: 3 launches at B=1, then 3 at B=8.  With
-    --ncu-fmt 13 or 14 the same tensor shape in Q5_K / Q6_K instead (3 launches at B=1, then 3 at
-    B=8)."""
+    --ncu-fmt 13, 14 or 23 the same tensor shape in Q5_K / Q6_K / IQ4_XS instead (3 launches at
+    B=1, then 3 at B=8); --variant picks the kernel variant (0: the library's default, 5: the
+    tcgen05 kernel)."""
     import torch
     from quant_dequant_gemv_q4_b200 import build as qbuild
     qbuild.build()
@@ -573,7 +575,8 @@ def run_ncu_case(args):
         del Wd, xd, yd
     print(json.dumps({"ncu_case": "done", "kernel_hash": kernel_source_hash(),
                       "rows_kernel_hash": kernel_source_hash(ROWS_KERNEL_FILES),
-                      "mma_kernel_hash": kernel_source_hash(MMA_KERNEL_FILES)}), flush=True)
+                      "mma_kernel_hash": kernel_source_hash(MMA_KERNEL_FILES),
+                      "umma_kernel_hash": kernel_source_hash(UMMA_KERNEL_FILES)}), flush=True)
     return 0
 
 
@@ -613,7 +616,7 @@ def main(argv=None):
                     help="launch the headline call 3x at B=1 then 3x at B=8 on one weight copy "
                          "and exit (the small case an ncu capture runs; nothing is timed)")
     ap.add_argument("--ncu-fmt", type=int, default=12,
-                    help="--ncu-case format: 12 Q4_K (default), 13 Q5_K, 14 Q6_K")
+                    help="--ncu-case format: 12 Q4_K (default), 13 Q5_K, 14 Q6_K, 23 IQ4_XS")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
 
