@@ -197,6 +197,25 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
 #pragma unroll
                         for (int k = 0; k < 4; ++k) rw[u][(4 * q + k) / W][(4 * q + k) % W] = vv[k];
                     }
+                } else if (FMT == kFmtIQ4_XS && B == BP && BP >= 4 && (addr & 15) == 0) {
+                    // two runs of 2 rows (e, e + 1 and e + 16, e + 17): BP / 4 16-byte loads each
+#pragma unroll
+                    for (int run = 0; run < 2; ++run)
+#pragma unroll
+                        for (int q = 0; q < BP / 4; ++q) {
+                            const uint4 v = reinterpret_cast<const uint4 *>(src + 16 * run * B)[q];
+                            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                rw[u][2 * run + (4 * q + k) / W][(4 * q + k) % W] = vv[k];
+                        }
+                } else if (FMT == kFmtIQ4_XS && B == BP && BP == 2 && (addr & 7) == 0) {
+#pragma unroll
+                    for (int run = 0; run < 2; ++run) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(src + 16 * run * B);
+                        rw[u][2 * run][0] = v.x;
+                        rw[u][2 * run + 1][0] = v.y;
+                    }
                 } else if (FMT != kFmtIQ4_XS && B == 1 && BP == 1 && (addr & 7) == 0) {
                     const uint2 v = *reinterpret_cast<const uint2 *>(src);
                     rw[u][0][0] = v.x & 0xFFFFu; rw[u][1][0] = v.x >> 16;
