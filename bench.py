@@ -384,6 +384,28 @@ def time_e2e(cs: CallSet, steps: int, warmup: int, variant: int):
     return secs, h2d, d2h
 
 
+def time_latency(cs: CallSet, calls: int, variant: int) -> dict:
+    """Per-call latency distribution: eager launches on one stream with a CUDA-event pair around
+    each call (on rotating weight copies, so every call reads HBM); median, p10 and p90 in us.
+    A call here is not overlapped with its neighbours, unlike the graph-replayed chain."""
+    import torch
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(calls)]
+    for r in range(min(cs.copies, 3)):
+        cs.launch(r, stream, variant)
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        cs.launch(i % cs.copies, stream, variant)
+        b.record(stream)
+    torch.cuda.synchronize()
+    us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
+    return {"median": round(float(np.median(us)), 3), "p10": round(float(np.percentile(us, 10)), 3),
+            "p90": round(float(np.percentile(us, 90)), 3), "calls": calls,
+            "how": "eager launches, a CUDA-event pair around each call on the launching stream"}
+
+
 def hbm_probe(device, nbytes=1 << 30, reps=10):
     """Copy (read+write) and read-only bandwidth of this library's probe kernels, best of reps."""
     import torch
@@ -744,6 +766,9 @@ def main(argv=None):
             del cst
             torch.cuda.empty_cache()
 
+    # per-call latency of isolated calls (not overlapped with their neighbours)
+    latency = time_latency(cs, 200, args.variant)
+
     # end to end through the Python API with host buffers
     e2e_steps = min(args.steps, 3000)
     s_e, h2d, d2h = time_e2e(cs, e2e_steps, min(args.warmup, 50), args.variant)
@@ -782,8 +807,10 @@ def main(argv=None):
                 "x ~ N(0,1) fp16)",
         "config": bench_config(world),
         "timing": {"l2": f"{cs_copies_note(HEADLINE, l2)}; L2 {l2 >> 20} MiB",
-                   "how": "CUDA graphs of one call per weight copy, CUDA events on the "
-                          "launching stream; B=8 on the same tensor in 'b8'"},
+                   "how": "one CUDA graph per measurement: lead calls, a start-event node on a "
+                          "side branch, exactly `steps` calls on rotating weight copies, an "
+                          "end-event node; B=8 on the same tensor in 'b8'"},
+        "latency_us": latency,
         "us_per_call": round(secs_max * 1e6 / args.steps, 3),
         "frac_of_hbm": round(value / world / hbm, 4),
         "variant": variant_used,
