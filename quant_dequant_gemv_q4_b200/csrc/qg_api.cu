@@ -9,6 +9,7 @@
 #include <map>
 #include <mutex>
 #include <set>
+#include <tuple>
 #include <utility>
 
 #include "../../include/qg.h"
@@ -30,6 +31,7 @@ struct DeviceInfo {
 
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_dev;
+constexpr size_t kCachePlans = 4096;  // bound of the launch-plan cache
 std::set<std::pair<int, const void *>> g_attr_set;
 
 thread_local int t_last_variant = 0;
@@ -394,6 +396,27 @@ RowsPlan make_umma_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     return best;  // smem == 0 if nothing fits
 }
 
+// The plan of a call (a pure function of the device's SM count and shared memory, the kernel
+// variant and the shape), cached: kind 0 = CUDA-core rows kernel, 1 = tensor-core kernel,
+// 2 = tcgen05 kernel.
+std::map<std::tuple<int, int, int, int, int64_t, int64_t, int, int>, RowsPlan> g_plans;
+
+RowsPlan plan_cached(int kind, int fmt, int64_t N, int64_t K, int B, const DeviceInfo &di, int mats = 1)
+{
+    const auto key = std::make_tuple(di.sms, di.smem_optin, kind, fmt, N, K, B, mats);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_plans.find(key);
+        if (it != g_plans.end()) return it->second;
+    }
+    const RowsPlan p = (kind == 2) ? make_umma_plan(fmt, N, K, B, di, mats)
+                                   : make_rows_plan(fmt, N, K, B, di, kind == 1, mats);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_plans.size() >= kCachePlans) g_plans.clear();
+    g_plans.emplace(key, p);
+    return p;
+}
+
 const void *umma_kernel_ptr(int fmt, int BP, int mats)
 {
 #define QG_UMMA_SWITCH(F, M)                                                              \
@@ -543,6 +566,33 @@ int make_weight_map(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *m
     return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
 }
 
+// Host work per call is part of a decode step's latency when calls are issued back to back, so
+// the two pure functions of a call's shape are cached: the tensor map of a weight tensor (it
+// encodes only the address, the format and the shape, so a map stays right for whatever tensor
+// later occupies the same address with the same shape) and the launch plan.  Both caches are
+// bounded: past kCacheMax entries they start over.
+constexpr size_t kCacheMax = 4096;
+std::map<std::tuple<const void *, int, int64_t, int64_t>, CUtensorMap> g_maps;
+
+int weight_map_cached(const void *W, int fmt, int64_t N, int64_t K, CUtensorMap *map)
+{
+    const auto key = std::make_tuple(W, fmt, N, K);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_maps.find(key);
+        if (it != g_maps.end()) {
+            *map = it->second;
+            return QG_OK;
+        }
+    }
+    const int rc = make_weight_map(W, fmt, N, K, map);
+    if (rc != QG_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_maps.size() >= kCacheMax) g_maps.clear();
+    g_maps.emplace(key, *map);
+    return QG_OK;
+}
+
 // Launch the row-band kernel (+ the split-K second pass when S > 1).  `err` is the device error
 // word; `part` holds S*N*B floats when S > 1.
 int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, int B, float *y,
@@ -561,8 +611,8 @@ int launch_rows(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x,
     // are 16-byte multiples, and a 144-byte box around each unit is a legal copy
     const bool per_lane = (fmt == kFmtQ6_K) || (fmt == kFmtIQ4_XS && (K / 256) % 2 != 0);
     if (!per_lane) {
-        if ((rc = make_weight_map(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
-        if (W2 && (rc = make_weight_map(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
+        if ((rc = weight_map_cached(W, fmt, N, K, &maps.m[0])) != QG_OK) return rc;
+        if (W2 && (rc = weight_map_cached(W2, fmt, N, K, &maps.m[1])) != QG_OK) return rc;
     }
     RowsArgs a;
     const int64_t wbytes = (int64_t)qg_weight_bytes(fmt, N, K);
@@ -699,8 +749,8 @@ int gemv_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x, i
     }
 
     if (var == QG_VARIANT_FACTORED || var == QG_VARIANT_TENSOR || var == QG_VARIANT_TCGEN05) {
-        const RowsPlan p = (var == QG_VARIANT_TCGEN05) ? make_umma_plan(fmt, N, K, B, di)
-                                                       : make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
+        const RowsPlan p = plan_cached(var == QG_VARIANT_TCGEN05 ? 2 : var == QG_VARIANT_TENSOR ? 1 : 0,
+                                       fmt, N, K, B, di);
         if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
         WsView ws;
         const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
@@ -786,7 +836,7 @@ int gate_up_impl(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K, 
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
-    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR, 2);
+    const RowsPlan p = plan_cached(var == QG_VARIANT_TENSOR ? 1 : 0, fmt, N, K, B, di, 2);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     WsView ws;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * 2 * (size_t)N * (size_t)B : 0;
@@ -818,7 +868,7 @@ int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
-    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
+    const RowsPlan p = plan_cached(var == QG_VARIANT_TENSOR ? 1 : 0, fmt, N, K, B, di);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     WsView ws;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
@@ -1187,7 +1237,7 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
         return rc;
     }
 
-    const RowsPlan p = make_rows_plan(fmt, N, K, B, di, var == QG_VARIANT_TENSOR);
+    const RowsPlan p = plan_cached(var == QG_VARIANT_TENSOR ? 1 : 0, fmt, N, K, B, di);
     if (p.smem == 0 || (size_t)di.smem_optin < p.smem) return QG_ERR_SHAPE;
     const size_t part_f = (p.S > 1) ? (size_t)p.S * (size_t)N * (size_t)B : 0;
     // one fixed layout for every call: the error word, kNoallocCounters band counters, then the
