@@ -267,10 +267,12 @@ int qg_hbm_read(const void *src, size_t bytes, uint32_t *out, void *stream);
  * variant); the kernel's scratch (an error word, one arrival counter per row band when K is
  * split, the split-K partial rows) lives in one file-scope device array of
  * QG_NOALLOC_SCRATCH_BYTES per GPU, which every GPU that loads the library holds until exit.
- *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library routine.  The counters
- *     start at zero (the array is zero-initialized) and every call leaves them at zero again (the
- *     last CTA of a band resets its counter); the partial rows are written before they are read.
- *     So nothing is cleared between calls.
+ *   - No device memory is allocated: no cudaMalloc/cudaFree, no allocating library routine.  The
+ *     counters start at zero (the array is zero-initialized) and every call leaves them at zero
+ *     again (the last CTA of a band resets its counter); the partial rows are written before they
+ *     are read.  So nothing is cleared between calls.  (On the host, the library's caches of
+ *     launch plans and weight tensor maps take a few hundred bytes of C++ heap the first time a
+ *     shape or a weight address is seen, shared with the other entry points.)
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current) and caches it; later calls reuse it.
  *   - Every call on every stream shares the one array: calls that overlap on the GPU race and give
