@@ -77,8 +77,8 @@ enum {
     QG_ERR_NULL = 1,    /* a required pointer is NULL */
     QG_ERR_FMT = 2,     /* unknown format flag */
     QG_ERR_SHAPE = 3,   /* N < 0, K < 1, or K not a multiple of the block size */
-    QG_ERR_BATCH = 4,   /* B outside 1..8 (1..16 for Q4_K, Q5_K, Q6_K with K % 256 == 0, and
-                           IQ4_XS with an even K / 256) */
+    QG_ERR_BATCH = 4,   /* B outside 1..8 (1..16 for Q4_K, Q5_K, Q6_K and Q8_0 with K % 256 == 0,
+                           and IQ4_XS with an even K / 256) */
     QG_ERR_ALIGN = 5,   /* W not 16-byte aligned, x not 2-byte aligned or y not 4-byte aligned */
     QG_ERR_CUDA = 6,    /* a CUDA runtime call failed (device query, launch, copy) */
     QG_ERR_NOMEM = 7,   /* the workspace could not be allocated */
@@ -89,7 +89,7 @@ enum {
 };
 
 /* Kernel variants of the GEMV (qg_gemv_variant).  QG_VARIANT_AUTO is what qg_gemv uses: when
- * K % 256 == 0, TENSOR with B >= 2 for Q4_K, Q5_K and IQ4_XS with an even K / 256, and with
+ * K % 256 == 0, TENSOR with B >= 2 for Q4_K, Q5_K, Q8_0 and IQ4_XS with an even K / 256, and with
  * B >= 3 for Q6_K, FACTORED otherwise; GENERIC when K % 256 != 0. */
 enum {
     QG_VARIANT_AUTO = 0,
@@ -112,13 +112,13 @@ enum {
      * are exact in fp32, so FACTORED's offset form (see below) and GENERIC differ only in their
      * summation. */
     QG_VARIANT_GENERIC = 3,
-    /* The K-quants (Q4_K, Q5_K, Q6_K) and IQ4_XS with an even K / 256: the FACTORED arithmetic
-     * with the code*x products on the tensor cores (mma.sync m16n8k16, f16 operands, fp32
-     * accumulation; the 8 columns of the instruction are the B columns of x), so B = 1..8 cost
-     * the same (up to 16 columns as two 8-column tiles).  The codes (IQ4_XS: the codebook levels)
-     * enter the MMA as exact normal fp16 numbers (or zero), so every product is exact.  Same error
-     * bound as FACTORED.  Requires K % 256 == 0; QG_ERR_VARIANT for Q8_0 and for IQ4_XS with an odd
-     * K / 256. */
+    /* The K-quants (Q4_K, Q5_K, Q6_K), Q8_0, and IQ4_XS with an even K / 256: the FACTORED
+     * arithmetic with the code*x products on the tensor cores (mma.sync m16n8k16, f16 operands,
+     * fp32 accumulation; the 8 columns of the instruction are the B columns of x), so B = 1..8
+     * cost the same (up to 16 columns as two 8-column tiles).  The codes (IQ4_XS: the codebook
+     * levels; Q8_0: the int8 values) enter the MMA as exact normal fp16 numbers (or zero), so every
+     * product is exact.  Same error bound as FACTORED (Q8_0: relative to sum |w*x|).  Requires
+     * K % 256 == 0; QG_ERR_VARIANT for IQ4_XS with an odd K / 256. */
     QG_VARIANT_TENSOR = 4,
     /* Q4_K and Q5_K: the FACTORED arithmetic with the q*x sums on the fifth-generation tensor
      * cores (tcgen05.mma kind::f16: the unpacked codes as the A operand in tensor memory, x as the
@@ -177,7 +177,7 @@ int qg_gemv_host(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *x
  *   x, B     as for qg_gemv; h: device, fp32 [N][B], 4-byte aligned, fully overwritten
  * The products and sums are those of qg_gemv's default kernels for (fmt, B); silu is evaluated in
  * fp32 with expf.  Errors as qg_gemv, plus QG_ERR_SHAPE when K % 256 != 0 (the fused path needs rows
- * of whole 256-weight units); B = 9..16 for Q4_K, Q5_K and IQ4_XS with an even K / 256 only
+ * of whole 256-weight units); B = 9..16 for Q4_K, Q5_K, Q8_0 and IQ4_XS with an even K / 256 only
  * (QG_ERR_BATCH otherwise). */
 int qg_gemv_gate_up_silu(const void *Wg, const void *Wu, int fmt, int64_t N, int64_t K,
                          const uint16_t *x, int B, float *h, void *stream);

@@ -263,6 +263,10 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
             LB = MmaFmt<kFmtQ6_K>::kUnitBytes;
             NW = MmaWarpsF<kFmtQ6_K, 1>::value;
             tab_floats = std::max(512, 32 * BP);
+        } else if (fmt == kFmtQ8_0) {
+            LB = MmaFmt<kFmtQ8_0>::kUnitBytes;
+            NW = BP >= 8 ? MmaWarpsF<kFmtQ8_0, 8>::value : MmaWarpsF<kFmtQ8_0, 1>::value;
+            tab_floats = std::max(256, 32 * BP);
         } else {
             LB = (fmt == kFmtQ5_K)     ? MmaFmt<kFmtQ5_K>::kUnitBytes
                  : (fmt == kFmtIQ4_XS) ? MmaFmt<kFmtIQ4_XS>::kUnitBytes
@@ -285,7 +289,8 @@ RowsPlan make_rows_plan(int fmt, int64_t N, int64_t K, int B, const DeviceInfo &
     // group, K part) pairs to keep every warp streaming).  Ties: fewer steps, then fewer slices.
     // The tensor-core kernel only takes slicings with at most one pair per warp.  If no slicing
     // qualifies, the one with the most busy lanes.
-    const int UB = tensor ? (fmt == kFmtQ5_K ? 176 : fmt == kFmtQ6_K ? 210 : fmt == kFmtIQ4_XS ? 136 : 144)
+    const int UB = tensor ? (fmt == kFmtQ5_K ? 176 : fmt == kFmtQ6_K ? 210 : fmt == kFmtIQ4_XS ? 136
+                             : fmt == kFmtQ8_0 ? 272 : 144)
                           : (fmt == kFmtQ6_K ? 210 : fmt == kFmtIQ4_XS ? 136 : LB);
     double best_cost = 1e300;
     int64_t best_steps = INT64_MAX;
@@ -461,6 +466,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #define QG_MMA6K2(bp) mma_gemv_kernel<bp, 2, kFmtQ6_K>
 #define QG_MMAIQ1(bp) mma_gemv_kernel<bp, 1, kFmtIQ4_XS>
 #define QG_MMAIQ2(bp) mma_gemv_kernel<bp, 2, kFmtIQ4_XS>
+#define QG_MMAQ81(bp) mma_gemv_kernel<bp, 1, kFmtQ8_0>
+#define QG_MMAQ82(bp) mma_gemv_kernel<bp, 2, kFmtQ8_0>
 #define QG_ROWS_Q4K1(bp) rows_gemv_kernel<kFmtQ4_K, bp, 1>
 #define QG_ROWS_Q4K2(bp) rows_gemv_kernel<kFmtQ4_K, bp, 2>
 #define QG_ROWS_Q801(bp) rows_gemv_kernel<kFmtQ8_0, bp, 1>
@@ -482,6 +489,10 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
     if (tensor && fmt == kFmtIQ4_XS) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMAIQ2) }
         QG_BP_SWITCH16(QG_MMAIQ1)
+    }
+    if (tensor && fmt == kFmtQ8_0) {
+        if (mats == 2) { QG_BP_SWITCH16(QG_MMAQ82) }
+        QG_BP_SWITCH16(QG_MMAQ81)
     }
     if (tensor) {
         if (mats == 2) { QG_BP_SWITCH16(QG_MMA2) }
@@ -515,6 +526,8 @@ const void *rows_kernel_ptr(int fmt, int BP, bool tensor, int mats)
 #undef QG_ROWS_Q801
 #undef QG_ROWS_Q4K2
 #undef QG_ROWS_Q4K1
+#undef QG_MMAQ82
+#undef QG_MMAQ81
 #undef QG_MMAIQ2
 #undef QG_MMAIQ1
 #undef QG_MMA6K2
@@ -680,12 +693,13 @@ int launch_rowwise(const void *W, int fmt, int64_t N, int64_t K, const uint16_t 
     return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
-// Formats with a tensor-core kernel: the K-quants, and IQ4_XS with an even number of units per row
-// (its rows are then 16-byte multiples, copied in tensor boxes).
+// Formats with a tensor-core kernel: the K-quants, IQ4_XS with an even number of units per row
+// (its rows are then 16-byte multiples, copied in tensor boxes), and Q8_0 with K % 256 == 0 (rows
+// of whole 8-block units).
 bool has_tensor_kernel(int fmt, int64_t K)
 {
     return fmt == QG_FMT_Q4_K || fmt == QG_FMT_Q5_K || fmt == QG_FMT_Q6_K ||
-           (fmt == QG_FMT_IQ4_XS && (K / 256) % 2 == 0);
+           (fmt == QG_FMT_IQ4_XS && (K / 256) % 2 == 0) || (fmt == QG_FMT_Q8_0 && K % 256 == 0);
 }
 
 // The variant qg_gemv takes: the tensor-core kernel where the format has one and B is past the

@@ -68,6 +68,11 @@ template <> struct MmaFmt<kFmtQ6_K> {  // rows arrive in 240-byte per-lane windo
 template <> struct MmaFmt<kFmtIQ4_XS> {
     static constexpr int kUnitBytes = 144, kQs = 8;
 };
+// Q8_0 with K % 256 == 0: a unit is 8 blocks of {fp16 d; i8 qs[32]}, 272 bytes (as in the
+// CUDA-core kernel); block b's qs start at byte 34 b + 2
+template <> struct MmaFmt<kFmtQ8_0> {
+    static constexpr int kUnitBytes = 272, kQs = 2;
+};
 
 // n-tiles of 8 columns per mma (16 columns: two, sharing the unpacked A fragment)
 template <int BP> struct MmaNT {
@@ -83,7 +88,9 @@ template <int FMT, int BP> struct MmaTabF {
     static constexpr int value = (FMT == kFmtQ6_K && MmaTab<BP>::value < 512) ? 512 : MmaTab<BP>::value;
 };
 template <int FMT, int BP> struct MmaWarpsF {
-    static constexpr int value = (FMT == kFmtQ6_K) ? 8 : MmaWarps<BP>::value;
+    // Q8_0: 272-byte units make each warp's ring twice Q4_K's, so fewer warps fit next to x
+    static constexpr int value = (FMT == kFmtQ6_K) ? 8 : (FMT == kFmtQ8_0) ? (BP >= 8 ? 6 : 8)
+                                                                          : MmaWarps<BP>::value;
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -170,10 +177,14 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
         const int lh = (gi >> 3) & 1, c = (gi >> 4) & 3, j = gi >> 6;
         return (FMT == kFmtQ6_K) ? j * 256 + 128 * (c >> 1) + 32 * (c & 1) + 64 * lh + 16 * h + 4 * t
                : (FMT == kFmtIQ4_XS) ? j * 256 + 32 * (2 * c + h) + 4 * t + 2 * lh
+               : (FMT == kFmtQ8_0)   ? j * 256 + 32 * (2 * c + lh) + 16 * h + 4 * t
                                      : j * 256 + 64 * c + 32 * lh + 8 * t + 4 * h;
     };
-    // x row r (0..3) of a group: e + r, or for IQ4_XS e + (r & 1) + 16 (r >> 1)
-    auto row_off = [](int r) { return (FMT == kFmtIQ4_XS) ? (r & 1) + 16 * (r >> 1) : r; };
+    // x row r (0..3) of a group: e + r; IQ4_XS e + (r & 1) + 16 (r >> 1); Q8_0 e, e+2, e+1, e+3
+    // (its fragment registers pair consecutive weights)
+    auto row_off = [](int r) {
+        return (FMT == kFmtIQ4_XS) ? (r & 1) + 16 * (r >> 1) : (FMT == kFmtQ8_0) ? ((r & 1) << 1) | (r >> 1) : r;
+    };
     for (int g0 = threadIdx.x; g0 < ngroups; g0 += NB * blockDim.x) {
         uint32_t rw[NB][4][W];  // raw x rows: [group][row][word], zero when absent
 #pragma unroll
@@ -189,13 +200,17 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
                 const uint16_t *src = xsl + (int64_t)e * B;
                 const uintptr_t addr = reinterpret_cast<uintptr_t>(src);
                 if (FMT != kFmtIQ4_XS && B == BP && BP >= 2 && (addr & 15) == 0) {
-                    // 4 rows x BP halves = 2 BP words, contiguous: BP / 2 16-byte loads
+                    // 4 rows x BP halves = 2 BP words, contiguous: BP / 2 16-byte loads (Q8_0: the
+                    // rows' slots in the order e, e+2, e+1, e+3)
 #pragma unroll
                     for (int q = 0; q < BP / 2; ++q) {
                         const uint4 v = reinterpret_cast<const uint4 *>(src)[q];
                         const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) rw[u][(4 * q + k) / W][(4 * q + k) % W] = vv[k];
+                        for (int k = 0; k < 4; ++k) {
+                            const int r = (4 * q + k) / W;
+                            rw[u][(FMT == kFmtQ8_0) ? row_off(r) : r][(4 * q + k) % W] = vv[k];
+                        }
                     }
                 } else if (FMT == kFmtIQ4_XS && B == BP && BP >= 4 && (addr & 15) == 0) {
                     // two runs of 2 rows (e, e + 1 and e + 16, e + 17): BP / 4 16-byte loads each
@@ -216,7 +231,7 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
                         rw[u][2 * run][0] = v.x;
                         rw[u][2 * run + 1][0] = v.y;
                     }
-                } else if (FMT != kFmtIQ4_XS && B == 1 && BP == 1 && (addr & 7) == 0) {
+                } else if (FMT != kFmtIQ4_XS && FMT != kFmtQ8_0 && B == 1 && BP == 1 && (addr & 7) == 0) {
                     const uint2 v = *reinterpret_cast<const uint2 *>(src);
                     rw[u][0][0] = v.x & 0xFFFFu; rw[u][1][0] = v.x >> 16;
                     rw[u][2][0] = v.y & 0xFFFFu; rw[u][3][0] = v.y >> 16;
@@ -236,7 +251,7 @@ __device__ __forceinline__ void mma_stage_x(const RowsArgs &a, int s, int US_s, 
             if (gi >= ngroups) break;  // uniform across the warp (ngroups and blockDim: multiples of 32)
             const int th = gi & 7, t = th >> 1, h = th & 1;
             const int lh = (gi >> 3) & 1, c = (gi >> 4) & 3, j = gi >> 6;
-            if (FMT != kFmtIQ4_XS) {
+            if (FMT != kFmtIQ4_XS && FMT != kFmtQ8_0) {  // (neither has an offset or a min)
                 // column sums of the 4 rows in fp32: (x0 + x1) + (x2 + x3)
                 float sc[BP];
 #pragma unroll
@@ -707,6 +722,101 @@ __device__ __forceinline__ void mma_iq4xs_step(const uint8_t *u0, int o, const u
     }
 }
 
+// One Q8_0 step: 32 rows (two 16-row tiles) x one 272-byte unit (8 blocks of 32 weights) at u0.
+// k-tile (block 2c + lh, half h) of a row holds qs bytes 16h .. 16h+15 of the block; thread (g, t)
+// takes the 4 bytes 16h + 4t .. +3 (weights e .. e+3, e = 32 (2c + lh) + 16h + 4t) of rows g and
+// g + 8: one 32-bit load (odd blocks start 4-byte aligned; even ones 2 bytes past, read as a funnel
+// shift of two words), an XOR with 0x80 per byte (q + 128, as unsigned bytes), one byte permute per
+// register under the exponent of 1024 (the fp16 pair 1024 + q + 128) and one f16x2 add of -1152:
+// the int8 codes as exact fp16 integers.  A register pairs consecutive weights (e, e+1) or
+// (e+2, e+3); x is staged in that order.  Both k-tiles of a block sum into one C fragment, scaled by
+// the block's d of its row (dtab: [8 blocks][32 positions]).
+template <int BP>
+__device__ __forceinline__ void mma_q8_step(const uint8_t *u0, const uint2 *xf, int j, float *dtab,
+                                            float (&acc)[2][MmaNT<BP>::value][4], int lane)
+{
+    constexpr int FMT = kFmtQ8_0;
+    constexpr int LB = MmaFmt<FMT>::kUnitBytes;
+    constexpr int NT = MmaNT<BP>::value;
+    const int g = lane >> 2, t = lane & 3;
+    const int pr = mma_frag_row<FMT>(g);
+    {
+        // the 8 block scales of row `lane`
+        const uint8_t *row = u0 + lane * LB;
+        const int pos = (lane & 7) * 4 + (lane >> 3);
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+            dtab[b * 32 + pos] = __half2float(*reinterpret_cast<const __half *>(row + 34 * b));
+    }
+    __syncwarp();
+    auto code_word = [&](const uint8_t *row, int blk, int h) {
+        const int off = 34 * blk + MmaFmt<FMT>::kQs + 16 * h + 4 * t;  // 4-byte aligned iff blk odd
+        uint32_t w;
+        if (blk & 1) {
+            w = *reinterpret_cast<const uint32_t *>(row + off);
+        } else {
+            const uint32_t *p = reinterpret_cast<const uint32_t *>(row + off - 2);
+            w = __funnelshift_r(p[0], p[1], 16);
+        }
+        return w ^ 0x80808080u;  // q + 128 per byte
+    };
+    auto codes = [](uint32_t v, uint32_t sel) {  // sel 0x4140: bytes 0, 1; 0x4342: bytes 2, 3
+        const uint32_t p = __byte_perm(v, 0x64646464u, sel);  // (1024 + q + 128, ...)
+        uint32_t r;
+        asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(p), "r"(0xE480E480u));  // - (1152, 1152)
+        return r;
+    };
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint2 xb[NT][2][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = (BP > 8) ? 8 * nt + g : g % BP;
+                    xb[nt][lh][h] = xf[mma_xf_idx(j, c, lh, h, col ^ mma_xf_swz(c, lh, h, BP), t, BP)];
+                }
+        const float4 D0 = *reinterpret_cast<const float4 *>(dtab + (2 * c) * 32 + 4 * pr);
+        const float4 D1 = *reinterpret_cast<const float4 *>(dtab + (2 * c + 1) * 32 + 4 * pr);
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            const uint8_t *rowA = u0 + (tile * 16 + pr) * LB;
+            const uint8_t *rowB = rowA + 8 * LB;
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh) {
+                const int blk = 2 * c + lh;
+                float cs[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) cs[nt][k] = 0.0f;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t vA = code_word(rowA, blk, h), vB = code_word(rowB, blk, h);
+                    const uint32_t a0 = codes(vA, 0x4140u), a1 = codes(vB, 0x4140u);
+                    const uint32_t a2 = codes(vA, 0x4342u), a3 = codes(vB, 0x4342u);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816(cs[nt], a0, a1, a2, a3, xb[nt][lh][h].x, xb[nt][lh][h].y);
+                }
+                const float4 D = lh ? D1 : D0;
+                const float da = tile ? D.z : D.x, db = tile ? D.w : D.y;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    acc[tile][nt][0] = fmaf(da, cs[nt][0], acc[tile][nt][0]);
+                    acc[tile][nt][2] = fmaf(db, cs[nt][2], acc[tile][nt][2]);
+                    if (BP > 1) {
+                        acc[tile][nt][1] = fmaf(da, cs[nt][1], acc[tile][nt][1]);
+                        acc[tile][nt][3] = fmaf(db, cs[nt][3], acc[tile][nt][3]);
+                    }
+                }
+            }
+        }
+    }
+}
+
 // One Q6_K step: 32 rows x one superblock from the warp's per-lane windows at u0 (window of row
 // r at u0 + 240 r; its superblock starts o_r = (m_r * 210) mod 16 bytes in, m_r its superblock
 // index in the tensor).  Chunk c = 2hf + p is ql[64hf + 32p ..]; its k-tile kk (words 4kk .. 4kk+3)
@@ -987,7 +1097,9 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
                 mma_q6k_step<BP>(myring + (step % kRowsStages) * BOX, xf, xsum, a.US, j, dtab, acc, accM,
                                  lane, a, row0, ucol0 + j, a.w[second ? MATS - 1 : 0]);
             } else {
-                if (FMT == kFmtIQ4_XS)
+                if (FMT == kFmtQ8_0)
+                    mma_q8_step<BP>(myring + (step % kRowsStages) * BOX, xf, j, dtab, acc, lane);
+                else if (FMT == kFmtIQ4_XS)
                     mma_iq4xs_step<BP>(myring + (step % kRowsStages) * BOX, (int)(((int64_t)(ucol0 + j) * UB) & 15),
                                        xf, j, dtab, acc, lane);
                 else if (FMT == kFmtQ5_K)

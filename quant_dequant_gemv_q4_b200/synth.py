@@ -222,5 +222,10 @@ WORKLOADS = {
         Gemv("ffn_gate_b2", IQ4_XS, 17408, 5120, 2, 0, 1e-3),
         Gemv("ffn_gate_b8", IQ4_XS, 17408, 5120, 8, 1, 1e-3),
         Gemv("ffn_gate_b16", IQ4_XS, 17408, 5120, 16, 2, 1e-3))),
+    # the Q8_0 attention projection on the batched-verify widths (tensor cores at B >= 2)
+    "q8_0_attn_q_verify": Workload("q8_0_attn_q_verify", 11, (
+        Gemv("attn_q_b2", Q8_0, 12288, 5120, 2, 0),
+        Gemv("attn_q_b8", Q8_0, 12288, 5120, 8, 1),
+        Gemv("attn_q_b16", Q8_0, 12288, 5120, 16, 2))),
 }
 FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q6_K: "Q6_K", Q8_0: "Q8_0", IQ4_XS: "IQ4_XS"}

@@ -227,7 +227,7 @@ def test_variant_checks(L):
     assert L.qg_gemv_variant(FAKE, 13, 4, 256, FAKE, 17, FAKE, None, qg.QG_VARIANT_TCGEN05) == qg.QG_ERR_BATCH
     # the tensor-core variant takes the K-quants, and IQ4_XS with an even K / 256 (rows of 16-byte
     # multiples); every streaming variant needs K % 256 == 0
-    assert L.qg_gemv_variant(FAKE, 8, 4, 256, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
+    assert L.qg_gemv_variant(FAKE, 8, 4, 96, FAKE, 1, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
     assert L.qg_gemv_variant(FAKE, 23, 4, 768, FAKE, 2, FAKE, None, qg.QG_VARIANT_TENSOR) == qg.QG_ERR_VARIANT
     for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_TENSOR):
         assert L.qg_gemv_variant(FAKE, 8, 4, 96, FAKE, 1, FAKE, None, v) == qg.QG_ERR_VARIANT
@@ -237,11 +237,14 @@ def test_variant_checks(L):
         for v in (qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC):
             assert L.qg_gemv_variant(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
         assert L.qg_gemv(FAKE, fmt, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
-    # Q8_0, and IQ4_XS with an odd K / 256: 1..8 columns; IQ4_XS with an even K / 256 takes 9..16
-    # on the tensor-core kernel only
+    # Q8_0 with K % 256 != 0 and IQ4_XS with an odd K / 256: 1..8 columns; otherwise 9..16 on the
+    # tensor-core kernel only
+    assert L.qg_gemv(FAKE, 8, 4, 96, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv(FAKE, 23, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
     for fmt in (8, 23):
-        assert L.qg_gemv(FAKE, fmt, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH
         assert L.qg_gemv(FAKE, fmt, 4, 300, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
+        for v in (qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC):
+            assert L.qg_gemv_variant(FAKE, fmt, 4, 512, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
     for v in (qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC):
         assert L.qg_gemv_variant(FAKE, 23, 4, 512, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
     assert L.qg_gemv(FAKE, 23, 4, 512, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
@@ -292,15 +295,16 @@ def test_residual_rejects_bad_arguments(L):
 
 
 def test_batch_width_limits(L):
-    # 1..8 everywhere; 9..16 only on the tensor-core kernel (Q4_K, K % 256 == 0)
+    # 1..8 everywhere; 9..16 only on the tensor-core kernel (rows of whole 256-weight units;
+    # IQ4_XS: an even K / 256).  Every call here is refused on the host (the pointers are fake).
     assert L.qg_gemv(FAKE, 12, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
-    assert L.qg_gemv(FAKE, 8, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # Q8_0
+    assert L.qg_gemv(FAKE, 8, 4, 96, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # Q8_0, K % 256 != 0
     for v in (qg.QG_VARIANT_DIRECT, qg.QG_VARIANT_FACTORED, qg.QG_VARIANT_GENERIC):
         assert L.qg_gemv_variant(FAKE, 12, 4, 256, FAKE, 9, FAKE, None, v) == qg.QG_ERR_BATCH
-    assert L.qg_gemv_noalloc(FAKE, 8, 4, 256, FAKE, 16, FAKE, None) == qg.QG_ERR_BATCH
-    assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 8, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_noalloc(FAKE, 8, 4, 96, FAKE, 16, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 23, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
     assert L.qg_gemv_gate_up_silu(FAKE, FAKE, 14, 4, 256, FAKE, 12, FAKE, None) == qg.QG_ERR_BATCH
-    assert L.qg_gemv_residual(FAKE, 8, 4, 256, FAKE, 12, FAKE, FAKE, None) == qg.QG_ERR_BATCH
+    assert L.qg_gemv_residual(FAKE, 23, 4, 256, FAKE, 12, FAKE, FAKE, None) == qg.QG_ERR_BATCH
 
 
 def test_gemv_host_rejects_bad_arguments(L):
@@ -309,7 +313,7 @@ def test_gemv_host_rejects_bad_arguments(L):
     assert f(FAKE, 99, 4, 256, FAKE, 1, FAKE, None) == qg.QG_ERR_FMT
     assert f(FAKE, 12, 4, 300, FAKE, 1, FAKE, None) == qg.QG_ERR_SHAPE
     assert f(FAKE, 12, 4, 256, FAKE, 0, FAKE, None) == qg.QG_ERR_BATCH
-    assert f(FAKE, 8, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # 9..16: tensor-core formats only
+    assert f(FAKE, 8, 4, 96, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH   # 9..16: tensor-core formats only
     assert f(FAKE, 23, 4, 256, FAKE, 9, FAKE, None) == qg.QG_ERR_BATCH  # IQ4_XS, odd K / 256
     assert f(FAKE, 23, 4, 512, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH
     assert f(FAKE, 14, 4, 256, FAKE, 17, FAKE, None) == qg.QG_ERR_BATCH

@@ -121,15 +121,49 @@ def test_q4k_gemv_small(dev, orc, variant, N, K, B):
     assert_within(y, yref, A, f"q4k v{variant} N={N} K={K} B={B}")
 
 
-@pytest.mark.parametrize("variant", [0, 3])
+@pytest.mark.parametrize("variant", [0, 2, 3, 4])
 @pytest.mark.parametrize("N,K", [(1, 256), (5, 5120), (77, 1024), (3, 96), (40, 800), (9, 32)])
 @pytest.mark.parametrize("B", [1, 2, 4, 7, 8])
 def test_q8_0_gemv_small(dev, orc, variant, N, K, B):
+    """Q8_0 on every variant it takes: the CUDA-core and tensor-core streaming kernels need
+    K % 256 == 0 (whole 8-block units); the per-row kernel takes any K."""
+    import quant_dequant_gemv_q4_b200 as qg
     W = synth.q8_0_weights(N, K, seed=N * 5 + K)
     x = synth.activations(K, B, seed=B + 10)
+    if variant in (2, 4) and K % 256 != 0:
+        with pytest.raises(qg.QgError) as e:
+            gpu_gemv(dev, W, Q8_0, N, K, x, variant)
+        assert e.value.status == qg.QG_ERR_VARIANT
+        return
     y = gpu_gemv(dev, W, Q8_0, N, K, x, variant)
     yref, A = orc.gemv(W, Q8_0, N, K, x, B)
     assert_within(y, yref, A, f"q8_0 v{variant} N={N} K={K} B={B}")
+
+
+@pytest.mark.parametrize("N,K", [(1, 256), (5, 5120), (77, 1024), (300, 2560)])
+@pytest.mark.parametrize("B", [9, 12, 16])
+def test_q8_0_gemv_wide(dev, orc, N, K, B):
+    """Q8_0 at B = 9..16 on the tensor-core kernel (two 8-column n-tiles)."""
+    import quant_dequant_gemv_q4_b200 as qg
+    W = synth.q8_0_weights(N, K, seed=N + K + B)
+    x = synth.activations(K, B, seed=B + 11, massive_frac=1e-3)
+    y = gpu_gemv(dev, W, Q8_0, N, K, x, 0)
+    assert qg.qg_last_variant() == qg.QG_VARIANT_TENSOR
+    yref, A = orc.gemv(W, Q8_0, N, K, x, B)
+    assert_within(y, yref, A, f"q8_0 N={N} K={K} B={B}")
+
+
+@pytest.mark.parametrize("N,K,B", [(12288, 5120, 2), (12288, 5120, 8), (12288, 5120, 16), (5120, 17408, 4)])
+def test_q8_0_tensor_full_size_sampled(dev, orc, N, K, B):
+    W = synth.q8_0_weights(N, K, seed=N + B)
+    x = synth.activations(K, B, seed=B + 12, massive_frac=1e-3)
+    y = gpu_gemv(dev, W, Q8_0, N, K, x, 4)
+    assert np.isfinite(y).all()
+    rows = _sample_rows(N, np.random.default_rng(B + 8), k=160)
+    yref, A = orc.gemv(W, Q8_0, N, K, x, B, rows=rows)
+    assert_within(y[rows], yref, A, f"q8_0 {N}x{K} B={B}")
+    y2 = gpu_gemv(dev, W, Q8_0, N, K, x, 4)
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32)), "not deterministic"
 
 
 @pytest.mark.parametrize("fmt,variant,N,K,B", [
@@ -140,6 +174,8 @@ def test_q8_0_gemv_small(dev, orc, variant, N, K, B):
     (Q4_K, 4, 96, 17408, 8),
     (Q4_K, 4, 17, 65536, 2),
     (Q8_0, 0, 64, 17408, 8),
+    (Q8_0, 2, 64, 17408, 8),
+    (Q8_0, 4, 40, 65536, 3),
 ])
 def test_split_k(dev, orc, fmt, variant, N, K, B):
     import quant_dequant_gemv_q4_b200 as qg
@@ -175,7 +211,7 @@ def test_q8_0_exact_integer_case(dev, orc):
     W = W.reshape(-1)
     x = rng.integers(-16, 17, size=(K, B)).astype(np.float16)
     yref, _ = orc.gemv(W, Q8_0, N, K, x, B)
-    for variant in (0, 3):
+    for variant in (0, 2, 3, 4):
         y = gpu_gemv(dev, W, Q8_0, N, K, x, variant)
         assert np.array_equal(y.astype(np.float64), yref), variant
 
@@ -359,10 +395,17 @@ def test_wide_b_rejected_off_the_tensor_kernel(dev):
         with pytest.raises(qg.QgError) as e:
             gpu_gemv(dev, W, Q4_K, 8, 256, x, v)
         assert e.value.status == qg.QG_ERR_BATCH
-    Wq = synth.q8_0_weights(8, 256, seed=1)
+    # Q8_0: 9..16 columns on the tensor-core kernel, which needs K % 256 == 0
+    Wq = synth.q8_0_weights(8, 96, seed=1)
+    x96 = synth.activations(96, 9, seed=1)
     with pytest.raises(qg.QgError) as e:
-        gpu_gemv(dev, Wq, Q8_0, 8, 256, x, 0)
+        gpu_gemv(dev, Wq, Q8_0, 8, 96, x96, 0)
     assert e.value.status == qg.QG_ERR_BATCH
+    Wq = synth.q8_0_weights(8, 256, seed=1)
+    for v in (2, 3):
+        with pytest.raises(qg.QgError) as e:
+            gpu_gemv(dev, Wq, Q8_0, 8, 256, x, v)
+        assert e.value.status == qg.QG_ERR_BATCH
 
 
 def test_verify_width_16_full_size_sampled(dev, orc):

@@ -76,7 +76,7 @@ def test_plan_invariants(sms, smem, fmt):
                 except qg.QgError as e:
                     # B > 8 is the tensor-core kernels' only (not the Q6_K pair's, and IQ4_XS's
                     # with an even K / 256); a small device may fit no plan
-                    wide_ok = fmt in (Q4_K, Q5_K) or (fmt == Q6_K and mats == 1) or \
+                    wide_ok = fmt in (Q4_K, Q5_K, Q8_0) or (fmt == Q6_K and mats == 1) or \
                         (fmt == IQ4_XS and UPR % 2 == 0)
                     assert (B > 8 and not wide_ok and e.status == qg.QG_ERR_BATCH) or \
                         e.status == qg.QG_ERR_SHAPE, (N, K, B, mats, e)
@@ -87,7 +87,7 @@ def test_plan_invariants(sms, smem, fmt):
                 assert S * US >= UPR > (S - 1) * US
                 assert 1 <= p["ctas"] <= sms
                 assert p["warps"] in (6, 8, 12, 16)
-                has_tc = fmt in (Q4_K, Q5_K, Q6_K) or (fmt == IQ4_XS and UPR % 2 == 0)
+                has_tc = fmt in (Q4_K, Q5_K, Q6_K, Q8_0) or (fmt == IQ4_XS and UPR % 2 == 0)
                 tc_min = 3 if fmt == Q6_K else 2  # Q6_K's CUDA-core kernel still wins at B = 2
                 assert p["variant"] == (TENSOR if has_tc and B >= tc_min else FACTORED)
     assert n > 0
@@ -113,10 +113,10 @@ def test_generic_and_direct_plans():
     ((Q4_K, 0, 5120, 1, 0, 1), qg.QG_ERR_SHAPE),
     ((Q4_K, 100, 5120, 0, 0, 1), qg.QG_ERR_BATCH),
     ((Q4_K, 100, 5120, 17, 0, 1), qg.QG_ERR_BATCH),
-    ((Q8_0, 100, 5120, 9, 0, 1), qg.QG_ERR_BATCH),
+    ((Q8_0, 100, 5152, 9, 0, 1), qg.QG_ERR_BATCH),   # K % 256 != 0: no tensor-core kernel
     ((Q4_K, 100, 5120, 9, FACTORED, 1), qg.QG_ERR_BATCH),
     ((Q4_K, 100, 5120, 1, 9, 1), qg.QG_ERR_VARIANT),
-    ((Q8_0, 100, 5120, 2, TENSOR, 1), qg.QG_ERR_VARIANT),
+    ((Q8_0, 100, 5152, 2, TENSOR, 1), qg.QG_ERR_VARIANT),
     ((Q8_0, 100, 5152, 1, FACTORED, 1), qg.QG_ERR_VARIANT),
     ((Q5_K, 100, 5120, 1, DIRECT, 1), qg.QG_ERR_VARIANT),
     ((Q4_K, 100, 5120, 1, FACTORED, 2), qg.QG_ERR_VARIANT),
