@@ -878,7 +878,7 @@ int residual_impl(const void *W, int fmt, int64_t N, int64_t K, const uint16_t *
         return QG_ERR_ALIGN;
     if (K % 256 != 0) return QG_ERR_SHAPE;  // rows of whole 256-weight units only
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16: the K-quants' tensor-core kernel
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16: the tensor-core kernel only
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;
@@ -1237,7 +1237,7 @@ extern "C" int qg_gemv_noalloc(const void *W, int fmt, int64_t N, int64_t K, con
     if (reinterpret_cast<uintptr_t>(x) % 2 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0)
         return QG_ERR_ALIGN;
     const int var = auto_variant(fmt, K, B);
-    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16: the K-quants' tensor-core kernel
+    if (B > 8 && var != QG_VARIANT_TENSOR) return QG_ERR_BATCH;  // 9..16: the tensor-core kernel only
     DeviceInfo di;
     int dev = 0;
     if ((rc = device_info(&di, &dev)) != QG_OK) return rc;

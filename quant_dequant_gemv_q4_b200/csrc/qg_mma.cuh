@@ -1,5 +1,5 @@
 // qg_mma.cuh -- the tensor-core streaming GEMV of libqg (sm_100a) for the K-quants (Q4_K, Q5_K,
-// Q6_K), B = 1..8 columns (Q4_K: up to 16).
+// Q6_K), Q8_0 and IQ4_XS, B = 1..16 columns (two 8-column n-tiles past 8).
 //
 // Operation (HARDWARE GROUND TRUTH: 2x NVIDIA Tesla T4 (Kaggle), second prompt, "SPEC"):
 //   y[n,b] = sum_k dequant(W)[n,k] * x[k,b], fp32 accumulation ("PHYSICS & CONTRACT"), Q4_K
@@ -7,11 +7,12 @@
 //
 // Why tensor cores here.  With B columns, the CUDA-core kernel spends one fp32 FMA per weight and
 // column, so at B = 8 the FMA pipe, not HBM, bounds it.  mma.sync.m16n8k16 (f16 x f16 -> f32)
-// multiplies a 16-row x 16-weight tile of 4-bit integers by a 16 x 8 tile of x in one
+// multiplies a 16-row x 16-weight tile of integer codes by a 16 x 8 tile of x in one
 // instruction: the 8 columns of the instruction are the B <= 8 columns of x, so B = 1..8 cost the
 // same tensor work, and the weights are unpacked once for all columns.  Products are exact
-// (integers up to 15 times fp16 x) and the sums are fp32, so the arithmetic is the factored form
-// of the CUDA-core kernel:
+// (small integers, or integers times a power of two, times fp16 x) and the sums are fp32, so the
+// arithmetic is the factored form of the CUDA-core kernel (Q4_K / Q5_K shown; Q6_K, Q8_0 and
+// IQ4_XS have their own scales and no min, see their step functions):
 //   sum_i w_i x_i = d * sum_j sc_j sum_{i in j} q_i x_i  -  sum_j M_j * sum_{i in j} x_i,
 //   M_j = dmin*m_j (exact in fp32), j = 32-weight sub-block.
 //
