@@ -770,12 +770,13 @@ def main(argv=None):
     latency = time_latency(cs, 200, args.variant)
 
     # end to end through the Python API with host buffers
-    e2e_steps = min(args.steps, 3000)
-    s_e, h2d, d2h = time_e2e(cs, e2e_steps, min(args.warmup, 50), args.variant)
+    # (at least 500 steps after 20 warm-up steps, so a short --steps still reads the steady state)
+    e2e_steps = max(min(args.steps, 3000), 500)
+    s_e, h2d, d2h = time_e2e(cs, e2e_steps, max(min(args.warmup, 50), 20), args.variant)
     s_e = dist_max(s_e, device)
     e2e = {"value": round(cs.bytes_per_step * e2e_steps * world / s_e / 1e9, 2), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "us_per_step": round(s_e * 1e6 / e2e_steps, 2),
+           "us_per_step": round(s_e * 1e6 / e2e_steps, 2), "steps": e2e_steps,
            "via": "qg_gemv_host through the C ABI: pinned host x and y, the copies and the call on "
                   "one stream, one call per step, host clock around all steps"}
     probe = hbm_probe(device)
