@@ -131,3 +131,16 @@ def test_argument_errors(args, status):
 
 def test_null_out():
     assert qg.lib().qg_plan(Q4_K, 100, 5120, 1, 0, 1, 148, 232448, None) == qg.QG_ERR_NULL
+
+
+@pytest.mark.parametrize("wl", sorted(synth.WORKLOADS))
+def test_every_workload_call_has_a_plan(wl):
+    """Every call of the synthetic workloads (the parity configurations and the bench table) plans
+    on a B200 with the default variant, and the variant is the one the default rule names."""
+    for c in synth.WORKLOADS[wl].calls:
+        p = qg.qg_plan(c.fmt, c.N, c.K, c.B, **B200)
+        assert p["smem"] <= B200["smem_optin"] and 1 <= p["ctas"] <= B200["sms"]
+        UPR = c.K // 256
+        has_tc = c.fmt in (Q4_K, Q5_K, Q6_K, Q8_0) or (c.fmt == IQ4_XS and UPR % 2 == 0)
+        tc_min = 3 if c.fmt == Q6_K else 2
+        assert p["variant"] == (TENSOR if has_tc and c.B >= tc_min else FACTORED), (wl, c.name)
