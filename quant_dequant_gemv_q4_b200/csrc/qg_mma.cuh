@@ -52,7 +52,7 @@ template <int BP> struct MmaWarps {
 };
 
 // Formats of the tensor-core kernel: Q4_K, Q5_K (the Q4_K superblock with a fifth-bit plane
-// qh[32] before qs) and Q6_K.  kQs: offset of qs in the superblock.
+// qh[32] before qs), Q6_K, and below IQ4_XS and Q8_0.  kQs: offset of qs in the superblock.
 template <int FMT> struct MmaFmt;
 template <> struct MmaFmt<kFmtQ4_K> {
     static constexpr int kUnitBytes = 144, kQs = 16;
@@ -1056,7 +1056,9 @@ __global__ void __launch_bounds__(MmaWarpsF<FMT, BP>::value * 32, 1)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // 3. x fragments and sub-block sums of this slice
     mma_stage_x<BP, FMT>(a, s, US_s, xf, xsum);
-    // the rest of the ring, once this warp's x loads have returned (as in rows_gemv_kernel)
+    // the rest of the ring, once this warp's x loads have returned (issuing it after the CTA's
+    // barrier instead, as rows_gemv_kernel does, measured no better here: B = 8 unchanged,
+    // Q5_K at B = 16 0.7 us slower)
     if (PER_LANE) {
         for (int i = kPreStages; i < kRowsStages && i < nsteps; ++i) issue_lanes(i);
     } else if (lane == 0) {

@@ -92,11 +92,18 @@ template <int FMT, int BP> struct RowsWarps {
 };
 
 constexpr int kRowsStages = 2;  // ring stages per warp (double buffering)
-// Ring stages issued before the wait for the previous kernel; the rest are issued once this
-// warp's x has arrived.  A deeper prefetch at entry queues more weight data on the SM's return
-// path ahead of x, and x then arrives later (measured: 1 of 2 stages early is 0.6-0.9 us faster
-// per call than 2 of 2, and than any order that issues the second stage before x is in).
+// Ring stages issued before the wait for the previous kernel; the rest are issued once the whole
+// CTA's x is staged (after the barrier), or, for Q8_0, once this warp's own x has arrived.  A
+// deeper prefetch at entry queues more weight data on the SM's return path ahead of x, and x then
+// arrives later (measured: 1 of 2 stages early is 0.6-0.9 us faster per call than 2 of 2, and
+// than any order that issues the second stage before x is in).  Refills issued by the warps whose
+// x came in first likewise delay the x of the others: waiting for the barrier saves 0.3-0.45 us
+// per call on the Q4_K, Q5_K and IQ4_XS FFN and attention shapes, while Q8_0 (272-byte units)
+// measured 0.2 us faster with each warp refilling as soon as its own x is in.
 constexpr int kPreStages = 1;
+template <int FMT> struct RowsRefillAfterBarrier {
+    static constexpr bool value = FMT != kFmtQ8_0;
+};
 
 struct RowsArgs {
     const uint16_t *x;  // fp16 bits [K][B]
@@ -881,14 +888,17 @@ __global__ void __launch_bounds__(RowsWarps<FMT, BP>::value * 32, 1)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // 3. x for this slice -> shared memory (fp16 in consumer order) and per-sub-block sums,
-    //    then the rest of the ring (this warp's x loads have returned by now)
+    //    then the rest of the ring: after the CTA's barrier, or (Q8_0) as soon as this warp's own
+    //    x loads have returned
+    constexpr bool REFILL_LATE = RowsRefillAfterBarrier<FMT>::value;
     rows_stage_x<BP, FMT>(a, s, US_s, xs, xsum);
+    if (REFILL_LATE) __syncthreads();
     if (lane_copy) {
         for (int i = kPreStages; i < NS && i < nsteps; ++i) issue_lanes();
     } else if (lane == 0) {
         for (int i = kPreStages; i < NS && i < nsteps; ++i) issue();
     }
-    __syncthreads();
+    if (!REFILL_LATE) __syncthreads();
 
     int step = 0, cslot = 0;
     uint32_t cphase = 0;  // consumer: ring slot and its phase parity
